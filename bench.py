@@ -1,0 +1,348 @@
+"""Benchmark: Echo 4-bit error-compensated all-reduce, simulated over P = 8
+virtual ranks on one B200, on the 1 GB-per-rank message (131072 x 4096 bf16,
+Student-t nu=3 values scaled to unit variance, groups of 128, INT4, feedback
+on: alpha_long 0.05, alpha_short 0.5, w 0.5, eta 1).
+
+One step = one full call (the three kernels: non-owner quantize with fused
+feedback, owner reduce/requantize, gather dequantize), inputs resident in HBM.
+Metric: GB/s of bf16 input (all P ranks' inputs) per second.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+With N > 1 (launched by torchrun, one process per GPU) every rank runs its own
+independent 1 GB call (the simulation shards by message, no collective on the
+data path): weak scaling, value = all ranks' input bytes / max-over-ranks time.
+
+``--impl reference`` times the oracle (plain C, single thread) on the host on a
+bounded sample of group columns of the same workload, rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "Echo 4-bit all-reduce sim GB/s of bf16 input (P=8, 1 GB); % HBM roofline"
+FALLBACK_HBM_GBS = 6650.0
+
+# group columns of the workload timed on the host (one oracle call each)
+CPU_BASELINE_COLS = 1 << 17
+REFERENCE_STEP_COLS = 1 << 14
+
+
+def _workload():
+    import workloads as W
+    return W.HEADLINE
+
+
+def _peak_hbm():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def algorithmic_bytes(P, n, group, bits, feedback=True):
+    """Minimal bytes each kernel must move per call: every tensor crosses HBM
+    once, each payload is written once and read once."""
+    G = -(-n // group)
+    pb = group * bits // 8 + 4                       # payload bytes per group
+    st = 16 if feedback else 0                       # two fp32 EMAs read + written
+    xb = 2 * group                                   # bf16 input of one group
+    q = (P - 1) * G * (xb + st * group + pb)          # non-owned rank-groups
+    r = G * (xb + st * group + (P - 1) * pb + pb)      # owners: own x + EMAs, P-1 payloads in, gather out
+    g = G * (pb + P * xb)                             # gather payload in, P outputs
+    return {"quantize": q, "reduce": r, "gather": g, "total": q + r + g}
+
+
+def _kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("echo_kernels.cuh", "echo_api.cu"):
+        with open(os.path.join(ROOT, "bit_error_compensated_group_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _measured_traffic():
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, or None when the kernel changed since it was captured."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+    except Exception:
+        return None
+    if t.get("source_hash") != _kernel_source_hash():
+        return None
+    return t.get("bytes_per_launch")
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        import torch
+        self.proc = None
+        self.path = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            self.path = f"/tmp/echo_clocks_{os.getpid()}.csv"
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", sel, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) == 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def cpu_sample_rate(cols, seed=123):
+    """Time the oracle (single thread, as it stands) on `cols` group columns
+    of the workload; returns (GB/s of bf16 input, seconds, element-ranks)."""
+    import numpy as np
+    import torch
+    import oracle as O
+    import workloads as W
+    w = _workload()
+    P, group = w.P, w.group
+    G = -(-w.n // group)
+    j0 = (G // 2) - cols // 2                     # straddles an owner boundary at P = 8
+    m = cols * group
+    x = np.empty((P, m), np.uint16)
+    for r in range(P):
+        x[r] = W.bf16_bits(W.student_t3_unit_f32(m, W.seed_of(w.cid, 7, r)).to(torch.bfloat16))
+    el = np.zeros((P, m), np.float32)
+    es = np.zeros((P, m), np.float32)
+    t0 = time.perf_counter()
+    O.echo_allreduce(x, n_total=w.n, group=group, bits=w.bits, e_long=el, e_short=es, eta=w.eta,
+                     alpha_long=w.alpha_long, alpha_short=w.alpha_short, w=w.w, j0=j0, jc=cols)
+    dt = time.perf_counter() - t0
+    return P * m * 2 / dt / 1e9, dt, P * m
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = _workload()
+    cols = REFERENCE_STEP_COLS
+    for _ in range(args.warmup):
+        cpu_sample_rate(cols)
+    times = []
+    for _ in range(args.steps):
+        _, dt, er = cpu_sample_rate(cols)
+        times.append(dt)
+    tot = sum(times)
+    er = w.P * cols * w.group
+    value = args.steps * er * 2 / tot / 1e9
+    sample = f"{cols} of {-(-w.n // w.group)} group columns x P={w.P} per step ({er} element-ranks)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": _config(w),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _config(w):
+    return {"workload": w.name, "P": w.P, "n": w.n, "tokens": w.tokens, "hidden": w.hidden, "group": w.group,
+            "bits": w.bits, "feedback": True, "eta": w.eta, "alpha_long": w.alpha_long,
+            "alpha_short": w.alpha_short, "w": w.w, "values": "Student-t nu=3 / sqrt(3)",
+            "l2": "no flush: each step touches ~90 GB, far larger than the 126 MB L2"}
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+    import workloads as W
+    import bit_error_compensated_group_b200 as E
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    w = _workload()
+    P, n, group, bits = w.P, w.n, w.group, w.bits
+    ar = E.EchoAllReduce(n, P, group, bits, feedback=True, device=dev)
+    inputs = []
+    for r in range(P):
+        inputs.append(W.rank_input(w, r, site=rank, device=dev))   # each GPU its own message
+    outputs = [torch.empty_like(t) for t in inputs]
+    stream = torch.cuda.current_stream(dev)
+    h = ar.handle
+    fb = (w.eta, w.alpha_long, w.alpha_short, w.w)
+
+    def step(evs=None):
+        if evs is not None:
+            evs[0].record(stream)
+        E.echo_phase_quantize(inputs, h, bits, *fb, stream=stream)
+        if evs is not None:
+            evs[1].record(stream)
+        E.echo_phase_reduce(inputs, None, h, bits, *fb, stream=stream)
+        if evs is not None:
+            evs[2].record(stream)
+        E.echo_phase_gather(outputs, h, bits, stream=stream)
+        if evs is not None:
+            evs[3].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    barrier()
+    for i in range(args.steps):
+        step(evs[i])
+    barrier()
+    clock_info = clocks.stop()
+    rc, flags = ar.status()
+    per_phase = {"quantize": 0.0, "reduce": 0.0, "gather": 0.0}
+    total_ms = evs[0][0].elapsed_time(evs[-1][3])
+    for e in evs:
+        per_phase["quantize"] += e[0].elapsed_time(e[1])
+        per_phase["reduce"] += e[1].elapsed_time(e[2])
+        per_phase["gather"] += e[2].elapsed_time(e[3])
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+
+    # end to end through the public call with host buffers: pinned inputs
+    # copied in, the call, the reduced result copied out, every step
+    e2e = None
+    if not args.no_e2e:
+        e2e_steps = max(1, min(args.steps, 4))
+        host_in = [torch.empty(n, dtype=torch.bfloat16, pin_memory=True) for _ in range(P)]
+        for r in range(P):
+            host_in[r].copy_(inputs[r])
+        host_out = torch.empty(n, dtype=torch.bfloat16, pin_memory=True)
+
+        def e2e_step():
+            for r in range(P):
+                inputs[r].copy_(host_in[r], non_blocking=True)
+            E.echo_allreduce_sim(inputs, outputs, h, n, P, bits, group, *fb, stream=stream)
+            host_out.copy_(outputs[0], non_blocking=True)
+
+        e2e_step()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        b.record(stream)
+        barrier()
+        et = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(et, op=dist.ReduceOp.MAX)
+        e2e_ms = float(et.item()) / e2e_steps
+        e2e = {"value": world * P * n * 2 / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": P * n * 2, "d2h_bytes_per_step": n * 2,
+               "ms_per_step": e2e_ms, "steps": e2e_steps}
+        del host_in, host_out
+
+    if rank == 0:
+        ms = max_ms / args.steps
+        in_bytes = P * n * 2
+        value = world * in_bytes / (ms * 1e-3) / 1e9
+        peak, peak_kind = _peak_hbm()
+        ab = algorithmic_bytes(P, n, group, bits)
+        q_ms = per_phase["quantize"] / args.steps
+        achieved = ab["quantize"] / (q_ms * 1e-3) / 1e9
+        traffic = _measured_traffic()
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": _config(w),
+            "roofline": {"bound": "hbm", "kernel": "k_quantize", "achieved": achieved, "peak": peak,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
+                         "algorithmic_bytes": ab["quantize"]},
+            "roofline_call": {"bytes": ab["total"], "achieved": ab["total"] / (ms * 1e-3) / 1e9,
+                              "frac": ab["total"] / (ms * 1e-3) / 1e9 / peak},
+            "phases_ms": {k: v / args.steps for k, v in per_phase.items()},
+            "elements_per_s": world * P * n / (ms * 1e-3),
+            "gpu_launches": 3 * args.steps if P >= 2 else args.steps,
+            "clocks": clock_info, "status": rc, "flags": flags,
+            "e2e": e2e,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            gbs, dt, er = cpu_sample_rate(CPU_BASELINE_COLS)
+            line["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                    "sample": f"{CPU_BASELINE_COLS} group columns x P={P} "
+                                              f"({er} element-ranks, {dt:.1f} s, single thread)"}
+        print(json.dumps(line), flush=True)
+    ar.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="echo", choices=["echo", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,314 @@
+// echo_api.cu -- the C ABI declared in include/echo.h: argument checks,
+// workspace layout and kernel launches. The library never allocates device
+// memory; all work goes on the caller's stream.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <new>
+
+#include "echo.h"
+#include "echo_kernels.cuh"
+#include "echo_pipeline.cuh"
+
+struct echo_state {
+    int64_t n;
+    int P;
+    int group;
+    int max_bits;
+    int64_t G;
+    int64_t S;
+    float* state;          // nullptr: no feedback
+    uint8_t* workspace;
+    int device;
+    int sm_count;
+};
+
+namespace {
+
+constexpr uint64_t kAlign = 256;
+constexpr int64_t kMaxN = int64_t(1) << 40;
+
+uint64_t align_up(uint64_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool valid_group(int g) { return g == 32 || g == 64 || g == 128 || g == 256; }
+bool valid_bits(int b) { return b == 4 || b == 8; }
+bool valid_sizes(int64_t n, int P, int group) {
+    return n >= 1 && n < kMaxN && P >= 1 && P <= ECHO_MAX_RANKS && valid_group(group);
+}
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+bool in_unit(float v) { return v >= 0.0f && v <= 1.0f; }   // NaN fails
+
+bool layout(int64_t n, int P, int group, int max_bits, int bits, echo_layout* L) {
+    if (!valid_sizes(n, P, group) || !valid_bits(max_bits) || !valid_bits(bits) || bits > max_bits) return false;
+    const uint64_t G = (uint64_t)((n + group - 1) / group);
+    const uint64_t cb_max = (uint64_t)group * (uint64_t)max_bits / 8;
+    L->groups = (int64_t)G;
+    L->state_stride = (int64_t)(G * (uint64_t)group);
+    L->code_bytes = (uint64_t)group * (uint64_t)bits / 8;
+    uint64_t off = 0;
+    L->flags_offset = off;
+    off += kAlign;
+    L->a2a_codes_offset = off;
+    off = align_up(off + (uint64_t)P * G * cb_max);
+    L->a2a_params_offset = off;
+    off = align_up(off + (uint64_t)P * G * 4);
+    L->gather_codes_offset = off;
+    off = align_up(off + G * cb_max);
+    L->gather_params_offset = off;
+    off = align_up(off + G * 4);
+    L->workspace_bytes = off;
+    L->state_bytes = (uint64_t)P * 2 * G * (uint64_t)group * sizeof(float);
+    return true;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? ECHO_OK : ECHO_ECUDA; }
+
+template <typename K>
+int grid_for(K kernel, const echo_state* st, int threads = echo_dev::kThreads, int smem = 0) {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) != cudaSuccess ||
+        per_sm < 1) {
+        per_sm = 1;
+    }
+    return st->sm_count * per_sm;
+}
+
+// Pipelined kernels: opt in to their dynamic shared memory once.
+template <typename K>
+int pipe_grid(K kernel, const echo_state* st) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, echo_dev::kPipeSmem) !=
+        cudaSuccess) {
+        return 0;
+    }
+    return grid_for(kernel, st, echo_dev::kPipeThreads, echo_dev::kPipeSmem);
+}
+
+enum class Stage { Quantize, Reduce, Gather };
+
+template <int GROUP, int BITS>
+int launch_stage(Stage stage, const echo_dev::Args& a, const echo_state* st, cudaStream_t s) {
+    switch (stage) {
+        case Stage::Quantize: {
+            auto k = echo_dev::k_quantize_tma<GROUP, BITS>;
+            static int grid = 0;
+            if (grid == 0) grid = pipe_grid(k, st);
+            if (grid == 0) return ECHO_ECUDA;
+            k<<<grid, echo_dev::kPipeThreads, echo_dev::kPipeSmem, s>>>(a);
+            break;
+        }
+        case Stage::Reduce: {
+            auto k = echo_dev::k_reduce_tma<GROUP, BITS>;
+            static int grid = 0;
+            if (grid == 0) grid = pipe_grid(k, st);
+            if (grid == 0) return ECHO_ECUDA;
+            k<<<grid, echo_dev::kPipeThreads, echo_dev::kPipeSmem, s>>>(a);
+            break;
+        }
+        case Stage::Gather: {
+            auto k = echo_dev::k_gather<GROUP, BITS>;
+            static int grid = 0;
+            if (grid == 0) grid = grid_for(k, st);
+            k<<<grid, echo_dev::kThreads, 0, s>>>(a);
+            break;
+        }
+    }
+    return cuda_status(cudaGetLastError());
+}
+
+template <int GROUP>
+int launch_bits(Stage stage, int bits, const echo_dev::Args& a, const echo_state* st, cudaStream_t s) {
+    return bits == 4 ? launch_stage<GROUP, 4>(stage, a, st, s) : launch_stage<GROUP, 8>(stage, a, st, s);
+}
+
+int launch(Stage stage, int bits, const echo_dev::Args& a, const echo_state* st, cudaStream_t s) {
+    switch (st->group) {
+        case 32: return launch_bits<32>(stage, bits, a, st, s);
+        case 64: return launch_bits<64>(stage, bits, a, st, s);
+        case 128: return launch_bits<128>(stage, bits, a, st, s);
+        case 256: return launch_bits<256>(stage, bits, a, st, s);
+    }
+    return ECHO_EINVAL;
+}
+
+bool valid_feedback(float eta, float aL, float aS, float w) {
+    return std::isfinite(eta) && in_unit(aL) && in_unit(aS) && in_unit(w);
+}
+
+// Fill the kernel arguments; false when a pointer is missing or misaligned.
+bool make_args(const echo_state* st, int bits, const void* const* inputs, void* const* outputs,
+               float eta, float aL, float aS, float w, echo_dev::Args* a) {
+    std::memset(a, 0, sizeof(*a));
+    echo_layout L;
+    if (!layout(st->n, st->P, st->group, st->max_bits, bits, &L)) return false;
+    for (int r = 0; r < st->P; ++r) {
+        if (inputs) {
+            if (!inputs[r] || !aligned(inputs[r], 16)) return false;
+            a->in[r] = static_cast<const uint16_t*>(inputs[r]);
+        }
+        if (outputs) {
+            if (!outputs[r] || !aligned(outputs[r], 16)) return false;
+            a->out[r] = static_cast<uint16_t*>(outputs[r]);
+        }
+    }
+    a->state = st->state;
+    a->a2a_codes = st->workspace + L.a2a_codes_offset;
+    a->a2a_params = reinterpret_cast<uint32_t*>(st->workspace + L.a2a_params_offset);
+    a->g_codes = st->workspace + L.gather_codes_offset;
+    a->g_params = reinterpret_cast<uint32_t*>(st->workspace + L.gather_params_offset);
+    a->flags = reinterpret_cast<uint32_t*>(st->workspace + L.flags_offset);
+    a->n = st->n;
+    a->G = st->G;
+    a->S = st->S;
+    a->P = st->P;
+    a->eta = eta;
+    a->w = w;
+    a->one_minus_w = 1.0f - w;
+    a->a_long = aL;
+    a->keep_long = 1.0f - aL;
+    a->a_short = aS;
+    a->keep_short = 1.0f - aS;
+    return true;
+}
+
+int set_device(const echo_state* st) {
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) return ECHO_ECUDA;
+    if (cur != st->device && cudaSetDevice(st->device) != cudaSuccess) return ECHO_ECUDA;
+    return ECHO_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t echo_state_bytes(int64_t n, int P, int group) {
+    echo_layout L;
+    return layout(n, P, group, 4, 4, &L) ? (size_t)L.state_bytes : 0;
+}
+
+size_t echo_workspace_bytes(int64_t n, int P, int group, int max_bits) {
+    echo_layout L;
+    return layout(n, P, group, max_bits, valid_bits(max_bits) ? max_bits : 0, &L) ? (size_t)L.workspace_bytes : 0;
+}
+
+int echo_query_layout(int64_t n, int P, int group, int max_bits, int bits, echo_layout* out) {
+    if (!out) return ECHO_EINVAL;
+    echo_layout L;
+    if (!layout(n, P, group, max_bits, bits, &L)) return ECHO_EINVAL;
+    *out = L;
+    return ECHO_OK;
+}
+
+int echo_init_state(echo_state** out, int64_t n, int P, int group, int max_bits, void* state_dev,
+                    void* workspace_dev, echo_stream_t stream) {
+    echo_layout L;
+    if (!out || !layout(n, P, group, max_bits, max_bits, &L)) return ECHO_EINVAL;
+    if (!workspace_dev || !aligned(workspace_dev, kAlign)) return ECHO_EINVAL;
+    if (state_dev && !aligned(state_dev, 16)) return ECHO_EINVAL;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ECHO_ECUDA;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return ECHO_ECUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (state_dev && cudaMemsetAsync(state_dev, 0, L.state_bytes, s) != cudaSuccess) return ECHO_ECUDA;
+    if (cudaMemsetAsync(static_cast<uint8_t*>(workspace_dev) + L.flags_offset, 0, kAlign, s) != cudaSuccess)
+        return ECHO_ECUDA;
+    echo_state* st = new (std::nothrow) echo_state;
+    if (!st) return ECHO_EINVAL;
+    st->n = n;
+    st->P = P;
+    st->group = group;
+    st->max_bits = max_bits;
+    st->G = L.groups;
+    st->S = L.state_stride;
+    st->state = static_cast<float*>(state_dev);
+    st->workspace = static_cast<uint8_t*>(workspace_dev);
+    st->device = dev;
+    st->sm_count = sms;
+    *out = st;
+    return ECHO_OK;
+}
+
+int echo_phase_quantize(const void* const* inputs, echo_state* st, int bits, float eta, float alpha_long,
+                        float alpha_short, float w, echo_stream_t stream) {
+    if (!st || !inputs || !valid_bits(bits) || bits > st->max_bits) return ECHO_EINVAL;
+    if (!valid_feedback(eta, alpha_long, alpha_short, w)) return ECHO_EINVAL;
+    echo_dev::Args a;
+    if (!make_args(st, bits, inputs, nullptr, eta, alpha_long, alpha_short, w, &a)) return ECHO_EINVAL;
+    if (int rc = set_device(st)) return rc;
+    if (st->P < 2) return ECHO_OK;
+    return launch(Stage::Quantize, bits, a, st, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int echo_phase_reduce(const void* const* inputs, void* const* outputs, echo_state* st, int bits, float eta,
+                      float alpha_long, float alpha_short, float w, echo_stream_t stream) {
+    if (!st || !inputs || !valid_bits(bits) || bits > st->max_bits) return ECHO_EINVAL;
+    if (!valid_feedback(eta, alpha_long, alpha_short, w)) return ECHO_EINVAL;
+    if (st->P == 1 && !outputs) return ECHO_EINVAL;
+    echo_dev::Args a;
+    if (!make_args(st, bits, inputs, st->P == 1 ? outputs : nullptr, eta, alpha_long, alpha_short, w, &a))
+        return ECHO_EINVAL;
+    if (int rc = set_device(st)) return rc;
+    return launch(Stage::Reduce, bits, a, st, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int echo_phase_gather(void* const* outputs, echo_state* st, int bits, echo_stream_t stream) {
+    if (!st || !outputs || !valid_bits(bits) || bits > st->max_bits) return ECHO_EINVAL;
+    echo_dev::Args a;
+    if (!make_args(st, bits, nullptr, outputs, 0.0f, 0.0f, 0.0f, 0.0f, &a)) return ECHO_EINVAL;
+    if (int rc = set_device(st)) return rc;
+    if (st->P < 2) return ECHO_OK;
+    return launch(Stage::Gather, bits, a, st, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int echo_allreduce_sim(const void* const* inputs, void* const* outputs, echo_state* st, int64_t n, int P, int bits,
+                       int group, float eta, float alpha_long, float alpha_short, float w, echo_stream_t stream) {
+    if (!st || !inputs || !outputs) return ECHO_EINVAL;
+    if (n != st->n || P != st->P || group != st->group) return ECHO_EINVAL;
+    if (!valid_bits(bits) || bits > st->max_bits) return ECHO_EINVAL;
+    if (!valid_feedback(eta, alpha_long, alpha_short, w)) return ECHO_EINVAL;
+    echo_dev::Args a;
+    if (!make_args(st, bits, inputs, outputs, eta, alpha_long, alpha_short, w, &a)) return ECHO_EINVAL;
+    if (int rc = set_device(st)) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (P >= 2) {
+        if (int rc = launch(Stage::Quantize, bits, a, st, s)) return rc;
+    }
+    if (int rc = launch(Stage::Reduce, bits, a, st, s)) return rc;
+    if (P >= 2) {
+        if (int rc = launch(Stage::Gather, bits, a, st, s)) return rc;
+    }
+    return ECHO_OK;
+}
+
+int echo_get_status(echo_state* st, echo_stream_t stream, uint32_t* device_flags) {
+    if (!st) return ECHO_EINVAL;
+    if (int rc = set_device(st)) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t flags = 0;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return ECHO_ECUDA;
+    if (cudaMemcpy(&flags, st->workspace, sizeof(flags), cudaMemcpyDeviceToHost) != cudaSuccess) return ECHO_ECUDA;
+    if (cudaMemset(st->workspace, 0, sizeof(flags)) != cudaSuccess) return ECHO_ECUDA;
+    if (device_flags) *device_flags = flags;
+    if (flags & ECHO_FLAG_TIMEOUT) return ECHO_ETIMEOUT;
+    return (flags & ECHO_FLAG_RANGE) ? ECHO_ERANGE : ECHO_OK;
+}
+
+int echo_free(echo_state* st) {
+    delete st;
+    return ECHO_OK;
+}
+
+const char* echo_status_string(int status) {
+    switch (status) {
+        case ECHO_OK: return "ok";
+        case ECHO_EINVAL: return "invalid argument";
+        case ECHO_ECUDA: return "CUDA error";
+        case ECHO_ERANGE: return "value outside the fp16 parameter range";
+        case ECHO_ETIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

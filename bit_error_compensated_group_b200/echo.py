@@ -1,0 +1,226 @@
+"""ctypes binding of ``libecho_b200.so`` (the C ABI in ``include/echo.h``).
+
+Argument marshalling only: every step of the all-reduce runs in the library's
+CUDA kernels. Functions keep the C names; tensors are passed as device
+pointers and the stream defaults to torch's current stream. A missing or
+unloadable library raises immediately -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+from . import _build
+
+ECHO_OK, ECHO_EINVAL, ECHO_ECUDA, ECHO_ERANGE, ECHO_ETIMEOUT = 0, 1, 2, 3, 4
+ECHO_FLAG_RANGE = 1
+ECHO_MAX_RANKS = 64
+
+LIB_PATH = _build.LIB
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+class EchoError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {echo_status_string(status)} ({status})")
+
+
+class EchoLayout(ctypes.Structure):
+    _fields_ = [
+        ("groups", ctypes.c_int64),
+        ("state_stride", ctypes.c_int64),
+        ("code_bytes", ctypes.c_uint64),
+        ("flags_offset", ctypes.c_uint64),
+        ("a2a_codes_offset", ctypes.c_uint64),
+        ("a2a_params_offset", ctypes.c_uint64),
+        ("gather_codes_offset", ctypes.c_uint64),
+        ("gather_params_offset", ctypes.c_uint64),
+        ("workspace_bytes", ctypes.c_uint64),
+        ("state_bytes", ctypes.c_uint64),
+    ]
+
+
+def lib() -> ctypes.CDLL:
+    """Load the CUDA library; raises if it was not built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"Echo CUDA library missing at {LIB_PATH}; build it with "
+                               "`python -m bit_error_compensated_group_b200._build`")
+        L = ctypes.CDLL(LIB_PATH)
+        V, I, I64, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
+        PP = ctypes.POINTER(ctypes.c_void_p)
+        L.echo_state_bytes.argtypes = [I64, I, I]
+        L.echo_state_bytes.restype = ctypes.c_size_t
+        L.echo_workspace_bytes.argtypes = [I64, I, I, I]
+        L.echo_workspace_bytes.restype = ctypes.c_size_t
+        L.echo_query_layout.argtypes = [I64, I, I, I, I, ctypes.POINTER(EchoLayout)]
+        L.echo_query_layout.restype = I
+        L.echo_init_state.argtypes = [ctypes.POINTER(V), I64, I, I, I, V, V, V]
+        L.echo_init_state.restype = I
+        L.echo_allreduce_sim.argtypes = [PP, PP, V, I64, I, I, I, F, F, F, F, V]
+        L.echo_allreduce_sim.restype = I
+        L.echo_phase_quantize.argtypes = [PP, V, I, F, F, F, F, V]
+        L.echo_phase_quantize.restype = I
+        L.echo_phase_reduce.argtypes = [PP, PP, V, I, F, F, F, F, V]
+        L.echo_phase_reduce.restype = I
+        L.echo_phase_gather.argtypes = [PP, V, I, V]
+        L.echo_phase_gather.restype = I
+        L.echo_get_status.argtypes = [V, V, ctypes.POINTER(ctypes.c_uint32)]
+        L.echo_get_status.restype = I
+        L.echo_free.argtypes = [V]
+        L.echo_free.restype = I
+        L.echo_status_string.argtypes = [I]
+        L.echo_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def echo_status_string(status: int) -> str:
+    return lib().echo_status_string(status).decode()
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != ECHO_OK:
+        raise EchoError(rc, what)
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError("Echo buffers must be contiguous CUDA tensors")
+    return t.data_ptr()
+
+
+def _ptr_array(ts: Sequence) -> ctypes.Array:
+    return (ctypes.c_void_p * len(ts))(*[_ptr(t) for t in ts])
+
+
+# ----------------------------------------------------------------- sizes
+
+def echo_state_bytes(n: int, P: int, group: int) -> int:
+    return int(lib().echo_state_bytes(n, P, group))
+
+
+def echo_workspace_bytes(n: int, P: int, group: int, max_bits: int) -> int:
+    return int(lib().echo_workspace_bytes(n, P, group, max_bits))
+
+
+def echo_query_layout(n: int, P: int, group: int, max_bits: int, bits: int) -> EchoLayout:
+    out = EchoLayout()
+    _check(lib().echo_query_layout(n, P, group, max_bits, bits, ctypes.byref(out)), "echo_query_layout")
+    return out
+
+
+# ----------------------------------------------------------------- calls
+
+def echo_init_state(n: int, P: int, group: int, max_bits: int, state, workspace, stream=None) -> ctypes.c_void_p:
+    h = ctypes.c_void_p()
+    _check(lib().echo_init_state(ctypes.byref(h), n, P, group, max_bits, _ptr(state), _ptr(workspace),
+                                 _stream(stream)), "echo_init_state")
+    return h
+
+
+def echo_allreduce_sim(inputs: Sequence, outputs: Sequence, st, n: int, P: int, bits: int, group: int,
+                       eta: float, alpha_long: float, alpha_short: float, w: float, stream=None) -> None:
+    _check(lib().echo_allreduce_sim(_ptr_array(inputs), _ptr_array(outputs), st, n, P, bits, group,
+                                    eta, alpha_long, alpha_short, w, _stream(stream)), "echo_allreduce_sim")
+
+
+def echo_phase_quantize(inputs: Sequence, st, bits: int, eta: float, alpha_long: float, alpha_short: float,
+                        w: float, stream=None) -> None:
+    _check(lib().echo_phase_quantize(_ptr_array(inputs), st, bits, eta, alpha_long, alpha_short, w,
+                                     _stream(stream)), "echo_phase_quantize")
+
+
+def echo_phase_reduce(inputs: Sequence, outputs: Optional[Sequence], st, bits: int, eta: float,
+                      alpha_long: float, alpha_short: float, w: float, stream=None) -> None:
+    outs = _ptr_array(outputs) if outputs is not None else None
+    _check(lib().echo_phase_reduce(_ptr_array(inputs), outs, st, bits, eta, alpha_long, alpha_short, w,
+                                   _stream(stream)), "echo_phase_reduce")
+
+
+def echo_phase_gather(outputs: Sequence, st, bits: int, stream=None) -> None:
+    _check(lib().echo_phase_gather(_ptr_array(outputs), st, bits, _stream(stream)), "echo_phase_gather")
+
+
+def echo_get_status(st, stream=None):
+    """Returns (status, flags); synchronizes the stream."""
+    flags = ctypes.c_uint32(0)
+    rc = lib().echo_get_status(st, _stream(stream), ctypes.byref(flags))
+    if rc not in (ECHO_OK, ECHO_ERANGE):
+        raise EchoError(rc, "echo_get_status")
+    return rc, int(flags.value)
+
+
+def echo_free(st) -> None:
+    lib().echo_free(st)
+
+
+# ----------------------------------------------------------------- convenience
+
+class EchoAllReduce:
+    """Owns (through torch) the EMA state and workspace of one message shape
+    and the library handle; ``__call__`` runs echo_allreduce_sim."""
+
+    def __init__(self, n: int, P: int, group: int = 128, max_bits: int = 4, feedback: bool = True,
+                 device=None, stream=None):
+        device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        self.n, self.P, self.group, self.max_bits = n, P, group, max_bits
+        self.layout = echo_query_layout(n, P, group, max_bits, max_bits)
+        self.workspace = torch.empty(int(self.layout.workspace_bytes), dtype=torch.uint8, device=device)
+        self.state = None
+        if feedback:
+            self.state = torch.empty(int(self.layout.state_bytes) // 4, dtype=torch.float32, device=device)
+        self.handle = echo_init_state(n, P, group, max_bits, self.state, self.workspace, stream)
+
+    def __call__(self, inputs, outputs, bits: int = 4, eta: float = 1.0, alpha_long: float = 0.05,
+                 alpha_short: float = 0.5, w: float = 0.5, stream=None) -> None:
+        echo_allreduce_sim(inputs, outputs, self.handle, self.n, self.P, bits, self.group,
+                           eta, alpha_long, alpha_short, w, stream)
+
+    # views of the state: [P][2][S] -> (e_long [P][n], e_short [P][n])
+    def ema_views(self):
+        S = int(self.layout.state_stride)
+        st = self.state.view(self.P, 2, S)
+        return st[:, 0, :self.n], st[:, 1, :self.n]
+
+    def payload_views(self, bits: int):
+        """(a2a_codes [P][G][cb], a2a_params [P][G] int32, gather_codes [G][cb], gather_params [G])."""
+        L = echo_query_layout(self.n, self.P, self.group, self.max_bits, bits)
+        G, cb, ws = int(L.groups), int(L.code_bytes), self.workspace
+        a2a_c = ws[L.a2a_codes_offset:L.a2a_codes_offset + self.P * G * cb].view(self.P, G, cb)
+        a2a_p = ws[L.a2a_params_offset:L.a2a_params_offset + self.P * G * 4].view(torch.int32).view(self.P, G)
+        g_c = ws[L.gather_codes_offset:L.gather_codes_offset + G * cb].view(G, cb)
+        g_p = ws[L.gather_params_offset:L.gather_params_offset + G * 4].view(torch.int32)
+        return a2a_c, a2a_p, g_c, g_p
+
+    def status(self, stream=None):
+        return echo_get_status(self.handle, stream)
+
+    def close(self) -> None:
+        if self.handle is not None:
+            echo_free(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,215 @@
+/*
+ * echo.h -- C ABI of the single-GPU simulation of Echo's 4-bit
+ * error-compensated all-reduce.
+ *
+ * The method (sources, in prose only -- the pages print no code):
+ *   [ABS] "Echo: Error-Compensated 4-Bit Tensor-Parallel Communication for
+ *         LLM Training and Inference" (arXiv 2610.14277), abstract;
+ *   [EXP] the explainer "テンソル並列の通信を4bitに圧縮する「Echo」",
+ *         sections "Echoの仕組み①" (mechanism 1: the all-reduce becomes an
+ *         all-to-all of 4-bit non-owned segments, a high-precision sum at each
+ *         segment's owner and a 4-bit all-gather of the requantized sum),
+ *         "Echoの仕組み②" (mechanism 2: the residuals the ranks keep sum to
+ *         minus the injected error; a long and a short moving average of them
+ *         are added back into the next call's input, fused into the entry
+ *         pass), "実測性能と精度" (an 8-bit mode for early layers) and
+ *         "よくある質問" (FAQ: the payload is 4-bit integers plus
+ *         half-precision parameters).
+ *
+ * One call of echo_allreduce_sim computes, for P virtual ranks whose bf16
+ * partial sums all sit in the memory of ONE GPU, the five phases:
+ *   1. feedback injection  x' = x + eta * (w * e_short + (1 - w) * e_long)
+ *   2. per-group asymmetric quantization of every rank's NON-owned groups
+ *      (fp16 scale s and zero z, codes packed two per byte): the all-to-all
+ *      payload, written to device memory;
+ *   3. at each group's owner: binary32 sum, in rank order 0..P-1, of its own
+ *      unquantized x' and the P-1 dequantized payloads, requantized into the
+ *      all-gather payload;
+ *   4. every rank dequantizes the gathered payload into its bf16 output;
+ *   5. the residuals (non-owner: x' - x_hat; owner: sum - y) update both
+ *      EMAs:  e <- (1 - alpha) * e + alpha * rho.
+ * The "transport" is the payload buffers in device memory; nothing crosses
+ * GPUs. The exact arithmetic (directed fp16 rounding of z and s, half-to-even
+ * codes, no fused multiply-add) is stated at echo_allreduce_sim below.
+ *
+ * Memory: the library never allocates device memory. The caller owns the P
+ * input and output buffers, the EMA state and a workspace; their sizes come
+ * from echo_state_bytes / echo_workspace_bytes. All work is enqueued on the
+ * caller's stream. Every function is host-callable, returns an echo_status
+ * and does not block unless stated.
+ */
+#ifndef ECHO_H
+#define ECHO_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Exported symbols keep default visibility when the library is built with
+ * hidden visibility. */
+#if defined(__GNUC__)
+#define ECHO_API __attribute__((visibility("default")))
+#else
+#define ECHO_API
+#endif
+
+/* Largest number of virtual ranks a call accepts. */
+#define ECHO_MAX_RANKS 64
+
+/* Sticky device flags read by echo_get_status. */
+#define ECHO_FLAG_RANGE 1u   /* a quantized group (or a P == 1 output) held a
+                                value outside [-65504, 65504] or a NaN: the
+                                fp16 parameters cannot describe it; outputs
+                                and state of that group are unspecified */
+#define ECHO_FLAG_TIMEOUT 2u /* a bounded device-side wait (between the
+                                bulk-copy producer and the compute warps of
+                                a kernel) expired; that call's results are
+                                unspecified */
+
+typedef enum echo_status {
+    ECHO_OK = 0,
+    ECHO_EINVAL = 1,     /* bad argument; nothing was enqueued */
+    ECHO_ECUDA = 2,      /* a CUDA runtime call or kernel launch failed */
+    ECHO_ERANGE = 3,     /* returned by echo_get_status when ECHO_FLAG_RANGE is set */
+    ECHO_ETIMEOUT = 4    /* returned by echo_get_status when ECHO_FLAG_TIMEOUT is set */
+} echo_status;
+
+/* Same object as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* echo_stream_t;
+
+/* Opaque host-side handle: sizes, the caller's state/workspace pointers and
+ * the launch configuration. It owns no device memory. */
+typedef struct echo_state echo_state;
+
+/* Byte offsets inside the workspace for a call with `bits`, and sizes.
+ *   flags          uint32 sticky flag word (ECHO_FLAG_*)
+ *   a2a codes      [P][G][code_bytes]  slot [r][j]: rank r's packed codes of
+ *                  group j, sent to owner(j); the owner's own slot is unused
+ *   a2a params     [P][G] uint32: fp16 bits of s in the low half, of z in the
+ *                  high half (little-endian: {s, z} as two uint16)
+ *   gather codes   [G][code_bytes]   the owner's requantized sum of group j
+ *   gather params  [G] uint32        as above
+ * Codes of a 4-bit group: element 2i in the low nibble, 2i+1 in the high
+ * nibble of byte i; 8-bit: one byte per element; a partial last group is
+ * padded with code 0. Group j covers elements [j*group, min(n, (j+1)*group))
+ * of the flattened message; owner(j) = the s with
+ * floor(s*G/P) <= j < floor((s+1)*G/P). */
+typedef struct echo_layout {
+    int64_t groups;              /* G = ceil(n / group) */
+    int64_t state_stride;        /* S = G * group floats per EMA per rank */
+    uint64_t code_bytes;         /* group * bits / 8 */
+    uint64_t flags_offset;
+    uint64_t a2a_codes_offset;
+    uint64_t a2a_params_offset;
+    uint64_t gather_codes_offset;
+    uint64_t gather_params_offset;
+    uint64_t workspace_bytes;    /* for max_bits */
+    uint64_t state_bytes;
+} echo_layout;
+
+/* Bytes of EMA state: float32 [P][2][S], S = ceil(n/group)*group; [r][0] is
+ * rank r's long EMA, [r][1] its short EMA; element k of the message at
+ * offset k (the padding past n is never read or written). 0 on bad sizes. */
+ECHO_API size_t echo_state_bytes(int64_t n, int P, int group);
+
+/* Bytes of workspace for calls with bits <= max_bits. 0 on bad sizes. */
+ECHO_API size_t echo_workspace_bytes(int64_t n, int P, int group, int max_bits);
+
+/* Fill *out for a call with `bits` (<= max_bits). ECHO_EINVAL on bad sizes. */
+ECHO_API int echo_query_layout(int64_t n, int P, int group, int max_bits, int bits, echo_layout* out);
+
+/*
+ * Create a handle for messages of n elements per rank over P ranks.
+ *   n          1 <= n < 2^40
+ *   P          1..ECHO_MAX_RANKS
+ *   group      32, 64, 128 or 256 elements per quantization group
+ *   max_bits   4 or 8: the largest `bits` later calls will use
+ *   state_dev  device pointer to echo_state_bytes(n, P, group) bytes, 16-byte
+ *              aligned, or NULL for "no feedback" (x' = x, no state traffic)
+ *   workspace_dev  device pointer to echo_workspace_bytes(...) bytes,
+ *              256-byte aligned
+ *   stream     the EMAs (if any) and the flag word are zeroed on it
+ * The caller keeps ownership of both buffers and must keep them alive until
+ * echo_free. Returns ECHO_EINVAL (nothing enqueued, *out untouched) or
+ * ECHO_ECUDA.
+ */
+ECHO_API int echo_init_state(echo_state** out, int64_t n, int P, int group, int max_bits,
+                    void* state_dev, void* workspace_dev, echo_stream_t stream);
+
+/*
+ * One all-reduce call over the P virtual ranks (phases 1-5 above).
+ *   inputs     host array of P device pointers, each to n bf16 values
+ *              (16-byte aligned): rank r's partial sum
+ *   outputs    host array of P device pointers, each to n bf16 values
+ *              (16-byte aligned): rank r's copy of the reduced result. An
+ *              output may be the same buffer as an input; other overlaps are
+ *              undefined.
+ *   st         handle from echo_init_state; n, P and group must match it
+ *   bits       4 (INT4) or 8 (the early-site 8-bit mode), <= the handle's
+ *              max_bits
+ *   eta        feedback gain, finite
+ *   alpha_long, alpha_short   EMA rates in [0, 1]
+ *   w          weight of the short EMA in the compensation, in [0, 1]
+ *   stream     CUDA stream; the call is asynchronous on it
+ * Arithmetic (binary32, round-to-nearest, no contraction into fused
+ * multiply-add): c = eta*(w*e_short + (1-w)*e_long), x' = float(x) + c
+ * (x' = float(x) without state); per group mn = min + 0, mx = max + 0,
+ * z = fp16 rounded toward -inf of mn, s = fp16 rounded toward +inf of
+ * (mx - z)/Q with Q = 2^bits - 1, code = clamp(rint_even((v - z) * (1/s)),
+ * 0, Q) (all 0 when s == 0), x_hat = code*s + z; the owner sums in rank
+ * order; y = bf16 round-to-nearest-even of the requantized sum (of x' when
+ * P == 1); each EMA e <- (1-alpha)*e + alpha*rho.
+ * Errors: ECHO_EINVAL when an argument is out of range, a pointer is NULL
+ * or misaligned, or n/P/group differ from the handle (nothing is enqueued);
+ * ECHO_ECUDA when a launch fails. Data-dependent range violations do not
+ * stop the call: they set ECHO_FLAG_RANGE (see echo_get_status).
+ */
+ECHO_API int echo_allreduce_sim(const void* const* inputs, void* const* outputs, echo_state* st,
+                       int64_t n, int P, int bits, int group,
+                       float eta, float alpha_long, float alpha_short, float w,
+                       echo_stream_t stream);
+
+/*
+ * The three kernels of echo_allreduce_sim, callable one by one (same
+ * arguments and errors; running them in this order on one stream is exactly
+ * echo_allreduce_sim):
+ *   echo_phase_quantize  phases 1, 2 and 5 for every rank's non-owned groups:
+ *                        writes the all-to-all payload and those EMAs
+ *                        (does nothing when P == 1)
+ *   echo_phase_reduce    phases 1, 3 and 5 for every group's owner: reads the
+ *                        all-to-all payload, writes the all-gather payload
+ *                        and the owners' EMAs (P == 1: writes outputs[0])
+ *   echo_phase_gather    phase 4: reads the all-gather payload, writes all P
+ *                        outputs (does nothing when P == 1)
+ */
+ECHO_API int echo_phase_quantize(const void* const* inputs, echo_state* st, int bits,
+                        float eta, float alpha_long, float alpha_short, float w,
+                        echo_stream_t stream);
+ECHO_API int echo_phase_reduce(const void* const* inputs, void* const* outputs, echo_state* st, int bits,
+                      float eta, float alpha_long, float alpha_short, float w,
+                      echo_stream_t stream);
+ECHO_API int echo_phase_gather(void* const* outputs, echo_state* st, int bits, echo_stream_t stream);
+
+/*
+ * Synchronize `stream`, read the sticky flag word into *device_flags (may be
+ * NULL) and clear it. Returns ECHO_ETIMEOUT when ECHO_FLAG_TIMEOUT was set,
+ * else ECHO_ERANGE when ECHO_FLAG_RANGE was set, else ECHO_OK;
+ * ECHO_ECUDA if the synchronization or copy fails.
+ * Blocks the host.
+ */
+ECHO_API int echo_get_status(echo_state* st, echo_stream_t stream, uint32_t* device_flags);
+
+/* Release the host handle (never the caller's device buffers). NULL is a no-op. */
+ECHO_API int echo_free(echo_state* st);
+
+/* Static string for a status code. */
+ECHO_API const char* echo_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ECHO_H */

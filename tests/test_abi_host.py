@@ -1,0 +1,115 @@
+"""Host-side checks of the C ABI (no GPU needed, no kernel launched).
+
+* the library builds for sm_100a and loads;
+* it exports every function include/echo.h declares;
+* size and layout queries follow the documented layout;
+* bad arguments are rejected with ECHO_EINVAL before any CUDA call, and with
+  no GPU present a valid init fails loudly with ECHO_ECUDA.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import bit_error_compensated_group_b200 as E
+from bit_error_compensated_group_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    _build.build()
+    return E.lib()
+
+
+def declared_functions():
+    with open(os.path.join(ROOT, "include", "echo.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"ECHO_API\s+[\w\s\*]+?\b(echo_\w+)\s*\(", text)))
+
+
+def test_exports_every_declared_function(L):
+    names = declared_functions()
+    assert len(names) >= 11, names
+    for name in names:
+        assert hasattr(L, name), name
+    # nothing but the C ABI is exported
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", _build.LIB], capture_output=True, text=True).stdout
+    exported = sorted(line.split()[-1] for line in out.splitlines() if " T " in line)
+    assert exported == names
+
+
+def _G(n, g):
+    return -(-n // g)
+
+
+@pytest.mark.parametrize("n,P,g,mb", [(4096, 2, 128, 4), (1000, 3, 32, 8), (1 << 29, 8, 128, 4), (777, 64, 256, 8)])
+def test_layout(L, n, P, g, mb):
+    G = _G(n, g)
+    assert E.echo_state_bytes(n, P, g) == P * 2 * G * g * 4
+    for bits in (4, 8):
+        if bits > mb:
+            with pytest.raises(E.EchoError):
+                E.echo_query_layout(n, P, g, mb, bits)
+            continue
+        lay = E.echo_query_layout(n, P, g, mb, bits)
+        assert lay.groups == G and lay.state_stride == G * g
+        assert lay.code_bytes == g * bits // 8
+        regions = [(lay.flags_offset, 4), (lay.a2a_codes_offset, P * G * g * mb // 8),
+                   (lay.a2a_params_offset, P * G * 4), (lay.gather_codes_offset, G * g * mb // 8),
+                   (lay.gather_params_offset, G * 4)]
+        for (o1, s1), (o2, _) in zip(regions, regions[1:]):
+            assert o1 % 256 == 0 and o1 + s1 <= o2
+        assert regions[-1][0] + regions[-1][1] <= lay.workspace_bytes
+        assert lay.workspace_bytes == E.echo_workspace_bytes(n, P, g, mb)
+
+
+@pytest.mark.parametrize("n,P,g,mb", [(0, 2, 128, 4), (10, 0, 128, 4), (10, 65, 128, 4),
+                                      (10, 2, 48, 4), (10, 2, 128, 5), (1 << 41, 2, 128, 4)])
+def test_bad_sizes(L, n, P, g, mb):
+    assert E.echo_workspace_bytes(n, P, g, mb) == 0
+    lay = E.EchoLayout()
+    assert L.echo_query_layout(n, P, g, mb, 4, ctypes.byref(lay)) == E.ECHO_EINVAL
+    h = ctypes.c_void_p()
+    assert L.echo_init_state(ctypes.byref(h), n, P, g, mb, None, 256, None) == E.ECHO_EINVAL
+    assert h.value is None
+
+
+def test_init_rejects_bad_pointers_before_cuda(L):
+    h = ctypes.c_void_p()
+    # no workspace / misaligned workspace / misaligned state: rejected on the host
+    assert L.echo_init_state(ctypes.byref(h), 1024, 2, 128, 4, None, None, None) == E.ECHO_EINVAL
+    assert L.echo_init_state(ctypes.byref(h), 1024, 2, 128, 4, None, 4096 + 8, None) == E.ECHO_EINVAL
+    assert L.echo_init_state(ctypes.byref(h), 1024, 2, 128, 4, 4096 + 4, 4096, None) == E.ECHO_EINVAL
+    assert L.echo_init_state(None, 1024, 2, 128, 4, None, 4096, None) == E.ECHO_EINVAL
+
+
+def test_calls_reject_missing_handle(L):
+    arr = (ctypes.c_void_p * 2)(4096, 8192)
+    assert L.echo_allreduce_sim(arr, arr, None, 1024, 2, 4, 128, 1.0, 0.05, 0.5, 0.5, None) == E.ECHO_EINVAL
+    assert L.echo_phase_quantize(arr, None, 4, 1.0, 0.05, 0.5, 0.5, None) == E.ECHO_EINVAL
+    assert L.echo_phase_reduce(arr, arr, None, 4, 1.0, 0.05, 0.5, 0.5, None) == E.ECHO_EINVAL
+    assert L.echo_phase_gather(arr, None, 4, None) == E.ECHO_EINVAL
+    assert L.echo_get_status(None, None, None) == E.ECHO_EINVAL
+    assert L.echo_free(None) == E.ECHO_OK
+
+
+def test_status_strings(L):
+    for code in range(5):
+        assert E.echo_status_string(code)
+    assert E.echo_status_string(99) == "unknown status"
+
+
+def test_no_gpu_fails_loudly(L):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    h = ctypes.c_void_p()
+    rc = L.echo_init_state(ctypes.byref(h), 1024, 2, 128, 4, None, 4096, None)
+    assert rc == E.ECHO_ECUDA
+    with pytest.raises(E.EchoError) as ei:
+        E.echo_init_state(1024, 2, 128, 4, None, 4096, stream=0)
+    assert ei.value.status == E.ECHO_ECUDA
