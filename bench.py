@@ -21,7 +21,6 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -40,9 +39,15 @@ CPU_BASELINE_COLS = 1 << 17
 REFERENCE_STEP_COLS = 1 << 14
 
 
+_TOKENS = None   # --tokens: a smaller message of the same shape family (profiling only)
+
+
 def _workload():
+    import dataclasses
     import workloads as W
-    return W.HEADLINE
+    if _TOKENS is None:
+        return W.HEADLINE
+    return dataclasses.replace(W.HEADLINE, name=f"{W.HEADLINE.name}_tokens{_TOKENS}", tokens=_TOKENS)
 
 
 def _peak_hbm():
@@ -337,7 +342,11 @@ def main():
     ap.add_argument("--impl", default="echo", choices=["echo", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="tokens per rank (default 131072, the 1 GB message); smaller values are for profiling")
     args = ap.parse_args()
+    global _TOKENS
+    _TOKENS = args.tokens
     if args.impl == "reference":
         run_reference(args)
     else:

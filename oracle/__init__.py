@@ -27,7 +27,9 @@ _lib = None
 def lib() -> ctypes.CDLL:
     global _lib
     if _lib is None:
-        path = _build.build()
+        # ECHO_ORACLE_LIB lets the mutation test load a deliberately broken
+        # copy of the oracle; normally the in-tree build is used
+        path = os.environ.get("ECHO_ORACLE_LIB") or _build.build()
         L = ctypes.CDLL(path)
         P = ctypes.c_void_p
         L.oracle_f32_to_f16.argtypes = [ctypes.c_float, ctypes.c_int]

@@ -147,18 +147,26 @@ def test_in_place_outputs():
         gpu.close()
 
 
-def test_range_flag_and_recovery():
+@pytest.mark.parametrize("feedback", [True, False])
+def test_range_flag_and_recovery(feedback):
+    """A value outside the fp16 parameter range raises the sticky flag;
+    echo_get_status reports and clears it. The EMAs of a flagged group are
+    unspecified, so the recovery call starts from fresh state."""
     P, n = 2, 4096
     x = _random_inputs(P, n, 10)
     x[1, 1234] = 1e6
-    gpu = GpuEcho(P, n)
+    gpu = GpuEcho(P, n, feedback=feedback)
     try:
         gpu.set_inputs(x)
         gpu.call(Params())
         rc, flags = gpu.status()
         assert rc == E.ECHO_ERANGE and flags & E.ECHO_FLAG_RANGE
+        rc, flags = gpu.status()                     # cleared by the read
+        assert rc == E.ECHO_OK and flags == 0
         x[1, 1234] = 0.5
         gpu.set_inputs(x)
+        if feedback:
+            gpu.set_state(np.zeros((P, n), np.float32), np.zeros((P, n), np.float32))
         gpu.call(Params())
         rc, flags = gpu.status()
         assert rc == E.ECHO_OK and flags == 0

@@ -132,6 +132,19 @@ def test_constant_group_is_exact(bits):
         assert np.all(gq.vhat == np.float32(c))
 
 
+@pytest.mark.parametrize("bits", [4, 8])
+def test_negative_zero_extremes_are_canonical(bits):
+    """A group whose minimum (or maximum) is -0 quantizes exactly as with +0:
+    the +0 added to min and max makes the parameters independent of how a
+    min/max reduction orders signed zeros."""
+    for v in ([-0.0, 1.0, 2.0, 0.5], [-0.0, -1.5, -0.25], [-0.0, -0.0], [-0.0, 0.0, 3.0]):
+        a = O.quantize_group(np.array(v, np.float32), bits)
+        b = O.quantize_group(np.array([0.0 if x == 0 else x for x in v], np.float32), bits)
+        assert (a.s_bits, a.z_bits) == (b.s_bits, b.z_bits)
+        assert a.z_bits != 0x8000 and a.s_bits != 0x8000
+        assert np.array_equal(a.codes, b.codes)
+
+
 def test_range_flag():
     assert O.quantize_group(np.array([1.0, 70000.0], np.float32), 4).flag == O.FLAG_RANGE
     assert O.quantize_group(np.array([1.0, np.nan], np.float32), 4).flag == O.FLAG_RANGE
