@@ -74,7 +74,7 @@ def algorithmic_bytes(P, n, group, bits, feedback=True):
 
 def _kernel_source_hash():
     h = hashlib.sha256()
-    for f in ("echo_kernels.cuh", "echo_api.cu"):
+    for f in ("echo_kernels.cuh", "echo_pipeline.cuh", "echo_api.cu"):
         with open(os.path.join(ROOT, "bit_error_compensated_group_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -138,6 +138,23 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
                 "reasons": reasons, "samples": len(rows)}
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The largest `value` over all ranks (every rank gets it); the job's time
+    is its slowest rank's."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_gbs(world: int, bytes_per_rank: int, max_ms: float) -> float:
+    """Whole-job GB/s: every rank moved its own message in the slowest rank's time."""
+    return world * bytes_per_rank / (max_ms * 1e-3) / 1e9
 
 
 def cpu_sample_rate(cols, seed=123):
@@ -260,10 +277,7 @@ def run_gpu(args):
         per_phase["quantize"] += e[0].elapsed_time(e[1])
         per_phase["reduce"] += e[1].elapsed_time(e[2])
         per_phase["gather"] += e[2].elapsed_time(e[3])
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
+    max_ms = max_over_ranks(total_ms, world, dev)
 
     # end to end through the public call with host buffers: pinned inputs
     # copied in, the call, the reduced result copied out, every step
@@ -289,19 +303,15 @@ def run_gpu(args):
             e2e_step()
         b.record(stream)
         barrier()
-        et = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(et, op=dist.ReduceOp.MAX)
-        e2e_ms = float(et.item()) / e2e_steps
-        e2e = {"value": world * P * n * 2 / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+        e2e_ms = max_over_ranks(a.elapsed_time(b), world, dev) / e2e_steps
+        e2e = {"value": weak_scaling_gbs(world, P * n * 2, e2e_ms), "unit": "GB/s",
                "h2d_bytes_per_step": P * n * 2, "d2h_bytes_per_step": n * 2,
                "ms_per_step": e2e_ms, "steps": e2e_steps}
         del host_in, host_out
 
     if rank == 0:
         ms = max_ms / args.steps
-        in_bytes = P * n * 2
-        value = world * in_bytes / (ms * 1e-3) / 1e9
+        value = weak_scaling_gbs(world, P * n * 2, ms)
         peak, peak_kind = _peak_hbm()
         ab = algorithmic_bytes(P, n, group, bits)
         q_ms = per_phase["quantize"] / args.steps

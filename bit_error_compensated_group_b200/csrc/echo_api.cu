@@ -282,6 +282,14 @@ int echo_allreduce_sim(const void* const* inputs, void* const* outputs, echo_sta
     return ECHO_OK;
 }
 
+int echo_check_watchdog(echo_state* st, uint32_t limit_us, echo_stream_t stream) {
+    if (!st || limit_us < 1 || limit_us > 10000000u) return ECHO_EINVAL;
+    if (int rc = set_device(st)) return rc;
+    echo_dev::k_watchdog_check<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<uint32_t*>(st->workspace), 1000ull * limit_us);
+    return cuda_status(cudaGetLastError());
+}
+
 int echo_get_status(echo_state* st, echo_stream_t stream, uint32_t* device_flags) {
     if (!st) return ECHO_EINVAL;
     if (int rc = set_device(st)) return rc;

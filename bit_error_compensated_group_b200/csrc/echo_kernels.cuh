@@ -440,32 +440,46 @@ __global__ void __launch_bounds__(kThreads) k_reduce(const Args a) {
 }
 
 // Stage 3: decode the gathered payload once per group, write all P outputs.
+// No group reduction here, so lane t simply owns the 8 contiguous elements
+// [8t, 8t + 8) of its group: one 32-bit (4-bit codes) or 64-bit (8-bit codes)
+// load, and one 16-byte store per output.
+template <int BITS>
+__device__ __forceinline__ uint2 load_codes8(const uint8_t* group_codes, int t) {
+    if (BITS == 4) return make_uint2(*reinterpret_cast<const uint32_t*>(group_codes + 4 * t), 0u);
+    return *reinterpret_cast<const uint2*>(group_codes + 8 * t);
+}
+
+template <int BITS>
+__device__ __forceinline__ int code8(uint2 w, int k) {
+    return BITS == 4 ? (int)((w.x >> (4 * k)) & 0xfu) : (int)(((k < 4 ? w.x : w.y) >> (8 * (k & 3))) & 0xffu);
+}
+
 template <int GROUP, int BITS>
 __global__ void __launch_bounds__(kThreads) k_gather(const Args a) {
-    using LN = Lane<GROUP>;
-    constexpr int GPW = LN::GPW, CB = GROUP * BITS / 8;
-    const LN ln;
+    constexpr int L = GROUP / 8, GPW = 32 / L, CB = GROUP * BITS / 8;
+    const int lane = threadIdx.x & 31;
+    const int sub = lane / L, t = lane % L;
     const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
     for (long long j0 = warp * GPW; j0 < a.G; j0 += nwarps * GPW) {
-        const long long j = j0 + ln.sub;
+        const long long j = j0 + sub;
         if (j >= a.G) continue;   // no shuffles below
-        const bool full = (j + 1) * GROUP <= a.n;
-        const uint8_t* codes = a.g_codes + (size_t)j * CB;
+        const uint2 w = load_codes8<BITS>(a.g_codes + (size_t)j * CB, t);
         const uint32_t p = a.g_params[j];
         const float s = param_s(p), z = param_z(p);
         uint32_t yb[8];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const uint32_t w = load_chunk_codes<BITS>(codes, ln.chunk(h));
+        for (int k = 0; k < 8; ++k) yb[k] = f2bf16(decode(code8<BITS>(w, k), s, z));
+        const long long e = j * GROUP + 8 * t;
+        if (e + 8 <= a.n) {
+            const uint4 v = make_uint4(yb[0] | (yb[1] << 16), yb[2] | (yb[3] << 16), yb[4] | (yb[5] << 16),
+                                       yb[6] | (yb[7] << 16));
+            for (int r = 0; r < a.P; ++r) __stcs(reinterpret_cast<uint4*>(a.out[r] + e), v);
+        } else {
+            for (int r = 0; r < a.P; ++r) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) yb[4 * h + k] = f2bf16(decode(unpack1<BITS>(w, k), s, z));
-        }
-        for (int r = 0; r < a.P; ++r) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const long long e = j * GROUP + 4 * ln.chunk(h);
-                store_y4(a.out[r], e, a.n, full, &yb[4 * h]);
+                for (int k = 0; k < 8; ++k)
+                    if (e + k < a.n) a.out[r][e + k] = (uint16_t)yb[k];
             }
         }
     }

@@ -494,4 +494,20 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
     }
 }
 
+// Watchdog self-check: one thread waits, with the same bounded wait the
+// pipelines use, on an mbarrier that expects one arrival nobody makes. The
+// wait expires after limit_ns, the kernel records ECHO_FLAG_TIMEOUT and
+// returns normally, leaving the context usable.
+__global__ void k_watchdog_check(uint32_t* flags, unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        mbar_fence_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !mbar_wait(&bar, 0u, limit_ns, nullptr)) {
+        atomicOr(flags, (unsigned)ECHO_FLAG_TIMEOUT);
+    }
+}
+
 }  // namespace echo_dev

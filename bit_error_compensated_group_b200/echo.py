@@ -17,6 +17,7 @@ from . import _build
 
 ECHO_OK, ECHO_EINVAL, ECHO_ECUDA, ECHO_ERANGE, ECHO_ETIMEOUT = 0, 1, 2, 3, 4
 ECHO_FLAG_RANGE = 1
+ECHO_FLAG_TIMEOUT = 2
 ECHO_MAX_RANKS = 64
 
 LIB_PATH = _build.LIB
@@ -71,6 +72,8 @@ def lib() -> ctypes.CDLL:
         L.echo_phase_reduce.restype = I
         L.echo_phase_gather.argtypes = [PP, V, I, V]
         L.echo_phase_gather.restype = I
+        L.echo_check_watchdog.argtypes = [V, ctypes.c_uint32, V]
+        L.echo_check_watchdog.restype = I
         L.echo_get_status.argtypes = [V, V, ctypes.POINTER(ctypes.c_uint32)]
         L.echo_get_status.restype = I
         L.echo_free.argtypes = [V]
@@ -160,11 +163,15 @@ def echo_phase_gather(outputs: Sequence, st, bits: int, stream=None) -> None:
     _check(lib().echo_phase_gather(_ptr_array(outputs), st, bits, _stream(stream)), "echo_phase_gather")
 
 
+def echo_check_watchdog(st, limit_us: int, stream=None) -> None:
+    _check(lib().echo_check_watchdog(st, limit_us, _stream(stream)), "echo_check_watchdog")
+
+
 def echo_get_status(st, stream=None):
     """Returns (status, flags); synchronizes the stream."""
     flags = ctypes.c_uint32(0)
     rc = lib().echo_get_status(st, _stream(stream), ctypes.byref(flags))
-    if rc not in (ECHO_OK, ECHO_ERANGE):
+    if rc not in (ECHO_OK, ECHO_ERANGE, ECHO_ETIMEOUT):
         raise EchoError(rc, "echo_get_status")
     return rc, int(flags.value)
 

@@ -202,6 +202,18 @@ ECHO_API int echo_phase_gather(void* const* outputs, echo_state* st, int bits, e
  */
 ECHO_API int echo_get_status(echo_state* st, echo_stream_t stream, uint32_t* device_flags);
 
+/*
+ * Failure-detection self-check (no counterpart on the pages; part of this
+ * library's error reporting). Launches one thread that waits, with the same
+ * bounded wait the bulk-copy pipelines use, on a barrier that nothing ever
+ * completes. After limit_us microseconds (1 .. 10^7) the wait gives up, the
+ * kernel sets ECHO_FLAG_TIMEOUT in st's flag word and returns; the next
+ * echo_get_status returns ECHO_ETIMEOUT and the context stays usable.
+ * Asynchronous on `stream`. ECHO_EINVAL on a NULL handle or a limit out of
+ * range, ECHO_ECUDA when the launch fails.
+ */
+ECHO_API int echo_check_watchdog(echo_state* st, uint32_t limit_us, echo_stream_t stream);
+
 /* Release the host handle (never the caller's device buffers). NULL is a no-op. */
 ECHO_API int echo_free(echo_state* st);
 

@@ -49,7 +49,7 @@ def _gpu_inputs_u16(inputs, c):
 
 def _compare_sampled(ar, outputs, S: Sampled, orcs, bits, site):
     a2a_c, a2a_p, g_c, g_p = ar.payload_views(bits)
-    el_v, es_v = ar.ema_views()
+    el_v, es_v = ar.ema_views() if ar.state is not None else (None, None)
     w = S.w
     for (j0, jc), orc in zip(S.ranges, orcs):
         c = S.cols(j0, jc)
