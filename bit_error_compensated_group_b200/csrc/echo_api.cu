@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <new>
 
 #include "echo.h"
@@ -308,6 +309,89 @@ int echo_free(echo_state* st) {
     return ECHO_OK;
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// No-allocation entry point: payloads and flag word in a fixed scratch array.
+
+// Scratch of echo_allreduce_sim_noalloc. In host code this name is only a
+// stand-in for the symbol; its device address comes from cudaGetSymbolAddress.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[ECHO_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kNoallocMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+uint8_t* g_noalloc_ptr[kNoallocMaxDevices];   // device address of the scratch, per device
+int g_noalloc_sms[kNoallocMaxDevices];
+
+// Once per device, with that device current: the scratch's device address and
+// the SM count.
+int noalloc_setup(int dev, uint8_t** ptr, int* sms) {
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return ECHO_ECUDA;
+        int count = 0;
+        if (cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return ECHO_ECUDA;
+        g_noalloc_sms[dev] = count;
+        g_noalloc_ptr[dev] = static_cast<uint8_t*>(p);
+    }
+    *ptr = g_noalloc_ptr[dev];
+    *sms = g_noalloc_sms[dev];
+    return ECHO_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int echo_allreduce_sim_noalloc(const void* const* inputs, void* const* outputs, void* state_dev, int64_t n, int P,
+                               int bits, int group, float eta, float alpha_long, float alpha_short, float w,
+                               uint32_t* flags_out, echo_stream_t stream) {
+    if (!inputs || !outputs) return ECHO_EINVAL;
+    echo_layout L;
+    if (!layout(n, P, group, bits, bits, &L)) return ECHO_EINVAL;
+    if (!valid_feedback(eta, alpha_long, alpha_short, w)) return ECHO_EINVAL;
+    if (state_dev && !aligned(state_dev, 16)) return ECHO_EINVAL;
+    if (L.workspace_bytes > (uint64_t)ECHO_NOALLOC_SCRATCH_BYTES) return ECHO_ENOSPACE;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoallocMaxDevices) return ECHO_ECUDA;
+    uint8_t* scratch = nullptr;
+    int sms = 0;
+    if (int rc = noalloc_setup(dev, &scratch, &sms)) return rc;
+    echo_state st;   // on the stack: describes the call, owns nothing
+    st.n = n;
+    st.P = P;
+    st.group = group;
+    st.max_bits = bits;
+    st.G = L.groups;
+    st.S = L.state_stride;
+    st.state = static_cast<float*>(state_dev);
+    st.workspace = scratch;
+    st.device = dev;
+    st.sm_count = sms;
+    echo_dev::Args a;
+    if (!make_args(&st, bits, inputs, outputs, eta, alpha_long, alpha_short, w, &a)) return ECHO_EINVAL;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(scratch + L.flags_offset, 0, sizeof(uint32_t), s) != cudaSuccess) return ECHO_ECUDA;
+    if (P >= 2) {
+        if (int rc = launch(Stage::Quantize, bits, a, &st, s)) return rc;
+    }
+    if (int rc = launch(Stage::Reduce, bits, a, &st, s)) return rc;
+    if (P >= 2) {
+        if (int rc = launch(Stage::Gather, bits, a, &st, s)) return rc;
+    }
+    if (flags_out) {
+        uint32_t f = 0;
+        if (cudaStreamSynchronize(s) != cudaSuccess) return ECHO_ECUDA;
+        if (cudaMemcpy(&f, scratch + L.flags_offset, sizeof(f), cudaMemcpyDeviceToHost) != cudaSuccess)
+            return ECHO_ECUDA;
+        *flags_out = f;
+    }
+    return ECHO_OK;
+}
+
 const char* echo_status_string(int status) {
     switch (status) {
         case ECHO_OK: return "ok";
@@ -315,6 +399,7 @@ const char* echo_status_string(int status) {
         case ECHO_ECUDA: return "CUDA error";
         case ECHO_ERANGE: return "value outside the fp16 parameter range";
         case ECHO_ETIMEOUT: return "device wait timed out";
+        case ECHO_ENOSPACE: return "message too large for the no-allocation scratch (ECHO_NOALLOC_SCRATCH_BYTES)";
     }
     return "unknown status";
 }

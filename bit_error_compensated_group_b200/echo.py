@@ -15,7 +15,8 @@ import torch
 
 from . import _build
 
-ECHO_OK, ECHO_EINVAL, ECHO_ECUDA, ECHO_ERANGE, ECHO_ETIMEOUT = 0, 1, 2, 3, 4
+ECHO_OK, ECHO_EINVAL, ECHO_ECUDA, ECHO_ERANGE, ECHO_ETIMEOUT, ECHO_ENOSPACE = 0, 1, 2, 3, 4, 5
+ECHO_NOALLOC_SCRATCH_BYTES = 16 << 20
 ECHO_FLAG_RANGE = 1
 ECHO_FLAG_TIMEOUT = 2
 ECHO_MAX_RANKS = 64
@@ -174,6 +175,26 @@ def echo_get_status(st, stream=None):
     if rc not in (ECHO_OK, ECHO_ERANGE, ECHO_ETIMEOUT):
         raise EchoError(rc, "echo_get_status")
     return rc, int(flags.value)
+
+
+def echo_allreduce_sim_noalloc(inputs: Sequence, outputs: Sequence, state, n: int, P: int, bits: int,
+                               group: int, eta: float, alpha_long: float, alpha_short: float, w: float,
+                               stream=None, read_flags: bool = True) -> Optional[int]:
+    """echo_allreduce_sim for callers that cannot allocate device memory:
+    the payloads live in the library's fixed scratch array, there is no
+    handle, and the caller passes the EMA state tensor (or None for no
+    feedback). Returns the call's ECHO_FLAG_* bits when `read_flags` (which
+    synchronizes the stream), else None."""
+    f = lib().echo_allreduce_sim_noalloc
+    V, I, I64, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
+    PP = ctypes.POINTER(ctypes.c_void_p)
+    f.argtypes = [PP, PP, V, I64, I, I, I, F, F, F, F, ctypes.POINTER(ctypes.c_uint32), V]
+    f.restype = I
+    flags = ctypes.c_uint32(0)
+    rc = f(_ptr_array(inputs), _ptr_array(outputs), _ptr(state), n, P, bits, group, eta, alpha_long, alpha_short,
+           w, ctypes.byref(flags) if read_flags else None, _stream(stream))
+    _check(rc, "echo_allreduce_sim_noalloc")
+    return int(flags.value) if read_flags else None
 
 
 def echo_free(st) -> None:

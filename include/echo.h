@@ -74,7 +74,9 @@ typedef enum echo_status {
     ECHO_EINVAL = 1,     /* bad argument; nothing was enqueued */
     ECHO_ECUDA = 2,      /* a CUDA runtime call or kernel launch failed */
     ECHO_ERANGE = 3,     /* returned by echo_get_status when ECHO_FLAG_RANGE is set */
-    ECHO_ETIMEOUT = 4    /* returned by echo_get_status when ECHO_FLAG_TIMEOUT is set */
+    ECHO_ETIMEOUT = 4,   /* returned by echo_get_status when ECHO_FLAG_TIMEOUT is set */
+    ECHO_ENOSPACE = 5    /* echo_allreduce_sim_noalloc: the message needs more
+                            scratch than ECHO_NOALLOC_SCRATCH_BYTES */
 } echo_status;
 
 /* Same object as cudaStream_t; NULL is the legacy default stream. */
@@ -213,6 +215,57 @@ ECHO_API int echo_get_status(echo_state* st, echo_stream_t stream, uint32_t* dev
  * range, ECHO_ECUDA when the launch fails.
  */
 ECHO_API int echo_check_watchdog(echo_state* st, uint32_t limit_us, echo_stream_t stream);
+
+/* Size of the fixed scratch array used by echo_allreduce_sim_noalloc. It is
+ * device memory that every GPU which loads this library holds until the
+ * process exits. */
+#define ECHO_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * echo_allreduce_sim for callers that cannot allocate device memory. The
+ * pages describe no such variant; this entry point has no counterpart in the
+ * paper.
+ *
+ * Who needs it: code that may not allocate device memory at the point where
+ * it runs the all-reduce -- a process whose framework reserved the device
+ * memory for its own pools at start-up (a serving engine that pre-allocates
+ * its KV cache, say), or a latency-critical path that cannot afford the
+ * implicit device-wide synchronization of cudaMalloc/cudaFree. Such callers
+ * cannot provide the workspace echo_init_state needs. Here the all-to-all and
+ * all-gather payloads and the flag word live in a fixed scratch array inside
+ * this library (ECHO_NOALLOC_SCRATCH_BYTES, 16 MiB), there is no handle, and
+ * nothing is allocated -- not by this call, not by the caller. The kernels and
+ * the arithmetic are those of echo_allreduce_sim, so the results are
+ * identical.
+ *
+ *   inputs, outputs, n, P, bits, group, eta, alpha_long, alpha_short, w,
+ *   stream     as for echo_allreduce_sim
+ *   state_dev  NULL (no feedback), or the caller's EMA state: device memory of
+ *              echo_state_bytes(n, P, group) bytes, 16-byte aligned, in the
+ *              layout documented at echo_state_bytes. The caller zeroes it
+ *              before the first call and keeps it between calls.
+ *   flags_out  NULL, or a host word that receives this call's ECHO_FLAG_*
+ *              bits; when given, the call synchronizes `stream` before
+ *              returning.
+ * Limit: the payloads of the message must fit the scratch:
+ *   echo_query_layout(n, P, group, bits, bits).workspace_bytes, about
+ *   (P + 1) * ceil(n / group) * (group * bits / 8 + 4) bytes, must not exceed
+ *   ECHO_NOALLOC_SCRATCH_BYTES (for P = 8, 4 bits, groups of 128: up to about
+ *   3.4 M elements per rank). A larger message returns ECHO_ENOSPACE before
+ *   anything is enqueued.
+ * Set-up: the first call on a device looks up, with that device current, the
+ *   device address of the scratch array and the device's SM count, and keeps
+ *   them for later calls. Make that first call on each device before any
+ *   stream capture on it.
+ * Sharing: all calls on a device use the same scratch, which keeps the last
+ *   call's payloads; each call clears the flag word before its kernels run.
+ *   Calls that overlap on the GPU (on streams with no ordering between them)
+ *   race on the scratch and give undefined results: order them.
+ * Errors: those of echo_allreduce_sim, plus ECHO_ENOSPACE.
+ */
+ECHO_API int echo_allreduce_sim_noalloc(const void* const* inputs, void* const* outputs, void* state_dev,
+                                        int64_t n, int P, int bits, int group, float eta, float alpha_long,
+                                        float alpha_short, float w, uint32_t* flags_out, echo_stream_t stream);
 
 /* Release the host handle (never the caller's device buffers). NULL is a no-op. */
 ECHO_API int echo_free(echo_state* st);
