@@ -108,10 +108,10 @@ int launch_stage(Stage stage, const echo_dev::Args& a, const echo_state* st, cud
             break;
         }
         case Stage::Gather: {
-            auto k = echo_dev::k_gather<GROUP, BITS>;
+            auto k = echo_dev::k_gather_tma<GROUP, BITS>;
             static int grid = 0;
-            if (grid == 0) grid = grid_for(k, st);
-            k<<<grid, echo_dev::kThreads, 0, s>>>(a);
+            if (grid == 0) grid = grid_for(k, st, echo_dev::kGatherThreads, echo_dev::kGatherSmem);
+            k<<<grid, echo_dev::kGatherThreads, echo_dev::kGatherSmem, s>>>(a);
             break;
         }
     }

@@ -1,28 +1,35 @@
-// echo_kernels.cuh -- sm_100a kernels of the Echo all-reduce simulation.
+// echo_kernels.cuh -- shared device helpers of the Echo all-reduce
+// simulation, and the scalar per-group paths.
 //
-// Three streaming kernels, one per stage of the restructured all-reduce of
-// the Echo explainer ("Echoの仕組み①": all-to-all of 4-bit non-owned
-// segments, high-precision sum at the owner, 4-bit all-gather), with the
-// feedback of "Echoの仕組み②" fused into the passes that read the inputs:
+// The call is three kernels (echo_pipeline.cuh), one per stage of the
+// restructured all-reduce of the Echo explainer ("Echoの仕組み①": all-to-all
+// of 4-bit non-owned segments, high-precision sum at the owner, 4-bit
+// all-gather), with the feedback of "Echoの仕組み②" fused into the passes
+// that read the inputs:
 //
-//   k_quantize  every rank's non-owned groups: x' = x + c, group min/max,
-//               fp16 {s, z}, packed codes -> all-to-all payload; residual
-//               x' - x_hat -> both EMAs.
-//   k_reduce    every group at its owner: x'_owner + dequantized payloads in
-//               rank order (binary32), requantize -> all-gather payload;
-//               residual sum - y -> the owner's EMAs.
-//   k_gather    every group: dequantize the gathered payload once, write the
-//               bf16 result into all P outputs.
+//   quantize  every rank's non-owned groups: x' = x + c, group min/max,
+//             fp16 {s, z}, packed codes -> all-to-all payload; residual
+//             x' - x_hat -> both EMAs.
+//   reduce    every group at its owner: x'_owner + dequantized payloads in
+//             rank order (binary32), requantize -> all-gather payload;
+//             residual sum - y -> the owner's EMAs.
+//   gather    every group: dequantize the gathered payload once, write the
+//             bf16 result into all P outputs.
 //
-// No tensor cores: this is a streaming codec, bound by HBM bandwidth. Thread
-// layout: a group of GROUP elements is handled by L = GROUP/8 lanes; lane t
-// holds the two 4-element chunks t and t+L, so every load and store
-// instruction of a group covers one contiguous span (bf16 chunk = 8 B,
-// binary32 chunk = 16 B). Group min/max use xor-shuffles inside the L lanes.
+// This file holds the argument block, the per-group grid (fp16 zero rounded
+// toward -inf from the minimum, fp16 step rounded toward +inf from
+// (max - z)/Q), and quantize_range / reduce_range: the same stages written
+// one element at a time with global loads and stores guarded against the
+// message end. The kernels use them for a partial last group (its byte size
+// is not a multiple of 16, so bulk copies cannot move it).
 //
-// Arithmetic is binary32 with explicit round-to-nearest intrinsics
-// (__fadd_rn / __fmul_rn / __fdiv_rn never contract into FMA) and the
-// directed fp16 conversions, so results are bit-reproducible.
+// Thread layout: a group of GROUP elements is handled by L = GROUP/8 lanes;
+// lane t holds the two 4-element chunks t and t+L, so every load and store
+// instruction of a group covers one contiguous span. Group min/max use
+// xor-shuffles inside the L lanes. Arithmetic is binary32 with explicit
+// round-to-nearest intrinsics (__fadd_rn / __fmul_rn / __fdiv_rn never
+// contract into FMA) and the directed fp16 conversions, so results are
+// bit-reproducible.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -287,18 +294,6 @@ __device__ __forceinline__ void quantize_range(const Args& a, int r, long long j
     }
 }
 
-template <int GROUP, int BITS>
-__global__ void __launch_bounds__(kThreads) k_quantize(const Args a) {
-    const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
-    for (int r = 0; r < a.P; ++r) {
-        const long long lo = (long long)r * a.G / a.P;          // rank r owns [lo, hi)
-        const long long hi = (long long)(r + 1) * a.G / a.P;
-        quantize_range<GROUP, BITS>(a, r, 0, lo, warp, nwarps);
-        quantize_range<GROUP, BITS>(a, r, hi, a.G, warp, nwarps);
-    }
-}
-
 // Stage 2: owner o sums and requantizes its groups [j_begin, j_end).
 template <int GROUP, int BITS>
 __device__ __forceinline__ void reduce_range(const Args& a, int o, long long j_begin, long long j_end,
@@ -428,61 +423,13 @@ __device__ __forceinline__ void reduce_range(const Args& a, int o, long long j_b
     }
 }
 
-template <int GROUP, int BITS>
-__global__ void __launch_bounds__(kThreads) k_reduce(const Args a) {
-    const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
-    for (int o = 0; o < a.P; ++o) {
-        const long long lo = (long long)o * a.G / a.P;
-        const long long hi = (long long)(o + 1) * a.G / a.P;
-        reduce_range<GROUP, BITS>(a, o, lo, hi, warp, nwarps);
-    }
-}
-
-// Stage 3: decode the gathered payload once per group, write all P outputs.
-// No group reduction here, so lane t simply owns the 8 contiguous elements
-// [8t, 8t + 8) of its group: one 32-bit (4-bit codes) or 64-bit (8-bit codes)
-// load, and one 16-byte store per output.
+// Stage 3 helper: lane t of a group owns the 8 contiguous elements
+// [8t, 8t + 8): their codes are one 32-bit (4-bit codes) or 64-bit (8-bit
+// codes) word.
 template <int BITS>
 __device__ __forceinline__ uint2 load_codes8(const uint8_t* group_codes, int t) {
     if (BITS == 4) return make_uint2(*reinterpret_cast<const uint32_t*>(group_codes + 4 * t), 0u);
     return *reinterpret_cast<const uint2*>(group_codes + 8 * t);
-}
-
-template <int BITS>
-__device__ __forceinline__ int code8(uint2 w, int k) {
-    return BITS == 4 ? (int)((w.x >> (4 * k)) & 0xfu) : (int)(((k < 4 ? w.x : w.y) >> (8 * (k & 3))) & 0xffu);
-}
-
-template <int GROUP, int BITS>
-__global__ void __launch_bounds__(kThreads) k_gather(const Args a) {
-    constexpr int L = GROUP / 8, GPW = 32 / L, CB = GROUP * BITS / 8;
-    const int lane = threadIdx.x & 31;
-    const int sub = lane / L, t = lane % L;
-    const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
-    for (long long j0 = warp * GPW; j0 < a.G; j0 += nwarps * GPW) {
-        const long long j = j0 + sub;
-        if (j >= a.G) continue;   // no shuffles below
-        const uint2 w = load_codes8<BITS>(a.g_codes + (size_t)j * CB, t);
-        const uint32_t p = a.g_params[j];
-        const float s = param_s(p), z = param_z(p);
-        uint32_t yb[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) yb[k] = f2bf16(decode(code8<BITS>(w, k), s, z));
-        const long long e = j * GROUP + 8 * t;
-        if (e + 8 <= a.n) {
-            const uint4 v = make_uint4(yb[0] | (yb[1] << 16), yb[2] | (yb[3] << 16), yb[4] | (yb[5] << 16),
-                                       yb[6] | (yb[7] << 16));
-            for (int r = 0; r < a.P; ++r) __stcs(reinterpret_cast<uint4*>(a.out[r] + e), v);
-        } else {
-            for (int r = 0; r < a.P; ++r) {
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    if (e + k < a.n) a.out[r][e + k] = (uint16_t)yb[k];
-            }
-        }
-    }
 }
 
 }  // namespace echo_dev

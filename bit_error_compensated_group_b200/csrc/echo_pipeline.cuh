@@ -235,6 +235,180 @@ __device__ __forceinline__ void produce(const Args& a, const PipeShared& p, RunW
 
 // ------------------------------------------------------------ quantize
 
+// ------------------------------------------------------------ packed math
+//
+// The tile paths compute two elements per instruction with the sm_100 paired
+// binary32 operations (add/fma.rn.f32x2: each component rounds exactly like
+// the scalar operation) where that cannot change a single bit:
+//  * dequantization code*s + z uses one fused multiply-add: code <= 255 and
+//    s is an fp16 value (11-bit significand), so code*s is exact in binary32
+//    and rounding once gives the same result as multiply-then-add;
+//  * a code is turned into an exact float by placing it in the mantissa of
+//    2^23 (bit pattern 0x4B000000 | code) and subtracting 2^23;
+//  * additions whose operands are not products (rank-ordered sums, x' - x_hat).
+// Every product that the definition rounds before an addition (compensation,
+// the quantizer's (v - z) * inv, both EMA terms) is a scalar __fmul_rn: the
+// assembler may fuse a paired multiply into the paired add that consumes it,
+// even with an explicit .rn (seen on sm_100a: a tie rounded the other way),
+// while scalar operations with an explicit rounding keep their own rounding.
+// Round-half-even of u in [0, 2^22) is (u + 2^23): binary32 spacing there is
+// 1, so the addition itself rounds u to the nearest integer, ties to even,
+// and the code sits in the low mantissa bits.
+// Group min/max use min.NaN / max.NaN so that a NaN anywhere in a group
+// reaches the range check.
+
+constexpr float kMagic = 8388608.0f;   // 2^23
+
+// Paired binary32 operations (PTX add/mul/fma.rn.f32x2).
+__device__ __forceinline__ float2 add2_rn(float2 a, float2 b) {
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rr;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rr, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, rr;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+
+__device__ __forceinline__ float2 fma2_rn(float2 a, float2 b, float2 c) {
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rc, rr;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rr, ra, rb, rc;\n\t"
+        "mov.b64 {%0, %1}, rr;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return r;
+}
+
+__device__ __forceinline__ float2 splat(float v) { return make_float2(v, v); }
+
+// round a pair to bf16 (nearest-even); element 0 in the low half
+__device__ __forceinline__ uint32_t bf16x2_rn(float2 v) {
+    const __nv_bfloat162 b = __float22bfloat162_rn(v);
+    return *reinterpret_cast<const uint32_t*>(&b);
+}
+
+__device__ __forceinline__ float nan_min(float a, float b) {
+    float r;
+    asm("min.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+
+__device__ __forceinline__ float nan_max(float a, float b) {
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+
+// Packed quantization grid of one group (same values as make_grid).
+struct GridP {
+    float2 s, z, ns, nz, inv;
+    uint32_t param;
+    bool bad;   // a value outside [-65504, 65504] or a NaN
+};
+
+template <int L, int Q>
+__device__ __forceinline__ GridP make_grid_p(float lane_min, float lane_max) {
+    float mn = lane_min, mx = lane_max;
+#pragma unroll
+    for (int o = L / 2; o > 0; o >>= 1) {
+        mn = nan_min(mn, __shfl_xor_sync(kFull, mn, o));
+        mx = nan_max(mx, __shfl_xor_sync(kFull, mx, o));
+    }
+    GridP g;
+    g.bad = !(mn >= -65504.0f && mx <= 65504.0f);
+    mn = __fadd_rn(mn, 0.0f);   // -0 -> +0
+    mx = __fadd_rn(mx, 0.0f);
+    const __half zh = __float2half_rd(mn);
+    const float z = __half2float(zh);
+    const __half sh = __float2half_ru(__fdiv_rn(__fsub_rn(mx, z), (float)Q));
+    const float s = __half2float(sh);
+    const float inv = (s != 0.0f) ? __fdiv_rn(1.0f, s) : 0.0f;
+    g.s = splat(s);
+    g.z = splat(z);
+    g.ns = splat(-s);
+    g.nz = splat(-z);
+    g.inv = splat(inv);
+    g.param = (uint32_t)__half_as_ushort(sh) | ((uint32_t)__half_as_ushort(zh) << 16);
+    return g;
+}
+
+// 2^23 + code for a pair of values: code = round_half_even((v - z) * inv)
+__device__ __forceinline__ float2 encode2(float2 v, const GridP& g) {
+    const float2 d = add2_rn(v, g.nz);   // v - z
+    return make_float2(__fadd_rn(__fmul_rn(d.x, g.inv.x), kMagic), __fadd_rn(__fmul_rn(d.y, g.inv.y), kMagic));
+}
+
+// four codes (2^23 + code each) -> one chunk of packed codes
+template <int BITS>
+__device__ __forceinline__ uint32_t pack_codes4(float2 t01, float2 t23) {
+    constexpr uint32_t Q = (1u << BITS) - 1u;
+    const uint32_t c0 = __float_as_uint(t01.x) & Q, c1 = __float_as_uint(t01.y) & Q;
+    const uint32_t c2 = __float_as_uint(t23.x) & Q, c3 = __float_as_uint(t23.y) & Q;
+    if (BITS == 4) return c0 | (c1 << 4) | (c2 << 8) | (c3 << 12);
+    return c0 | (c1 << 8) | (c2 << 16) | (c3 << 24);
+}
+
+// one chunk of packed codes -> the four codes as exact floats
+template <int BITS>
+__device__ __forceinline__ void unpack_codes4(uint32_t w, float2& q01, float2& q23) {
+    uint32_t m0, m1, m2, m3;
+    if (BITS == 4) {
+        const uint32_t lo = w & 0x0F0Fu;          // codes 0 and 2 in bytes 0 and 1
+        const uint32_t hi = (w >> 4) & 0x0F0Fu;   // codes 1 and 3
+        m0 = __byte_perm(lo, 0x4B000000u, 0x7650);
+        m1 = __byte_perm(hi, 0x4B000000u, 0x7650);
+        m2 = __byte_perm(lo, 0x4B000000u, 0x7651);
+        m3 = __byte_perm(hi, 0x4B000000u, 0x7651);
+    } else {
+        m0 = __byte_perm(w, 0x4B000000u, 0x7650);
+        m1 = __byte_perm(w, 0x4B000000u, 0x7651);
+        m2 = __byte_perm(w, 0x4B000000u, 0x7652);
+        m3 = __byte_perm(w, 0x4B000000u, 0x7653);
+    }
+    q01 = add2_rn(make_float2(__uint_as_float(m0), __uint_as_float(m1)), splat(-kMagic));
+    q23 = add2_rn(make_float2(__uint_as_float(m2), __uint_as_float(m3)), splat(-kMagic));
+}
+
+// x' = x + eta * (w * e_short + (1 - w) * e_long), two elements (scalar products)
+__device__ __forceinline__ float2 inject2(float2 x, float2 el, float2 es, const Args& a) {
+    return make_float2(inject(x.x, el.x, es.x, a), inject(x.y, el.y, es.y, a));
+}
+
+// e <- (1 - alpha) * e + alpha * rho, two elements (scalar products)
+__device__ __forceinline__ float2 ema2(float2 e, float2 rho, float keep, float alpha) {
+    return make_float2(ema(e.x, rho.x, keep, alpha), ema(e.y, rho.y, keep, alpha));
+}
+
+__device__ __forceinline__ void load_x8_smem(const uint16_t* xs, int c0, int c1, float2 v[4]) {
+    const uint2 u0 = *reinterpret_cast<const uint2*>(xs + c0);
+    const uint2 u1 = *reinterpret_cast<const uint2*>(xs + c1);
+    v[0] = make_float2(bf16_lo(u0.x), bf16_hi(u0.x));
+    v[1] = make_float2(bf16_lo(u0.y), bf16_hi(u0.y));
+    v[2] = make_float2(bf16_lo(u1.x), bf16_hi(u1.x));
+    v[3] = make_float2(bf16_lo(u1.y), bf16_hi(u1.y));
+}
+
+__device__ __forceinline__ void load_f8_smem(const float* p, int c0, int c1, float2 v[4]) {
+    const float4 a = *reinterpret_cast<const float4*>(p + c0);
+    const float4 b = *reinterpret_cast<const float4*>(p + c1);
+    v[0] = make_float2(a.x, a.y);
+    v[1] = make_float2(a.z, a.w);
+    v[2] = make_float2(b.x, b.y);
+    v[3] = make_float2(b.z, b.w);
+}
+
+__device__ __forceinline__ void store_f4_pair(float* p, float2 lo, float2 hi) {
+    __stcs(reinterpret_cast<float4*>(p), make_float4(lo.x, lo.y, hi.x, hi.y));
+}
+
+// ------------------------------------------------------------ quantize
+
 template <int GROUP, int BITS>
 __device__ __forceinline__ void quantize_tile_group(const Args& a, const uint8_t* st, const Tile& t, int gi,
                                                     bool act) {
@@ -243,60 +417,47 @@ __device__ __forceinline__ void quantize_tile_group(const Args& a, const uint8_t
     const LN ln;
     const int r = t.rank;
     const long long j = t.j0 + gi;
+    const int c0 = 4 * ln.chunk(0), c1 = 4 * ln.chunk(1);
     const uint16_t* xs = reinterpret_cast<const uint16_t*>(st) + gi * GROUP;
     const float* els = reinterpret_cast<const float*>(st + kTileElems * 2) + gi * GROUP;
     const float* ess = reinterpret_cast<const float*>(st + kTileElems * 6) + gi * GROUP;
-    float v[8], el[8], es[8];
+    float2 v[4], el[4], es[4];
     float lmin = __int_as_float(0x7f800000), lmax = -__int_as_float(0x7f800000);
-    bool bad = false;
     if (act) {
+        load_x8_smem(xs, c0, c1, v);
+        if (a.state) {
+            load_f8_smem(els, c0, c1, el);
+            load_f8_smem(ess, c0, c1, es);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int c = 4 * ln.chunk(h);
-            const uint2 u = *reinterpret_cast<const uint2*>(xs + c);
-            v[4 * h + 0] = bf16_lo(u.x);
-            v[4 * h + 1] = bf16_hi(u.x);
-            v[4 * h + 2] = bf16_lo(u.y);
-            v[4 * h + 3] = bf16_hi(u.y);
-            if (a.state) {
-                const float4 l4 = *reinterpret_cast<const float4*>(els + c);
-                const float4 s4 = *reinterpret_cast<const float4*>(ess + c);
-                el[4 * h + 0] = l4.x; el[4 * h + 1] = l4.y; el[4 * h + 2] = l4.z; el[4 * h + 3] = l4.w;
-                es[4 * h + 0] = s4.x; es[4 * h + 1] = s4.y; es[4 * h + 2] = s4.z; es[4 * h + 3] = s4.w;
-            }
+            for (int p = 0; p < 4; ++p) v[p] = inject2(v[p], el[p], es[p], a);
         }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            if (a.state) v[i] = inject(v[i], el[i], es[i], a);
-            lmin = fminf(lmin, v[i]);
-            lmax = fmaxf(lmax, v[i]);
-            bad |= outside_fp16_domain(v[i]);
+        for (int p = 0; p < 4; ++p) {
+            lmin = nan_min(lmin, nan_min(v[p].x, v[p].y));
+            lmax = nan_max(lmax, nan_max(v[p].x, v[p].y));
         }
     }
-    raise_flags(a, bad);
-    const Grid g = make_grid<L, Q>(lmin, lmax);
+    const GridP g = make_grid_p<L, Q>(lmin, lmax);
+    raise_flags(a, act && g.bad);
     if (!act) return;
     uint8_t* codes = a.a2a_codes + ((size_t)r * a.G + j) * CB;
     float* el_g = a.state ? a.state + (size_t)r * 2 * a.S + j * GROUP : nullptr;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-        const int c = 4 * ln.chunk(h);
-        int q[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int i = 4 * h + k;
-            q[k] = encode<Q>(v[i], g);
-            if (a.state) {
-                const float rho = __fsub_rn(v[i], decode(q[k], g.s, g.z));
-                el[i] = ema(el[i], rho, a.keep_long, a.a_long);
-                es[i] = ema(es[i], rho, a.keep_short, a.a_short);
-            }
-        }
-        store_chunk_codes<BITS>(codes, ln.chunk(h), pack4<BITS>(q));
+        const float2 t01 = encode2(v[2 * h], g);
+        const float2 t23 = encode2(v[2 * h + 1], g);
+        store_chunk_codes<BITS>(codes, ln.chunk(h), pack_codes4<BITS>(t01, t23));
         if (a.state) {
-            __stcs(reinterpret_cast<float4*>(el_g + c), make_float4(el[4 * h], el[4 * h + 1], el[4 * h + 2], el[4 * h + 3]));
-            __stcs(reinterpret_cast<float4*>(el_g + a.S + c),
-                   make_float4(es[4 * h], es[4 * h + 1], es[4 * h + 2], es[4 * h + 3]));
+            // residual x' - x_hat with x_hat = code*s + z (fused: code*s is exact)
+            const float2 q01 = add2_rn(t01, splat(-kMagic));
+            const float2 q23 = add2_rn(t23, splat(-kMagic));
+            const float2 rho01 = add2_rn(v[2 * h], fma2_rn(q01, g.ns, g.nz));
+            const float2 rho23 = add2_rn(v[2 * h + 1], fma2_rn(q23, g.ns, g.nz));
+            const int c = h ? c1 : c0;
+            store_f4_pair(el_g + c, ema2(el[2 * h], rho01, a.keep_long, a.a_long),
+                          ema2(el[2 * h + 1], rho23, a.keep_long, a.a_long));
+            store_f4_pair(el_g + a.S + c, ema2(es[2 * h], rho01, a.keep_short, a.a_short),
+                          ema2(es[2 * h + 1], rho23, a.keep_short, a.a_short));
         }
     }
     if (ln.t == 0) a.a2a_params[(size_t)r * a.G + j] = g.param;
@@ -345,35 +506,28 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
                                                   bool act) {
     using LN = Lane<GROUP>;
     constexpr int L = LN::L, Q = (1 << BITS) - 1, CB = GROUP * BITS / 8;
-    constexpr int RB = 8;
+    constexpr int RB = 8;   // ranks whose payload loads are issued together
     const LN ln;
     const int o = t.rank;
     const long long j = t.j0 + gi;
+    const int c0 = 4 * ln.chunk(0), c1 = 4 * ln.chunk(1);
     const uint16_t* xs = reinterpret_cast<const uint16_t*>(st) + gi * GROUP;
     const float* els = reinterpret_cast<const float*>(st + kTileElems * 2) + gi * GROUP;
     const float* ess = reinterpret_cast<const float*>(st + kTileElems * 6) + gi * GROUP;
-    float xo[8], acc[8];
+    float2 xo[4], acc[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) xo[i] = acc[i] = 0.0f;
+    for (int p = 0; p < 4; ++p) xo[p] = acc[p] = make_float2(0.0f, 0.0f);
     if (act) {
+        load_x8_smem(xs, c0, c1, xo);
+        if (a.state) {
+            float2 el[4], es[4];
+            load_f8_smem(els, c0, c1, el);
+            load_f8_smem(ess, c0, c1, es);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int c = 4 * ln.chunk(h);
-            const uint2 u = *reinterpret_cast<const uint2*>(xs + c);
-            xo[4 * h + 0] = bf16_lo(u.x);
-            xo[4 * h + 1] = bf16_hi(u.x);
-            xo[4 * h + 2] = bf16_lo(u.y);
-            xo[4 * h + 3] = bf16_hi(u.y);
-            if (a.state) {
-                const float4 l4 = *reinterpret_cast<const float4*>(els + c);
-                const float4 s4 = *reinterpret_cast<const float4*>(ess + c);
-                xo[4 * h + 0] = inject(xo[4 * h + 0], l4.x, s4.x, a);
-                xo[4 * h + 1] = inject(xo[4 * h + 1], l4.y, s4.y, a);
-                xo[4 * h + 2] = inject(xo[4 * h + 2], l4.z, s4.z, a);
-                xo[4 * h + 3] = inject(xo[4 * h + 3], l4.w, s4.w, a);
-            }
+            for (int p = 0; p < 4; ++p) xo[p] = inject2(xo[p], el[p], es[p], a);
         }
     }
+    // binary32 sum in rank order 0..P-1: own x' unquantized, others decoded
     for (int r0 = 0; r0 < a.P; r0 += RB) {
         uint32_t cw[RB][2];
         uint32_t pw[RB];
@@ -393,71 +547,83 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
 #pragma unroll
         for (int k = 0; k < RB; ++k) {
             const int r = r0 + k;
-            if (r < a.P) {
-                const float s = param_s(pw[k]);
-                const float z = param_z(pw[k]);
+            if (r >= a.P) break;
+            float2 term[4];
+            if (r == o) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float term = (r == o) ? xo[i] : decode(unpack1<BITS>(cw[k][i >> 2], i & 3), s, z);
-                    acc[i] = (r == 0) ? term : __fadd_rn(acc[i], term);
+                for (int p = 0; p < 4; ++p) term[p] = xo[p];
+            } else {
+                const float2 s2 = splat(param_s(pw[k]));
+                const float2 z2 = splat(param_z(pw[k]));
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    float2 q01, q23;
+                    unpack_codes4<BITS>(cw[k][h], q01, q23);
+                    term[2 * h] = fma2_rn(q01, s2, z2);
+                    term[2 * h + 1] = fma2_rn(q23, s2, z2);
                 }
+            }
+            if (r == 0) {
+#pragma unroll
+                for (int p = 0; p < 4; ++p) acc[p] = term[p];
+            } else {
+#pragma unroll
+                for (int p = 0; p < 4; ++p) acc[p] = add2_rn(acc[p], term[p]);
             }
         }
     }
     float lmin = __int_as_float(0x7f800000), lmax = -__int_as_float(0x7f800000);
-    bool bad = false;
     if (act) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            lmin = fminf(lmin, acc[i]);
-            lmax = fmaxf(lmax, acc[i]);
-            bad |= outside_fp16_domain(acc[i]);
+        for (int p = 0; p < 4; ++p) {
+            lmin = nan_min(lmin, nan_min(acc[p].x, acc[p].y));
+            lmax = nan_max(lmax, nan_max(acc[p].x, acc[p].y));
         }
     }
-    raise_flags(a, bad);
-    uint32_t yb[8];
+    uint32_t yb[4];   // bf16 pairs of the result
     if (a.P >= 2) {
-        const Grid g = make_grid<L, Q>(lmin, lmax);
+        const GridP g = make_grid_p<L, Q>(lmin, lmax);
+        raise_flags(a, act && g.bad);
         if (!act) return;
         uint8_t* codes = a.g_codes + (size_t)j * CB;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            int q[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                q[k] = encode<Q>(acc[4 * h + k], g);
-                yb[4 * h + k] = f2bf16(decode(q[k], g.s, g.z));
-            }
-            store_chunk_codes<BITS>(codes, ln.chunk(h), pack4<BITS>(q));
+            const float2 t01 = encode2(acc[2 * h], g);
+            const float2 t23 = encode2(acc[2 * h + 1], g);
+            store_chunk_codes<BITS>(codes, ln.chunk(h), pack_codes4<BITS>(t01, t23));
+            const float2 y01 = fma2_rn(add2_rn(t01, splat(-kMagic)), g.s, g.z);
+            const float2 y23 = fma2_rn(add2_rn(t23, splat(-kMagic)), g.s, g.z);
+            yb[2 * h] = bf16x2_rn(y01);
+            yb[2 * h + 1] = bf16x2_rn(y23);
         }
         if (ln.t == 0) a.g_params[j] = g.param;
     } else {
+        // a single rank sends nothing: its output is its own x'
+        raise_flags(a, act && !(lmin >= -65504.0f && lmax <= 65504.0f));
         if (!act) return;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) yb[i] = f2bf16(acc[i]);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) store_y4(a.out[0], j * GROUP + 4 * ln.chunk(h), a.n, true, &yb[4 * h]);
+        for (int p = 0; p < 4; ++p) yb[p] = bf16x2_rn(acc[p]);
+        *reinterpret_cast<uint2*>(a.out[0] + j * GROUP + c0) = make_uint2(yb[0], yb[1]);
+        *reinterpret_cast<uint2*>(a.out[0] + j * GROUP + c1) = make_uint2(yb[2], yb[3]);
     }
     if (a.state) {
+        float2 el[4], es[4];
+        load_f8_smem(els, c0, c1, el);
+        load_f8_smem(ess, c0, c1, es);
         float* el_g = a.state + (size_t)o * 2 * a.S + j * GROUP;
+        float2 rho[4];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int c = 4 * ln.chunk(h);
-            const float4 l4 = *reinterpret_cast<const float4*>(els + c);
-            const float4 s4 = *reinterpret_cast<const float4*>(ess + c);
-            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-            const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
-            float ol[4], os[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int i = 4 * h + k;
-                const float rho = __fsub_rn(acc[i], __uint_as_float(yb[i] << 16));
-                ol[k] = ema(lv[k], rho, a.keep_long, a.a_long);
-                os[k] = ema(sv[k], rho, a.keep_short, a.a_short);
-            }
-            __stcs(reinterpret_cast<float4*>(el_g + c), make_float4(ol[0], ol[1], ol[2], ol[3]));
-            __stcs(reinterpret_cast<float4*>(el_g + a.S + c), make_float4(os[0], os[1], os[2], os[3]));
+        for (int p = 0; p < 4; ++p) {
+            // -float(y): flip the sign bits of the bf16 pair, then widen exactly
+            const uint32_t ny = yb[p] ^ 0x80008000u;
+            rho[p] = add2_rn(acc[p], make_float2(__uint_as_float(ny << 16), __uint_as_float(ny & 0xffff0000u)));
         }
+        store_f4_pair(el_g + c0, ema2(el[0], rho[0], a.keep_long, a.a_long), ema2(el[1], rho[1], a.keep_long, a.a_long));
+        store_f4_pair(el_g + c1, ema2(el[2], rho[2], a.keep_long, a.a_long), ema2(el[3], rho[3], a.keep_long, a.a_long));
+        store_f4_pair(el_g + a.S + c0, ema2(es[0], rho[0], a.keep_short, a.a_short),
+                      ema2(es[1], rho[1], a.keep_short, a.a_short));
+        store_f4_pair(el_g + a.S + c1, ema2(es[2], rho[2], a.keep_short, a.a_short),
+                      ema2(es[3], rho[3], a.keep_short, a.a_short));
     }
 }
 
@@ -491,6 +657,104 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
         const long long j = a.G - 1;
         const int o = (int)((j * a.P + a.P - 1) / a.G);
         reduce_range<GROUP, BITS>(a, o, j, j + 1, 0, 1);
+    }
+}
+
+// ------------------------------------------------------------ gather
+//
+// Every rank receives the same decoded group, so the kernel decodes a tile of
+// the gathered payload once into shared memory and sends it to the P outputs
+// with P bulk stores (the TMA engine writes; no per-thread store traffic).
+// A ring of kGatherBufs tile buffers lets decoding run ahead of the stores.
+
+constexpr int kGatherThreads = 256;
+constexpr int kGatherTileElems = kGatherThreads * 8;                 // 2048 elements, 4 KB of bf16
+constexpr int kGatherBufs = 4;
+constexpr int kGatherSmem = kGatherBufs * kGatherTileElems * 2;     // 16 KB
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 1-D bulk copy shared -> global (no multicast); dst, src, bytes multiples of 16
+__device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_addr(src)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// eight contiguous decoded elements of a group as bf16 (codes word w: 4-bit in
+// w.x, 8-bit in w.x and w.y)
+template <int BITS>
+__device__ __forceinline__ uint4 decode8_bf16(uint2 w, uint32_t param) {
+    const float2 s2 = splat(param_s(param));
+    const float2 z2 = splat(param_z(param));
+    float2 q[4];
+    if (BITS == 4) {
+        unpack_codes4<4>(w.x & 0xffffu, q[0], q[1]);
+        unpack_codes4<4>(w.x >> 16, q[2], q[3]);
+    } else {
+        unpack_codes4<8>(w.x, q[0], q[1]);
+        unpack_codes4<8>(w.y, q[2], q[3]);
+    }
+    return make_uint4(bf16x2_rn(fma2_rn(q[0], s2, z2)), bf16x2_rn(fma2_rn(q[1], s2, z2)),
+                      bf16x2_rn(fma2_rn(q[2], s2, z2)), bf16x2_rn(fma2_rn(q[3], s2, z2)));
+}
+
+template <int GROUP, int BITS>
+__global__ void __launch_bounds__(kGatherThreads) k_gather_tma(const Args a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    constexpr int L = GROUP / 8, CB = GROUP * BITS / 8, T = kGatherTileElems / GROUP;
+    const long long G_full = a.n / GROUP;
+    const long long ntiles = (G_full + T - 1) / T;
+    const int tid = threadIdx.x;
+    const int gi = tid / L, t = tid % L;   // group within the tile, lane within the group
+    long long i = 0;
+    for (long long k = blockIdx.x; k < ntiles; k += gridDim.x, ++i) {
+        const int b = (int)(i % kGatherBufs);
+        uint16_t* buf = reinterpret_cast<uint16_t*>(smem + (size_t)b * kGatherTileElems * 2);
+        if (i >= kGatherBufs) {
+            // the stores that last read this buffer must be done reading it
+            if (tid == 0) bulk_wait_read<kGatherBufs - 1>();
+            __syncthreads();
+        }
+        const long long j0 = k * T;
+        const int cnt = (int)min((long long)T, G_full - j0);
+        if (gi < cnt) {
+            const long long j = j0 + gi;
+            const uint2 w = load_codes8<BITS>(a.g_codes + (size_t)j * CB, t);
+            *reinterpret_cast<uint4*>(buf + gi * GROUP + 8 * t) = decode8_bf16<BITS>(w, a.g_params[j]);
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            const uint32_t bytes = (uint32_t)cnt * GROUP * 2;
+            for (int r = 0; r < a.P; ++r) bulk_store(a.out[r] + j0 * GROUP, buf, bytes);
+            bulk_commit();
+        }
+    }
+    if (tid == 0) bulk_wait_all();
+    // the partial last group (not a multiple of 16 bytes): direct stores
+    if (G_full < a.G && blockIdx.x == gridDim.x - 1 && tid < L) {
+        const long long j = a.G - 1;
+        const uint2 w = load_codes8<BITS>(a.g_codes + (size_t)j * CB, tid);
+        const uint4 v = decode8_bf16<BITS>(w, a.g_params[j]);
+        const uint32_t yb[4] = {v.x, v.y, v.z, v.w};
+        const long long e = j * GROUP + 8 * tid;
+        for (int r = 0; r < a.P; ++r) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                if (e + k < a.n) a.out[r][e + k] = (uint16_t)(yb[k >> 1] >> (16 * (k & 1)));
+        }
     }
 }
 
