@@ -170,6 +170,7 @@ bool make_args(const echo_state* st, int bits, const void* const* inputs, void* 
     a->keep_long = 1.0f - aL;
     a->a_short = aS;
     a->keep_short = 1.0f - aS;
+    a->one = 1.0f;
     return true;
 }
 

@@ -56,6 +56,7 @@ struct Args {
     int P;
     float eta, w, one_minus_w;
     float a_long, keep_long, a_short, keep_short;
+    float one;   // 1.0f, passed at run time (see add_after_mul2 in echo_pipeline.cuh)
 };
 
 // ------------------------------------------------------------------ helpers

@@ -247,10 +247,12 @@ __device__ __forceinline__ void produce(const Args& a, const PipeShared& p, RunW
 //    2^23 (bit pattern 0x4B000000 | code) and subtracting 2^23;
 //  * additions whose operands are not products (rank-ordered sums, x' - x_hat).
 // Every product that the definition rounds before an addition (compensation,
-// the quantizer's (v - z) * inv, both EMA terms) is a scalar __fmul_rn: the
-// assembler may fuse a paired multiply into the paired add that consumes it,
-// even with an explicit .rn (seen on sm_100a: a tie rounded the other way),
-// while scalar operations with an explicit rounding keep their own rounding.
+// the quantizer's (v - z) * inv, both EMA terms) is a paired multiply, and
+// the addition that consumes it is written fma(product, one, other) with
+// `one` = 1.0 read from the kernel arguments: the assembler may fuse a paired
+// multiply into a paired add that consumes it, even with an explicit .rn
+// (seen on sm_100a: a tie rounded the other way), but it cannot fold a
+// multiplier it does not know, and fma(p, 1, q) rounds exactly like p + q.
 // Round-half-even of u in [0, 2^22) is (u + 2^23): binary32 spacing there is
 // 1, so the addition itself rounds u to the nearest integer, ties to even,
 // and the code sits in the low mantissa bits.
@@ -266,6 +268,18 @@ __device__ __forceinline__ float2 add2_rn(float2 a, float2 b) {
         "mov.b64 ra, {%2, %3};\n\t"
         "mov.b64 rb, {%4, %5};\n\t"
         "add.rn.f32x2 rr, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, rr;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+
+__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rr;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rr, ra, rb;\n\t"
         "mov.b64 {%0, %1}, rr;\n\t}"
         : "=f"(r.x), "=f"(r.y)
         : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
@@ -338,10 +352,15 @@ __device__ __forceinline__ GridP make_grid_p(float lane_min, float lane_max) {
     return g;
 }
 
+// p + q where p (or q) is a rounded product: fma(p, one, q), one = 1.0 at run time
+__device__ __forceinline__ float2 add_after_mul2(float2 p, float2 q, const Args& a) {
+    return fma2_rn(p, splat(a.one), q);
+}
+
 // 2^23 + code for a pair of values: code = round_half_even((v - z) * inv)
-__device__ __forceinline__ float2 encode2(float2 v, const GridP& g) {
-    const float2 d = add2_rn(v, g.nz);   // v - z
-    return make_float2(__fadd_rn(__fmul_rn(d.x, g.inv.x), kMagic), __fadd_rn(__fmul_rn(d.y, g.inv.y), kMagic));
+__device__ __forceinline__ float2 encode2(float2 v, const GridP& g, const Args& a) {
+    const float2 u = mul2_rn(add2_rn(v, g.nz), g.inv);   // (v - z) * inv
+    return add_after_mul2(u, splat(kMagic), a);
 }
 
 // four codes (2^23 + code each) -> one chunk of packed codes
@@ -375,14 +394,15 @@ __device__ __forceinline__ void unpack_codes4(uint32_t w, float2& q01, float2& q
     q23 = add2_rn(make_float2(__uint_as_float(m2), __uint_as_float(m3)), splat(-kMagic));
 }
 
-// x' = x + eta * (w * e_short + (1 - w) * e_long), two elements (scalar products)
+// x' = x + eta * (w * e_short + (1 - w) * e_long), two elements
 __device__ __forceinline__ float2 inject2(float2 x, float2 el, float2 es, const Args& a) {
-    return make_float2(inject(x.x, el.x, es.x, a), inject(x.y, el.y, es.y, a));
+    const float2 t = add_after_mul2(mul2_rn(splat(a.w), es), mul2_rn(splat(a.one_minus_w), el), a);
+    return add_after_mul2(mul2_rn(splat(a.eta), t), x, a);
 }
 
-// e <- (1 - alpha) * e + alpha * rho, two elements (scalar products)
-__device__ __forceinline__ float2 ema2(float2 e, float2 rho, float keep, float alpha) {
-    return make_float2(ema(e.x, rho.x, keep, alpha), ema(e.y, rho.y, keep, alpha));
+// e <- (1 - alpha) * e + alpha * rho, two elements
+__device__ __forceinline__ float2 ema2(float2 e, float2 rho, float keep, float alpha, const Args& a) {
+    return add_after_mul2(mul2_rn(splat(keep), e), mul2_rn(splat(alpha), rho), a);
 }
 
 __device__ __forceinline__ void load_x8_smem(const uint16_t* xs, int c0, int c1, float2 v[4]) {
@@ -444,8 +464,8 @@ __device__ __forceinline__ void quantize_tile_group(const Args& a, const uint8_t
     float* el_g = a.state ? a.state + (size_t)r * 2 * a.S + j * GROUP : nullptr;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-        const float2 t01 = encode2(v[2 * h], g);
-        const float2 t23 = encode2(v[2 * h + 1], g);
+        const float2 t01 = encode2(v[2 * h], g, a);
+        const float2 t23 = encode2(v[2 * h + 1], g, a);
         store_chunk_codes<BITS>(codes, ln.chunk(h), pack_codes4<BITS>(t01, t23));
         if (a.state) {
             // residual x' - x_hat with x_hat = code*s + z (fused: code*s is exact)
@@ -454,10 +474,10 @@ __device__ __forceinline__ void quantize_tile_group(const Args& a, const uint8_t
             const float2 rho01 = add2_rn(v[2 * h], fma2_rn(q01, g.ns, g.nz));
             const float2 rho23 = add2_rn(v[2 * h + 1], fma2_rn(q23, g.ns, g.nz));
             const int c = h ? c1 : c0;
-            store_f4_pair(el_g + c, ema2(el[2 * h], rho01, a.keep_long, a.a_long),
-                          ema2(el[2 * h + 1], rho23, a.keep_long, a.a_long));
-            store_f4_pair(el_g + a.S + c, ema2(es[2 * h], rho01, a.keep_short, a.a_short),
-                          ema2(es[2 * h + 1], rho23, a.keep_short, a.a_short));
+            store_f4_pair(el_g + c, ema2(el[2 * h], rho01, a.keep_long, a.a_long, a),
+                          ema2(el[2 * h + 1], rho23, a.keep_long, a.a_long, a));
+            store_f4_pair(el_g + a.S + c, ema2(es[2 * h], rho01, a.keep_short, a.a_short, a),
+                          ema2(es[2 * h + 1], rho23, a.keep_short, a.a_short, a));
         }
     }
     if (ln.t == 0) a.a2a_params[(size_t)r * a.G + j] = g.param;
@@ -588,8 +608,8 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
         uint8_t* codes = a.g_codes + (size_t)j * CB;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            const float2 t01 = encode2(acc[2 * h], g);
-            const float2 t23 = encode2(acc[2 * h + 1], g);
+            const float2 t01 = encode2(acc[2 * h], g, a);
+            const float2 t23 = encode2(acc[2 * h + 1], g, a);
             store_chunk_codes<BITS>(codes, ln.chunk(h), pack_codes4<BITS>(t01, t23));
             const float2 y01 = fma2_rn(add2_rn(t01, splat(-kMagic)), g.s, g.z);
             const float2 y23 = fma2_rn(add2_rn(t23, splat(-kMagic)), g.s, g.z);
@@ -618,12 +638,12 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
             const uint32_t ny = yb[p] ^ 0x80008000u;
             rho[p] = add2_rn(acc[p], make_float2(__uint_as_float(ny << 16), __uint_as_float(ny & 0xffff0000u)));
         }
-        store_f4_pair(el_g + c0, ema2(el[0], rho[0], a.keep_long, a.a_long), ema2(el[1], rho[1], a.keep_long, a.a_long));
-        store_f4_pair(el_g + c1, ema2(el[2], rho[2], a.keep_long, a.a_long), ema2(el[3], rho[3], a.keep_long, a.a_long));
-        store_f4_pair(el_g + a.S + c0, ema2(es[0], rho[0], a.keep_short, a.a_short),
-                      ema2(es[1], rho[1], a.keep_short, a.a_short));
-        store_f4_pair(el_g + a.S + c1, ema2(es[2], rho[2], a.keep_short, a.a_short),
-                      ema2(es[3], rho[3], a.keep_short, a.a_short));
+        store_f4_pair(el_g + c0, ema2(el[0], rho[0], a.keep_long, a.a_long, a), ema2(el[1], rho[1], a.keep_long, a.a_long, a));
+        store_f4_pair(el_g + c1, ema2(el[2], rho[2], a.keep_long, a.a_long, a), ema2(el[3], rho[3], a.keep_long, a.a_long, a));
+        store_f4_pair(el_g + a.S + c0, ema2(es[0], rho[0], a.keep_short, a.a_short, a),
+                      ema2(es[1], rho[1], a.keep_short, a.a_short, a));
+        store_f4_pair(el_g + a.S + c1, ema2(es[2], rho[2], a.keep_short, a.a_short, a),
+                      ema2(es[3], rho[3], a.keep_short, a.a_short, a));
     }
 }
 
