@@ -279,6 +279,34 @@ def run_gpu(args):
         per_phase["gather"] += e[2].elapsed_time(e[3])
     max_ms = max_over_ranks(total_ms, world, dev)
 
+    # the same message without feedback state (x' = x, no EMA traffic): its
+    # time and the difference, the cost of compensation (the pages quote
+    # 0.90 ms per 1 GB message on 8 A100s, fused into the entry pass)
+    variant = None
+    if not args.no_variants:
+        nf = E.EchoAllReduce(n, P, group, bits, feedback=False, device=dev)
+        nf_steps = max(3, min(args.steps, 10))
+
+        def nf_step():
+            E.echo_allreduce_sim(inputs, outputs, nf.handle, n, P, bits, group, *fb, stream=stream)
+
+        for _ in range(args.warmup):
+            nf_step()
+        barrier()
+        a0, b0 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(nf_steps):
+            nf_step()
+        b0.record(stream)
+        barrier()
+        nf_ms = max_over_ranks(a0.elapsed_time(b0), world, dev) / nf_steps
+        nf.close()
+        del nf
+        variant = {"ms_per_step": nf_ms, "steps": nf_steps,
+                   "value": weak_scaling_gbs(world, P * n * 2, nf_ms),
+                   "roofline_frac": algorithmic_bytes(P, n, group, bits, feedback=False)["total"] / (nf_ms * 1e-3)
+                   / 1e9 / _peak_hbm()[0]}
+
     # end to end through the public call with host buffers: pinned inputs
     # copied in, the call, the reduced result copied out, every step
     e2e = None
@@ -332,6 +360,9 @@ def run_gpu(args):
             "clocks": clock_info, "status": rc, "flags": flags,
             "e2e": e2e,
         }
+        if variant is not None:
+            line["no_feedback"] = variant
+            line["compensation_ms"] = ms - variant["ms_per_step"]
         if world == 1 and not args.no_cpu_baseline:
             gbs, dt, er = cpu_sample_rate(CPU_BASELINE_COLS)
             line["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
@@ -352,6 +383,7 @@ def main():
     ap.add_argument("--impl", default="echo", choices=["echo", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-variants", action="store_true", help="skip the no-feedback timing")
     ap.add_argument("--tokens", type=int, default=None,
                     help="tokens per rank (default 131072, the 1 GB message); smaller values are for profiling")
     args = ap.parse_args()

@@ -88,25 +88,38 @@ int pipe_grid(K kernel, const echo_state* st) {
 
 enum class Stage { Quantize, Reduce, Gather };
 
+// One pipelined launch; `grid` caches the grid (and the shared-memory opt-in)
+// of this kernel instantiation.
+template <typename K>
+int launch_pipe(K kernel, int* grid, const echo_dev::Args& a, const echo_state* st, cudaStream_t s) {
+    if (*grid == 0) *grid = pipe_grid(kernel, st);
+    if (*grid == 0) return ECHO_ECUDA;
+    kernel<<<*grid, echo_dev::kPipeThreads, echo_dev::kPipeSmem, s>>>(a);
+    return ECHO_OK;
+}
+
 template <int GROUP, int BITS>
 int launch_stage(Stage stage, const echo_dev::Args& a, const echo_state* st, cudaStream_t s) {
+    int rc = ECHO_OK;
     switch (stage) {
-        case Stage::Quantize: {
-            auto k = echo_dev::k_quantize_tma<GROUP, BITS>;
-            static int grid = 0;
-            if (grid == 0) grid = pipe_grid(k, st);
-            if (grid == 0) return ECHO_ECUDA;
-            k<<<grid, echo_dev::kPipeThreads, echo_dev::kPipeSmem, s>>>(a);
+        case Stage::Quantize:
+            if (a.state) {
+                static int grid = 0;
+                rc = launch_pipe(echo_dev::k_quantize_tma<GROUP, BITS, true>, &grid, a, st, s);
+            } else {
+                static int grid = 0;
+                rc = launch_pipe(echo_dev::k_quantize_tma<GROUP, BITS, false>, &grid, a, st, s);
+            }
             break;
-        }
-        case Stage::Reduce: {
-            auto k = echo_dev::k_reduce_tma<GROUP, BITS>;
-            static int grid = 0;
-            if (grid == 0) grid = pipe_grid(k, st);
-            if (grid == 0) return ECHO_ECUDA;
-            k<<<grid, echo_dev::kPipeThreads, echo_dev::kPipeSmem, s>>>(a);
+        case Stage::Reduce:
+            if (a.state) {
+                static int grid = 0;
+                rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, true>, &grid, a, st, s);
+            } else {
+                static int grid = 0;
+                rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, false>, &grid, a, st, s);
+            }
             break;
-        }
         case Stage::Gather: {
             auto k = echo_dev::k_gather_tma<GROUP, BITS>;
             static int grid = 0;
@@ -115,6 +128,7 @@ int launch_stage(Stage stage, const echo_dev::Args& a, const echo_state* st, cud
             break;
         }
     }
+    if (rc != ECHO_OK) return rc;
     return cuda_status(cudaGetLastError());
 }
 

@@ -106,9 +106,9 @@ struct Tile {
     int count;
 };
 
-template <int GROUP>
+template <int GROUP, int M = 1>
 struct RunWalker {
-    static constexpr int T = kTileElems / GROUP;   // groups per tile
+    static constexpr int T = M * kTileElems / GROUP;   // groups per tile (M sub-tiles)
     // kind 0: non-owned runs of every rank (quantize); kind 1: owned runs (reduce)
     int kind;
     long long G, G_full;
@@ -197,9 +197,10 @@ __device__ __forceinline__ void report_timeout(const Args& a, const PipeShared& 
 }
 
 // Producer lane: stream tiles of `walker` into the stage ring. `with_state`
-// adds the two EMA tiles of the tile's rank.
-template <int GROUP>
-__device__ __forceinline__ void produce(const Args& a, const PipeShared& p, RunWalker<GROUP>& walker,
+// adds the two EMA tiles of the tile's rank (then M == 1); without state a
+// stage holds M = 5 sub-tiles of bf16 inputs, the same 20 KB.
+template <int GROUP, int M>
+__device__ __forceinline__ void produce(const Args& a, const PipeShared& p, RunWalker<GROUP, M>& walker,
                                         bool with_state) {
     long long issued = 0;
     Tile t;
@@ -429,7 +430,7 @@ __device__ __forceinline__ void store_f4_pair(float* p, float2 lo, float2 hi) {
 
 // ------------------------------------------------------------ quantize
 
-template <int GROUP, int BITS>
+template <int GROUP, int BITS, bool FB>
 __device__ __forceinline__ void quantize_tile_group(const Args& a, const uint8_t* st, const Tile& t, int gi,
                                                     bool act) {
     using LN = Lane<GROUP>;
@@ -445,7 +446,7 @@ __device__ __forceinline__ void quantize_tile_group(const Args& a, const uint8_t
     float lmin = __int_as_float(0x7f800000), lmax = -__int_as_float(0x7f800000);
     if (act) {
         load_x8_smem(xs, c0, c1, v);
-        if (a.state) {
+        if (FB) {
             load_f8_smem(els, c0, c1, el);
             load_f8_smem(ess, c0, c1, es);
 #pragma unroll
@@ -461,13 +462,13 @@ __device__ __forceinline__ void quantize_tile_group(const Args& a, const uint8_t
     raise_flags(a, act && g.bad);
     if (!act) return;
     uint8_t* codes = a.a2a_codes + ((size_t)r * a.G + j) * CB;
-    float* el_g = a.state ? a.state + (size_t)r * 2 * a.S + j * GROUP : nullptr;
+    float* el_g = FB ? a.state + (size_t)r * 2 * a.S + j * GROUP : nullptr;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const float2 t01 = encode2(v[2 * h], g, a);
         const float2 t23 = encode2(v[2 * h + 1], g, a);
         store_chunk_codes<BITS>(codes, ln.chunk(h), pack_codes4<BITS>(t01, t23));
-        if (a.state) {
+        if (FB) {
             // residual x' - x_hat with x_hat = code*s + z (fused: code*s is exact)
             const float2 q01 = add2_rn(t01, splat(-kMagic));
             const float2 q23 = add2_rn(t23, splat(-kMagic));
@@ -483,20 +484,21 @@ __device__ __forceinline__ void quantize_tile_group(const Args& a, const uint8_t
     if (ln.t == 0) a.a2a_params[(size_t)r * a.G + j] = g.param;
 }
 
-template <int GROUP, int BITS>
+template <int GROUP, int BITS, bool FB>
 __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
+    constexpr int M = FB ? 1 : 5;
     const PipeShared p = pipe_shared(smem);
     pipe_init(p);
     const int warp = threadIdx.x >> 5;
     const long long G_full = a.n / GROUP;
-    RunWalker<GROUP> walker(0, a.G, G_full, a.P);
+    RunWalker<GROUP, M> walker(0, a.G, G_full, a.P);
     if (warp == kConsumerWarps) {
-        if ((threadIdx.x & 31) == 0) produce<GROUP>(a, p, walker, a.state != nullptr);
+        if ((threadIdx.x & 31) == 0) produce<GROUP, M>(a, p, walker, FB);
         return;
     }
     constexpr int GPW = Lane<GROUP>::GPW;
-    const int gi = warp * GPW + Lane<GROUP>().sub;
+    const int gi = warp * GPW + Lane<GROUP>().sub;   // + m * kConsumerWarps * GPW for sub-tile m
     long long i = 0;
     Tile t;
     for (long long k = blockIdx.x; walker.locate(k, &t); k += gridDim.x, ++i) {
@@ -505,7 +507,11 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
             if ((threadIdx.x & 31) == 0) report_timeout(a, p);
             return;
         }
-        quantize_tile_group<GROUP, BITS>(a, p.stages + (size_t)s * kStageBytes, t, gi, gi < t.count);
+#pragma unroll 1
+        for (int m = 0; m < M; ++m) {
+            const int g = gi + m * kConsumerWarps * GPW;
+            quantize_tile_group<GROUP, BITS, FB>(a, p.stages + (size_t)s * kStageBytes, t, g, g < t.count);
+        }
         __syncwarp();
         if ((threadIdx.x & 31) == 0) mbar_arrive(&p.empty[s]);
     }
@@ -521,7 +527,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
 
 // ------------------------------------------------------------ reduce
 
-template <int GROUP, int BITS>
+template <int GROUP, int BITS, bool FB>
 __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* st, const Tile& t, int gi,
                                                   bool act) {
     using LN = Lane<GROUP>;
@@ -539,7 +545,7 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
     for (int p = 0; p < 4; ++p) xo[p] = acc[p] = make_float2(0.0f, 0.0f);
     if (act) {
         load_x8_smem(xs, c0, c1, xo);
-        if (a.state) {
+        if (FB) {
             float2 el[4], es[4];
             load_f8_smem(els, c0, c1, el);
             load_f8_smem(ess, c0, c1, es);
@@ -626,7 +632,7 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
         *reinterpret_cast<uint2*>(a.out[0] + j * GROUP + c0) = make_uint2(yb[0], yb[1]);
         *reinterpret_cast<uint2*>(a.out[0] + j * GROUP + c1) = make_uint2(yb[2], yb[3]);
     }
-    if (a.state) {
+    if (FB) {
         float2 el[4], es[4];
         load_f8_smem(els, c0, c1, el);
         load_f8_smem(ess, c0, c1, es);
@@ -647,20 +653,21 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
     }
 }
 
-template <int GROUP, int BITS>
+template <int GROUP, int BITS, bool FB>
 __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
+    constexpr int M = FB ? 1 : 5;
     const PipeShared p = pipe_shared(smem);
     pipe_init(p);
     const int warp = threadIdx.x >> 5;
     const long long G_full = a.n / GROUP;
-    RunWalker<GROUP> walker(1, a.G, G_full, a.P);
+    RunWalker<GROUP, M> walker(1, a.G, G_full, a.P);
     if (warp == kConsumerWarps) {
-        if ((threadIdx.x & 31) == 0) produce<GROUP>(a, p, walker, a.state != nullptr);
+        if ((threadIdx.x & 31) == 0) produce<GROUP, M>(a, p, walker, FB);
         return;
     }
     constexpr int GPW = Lane<GROUP>::GPW;
-    const int gi = warp * GPW + Lane<GROUP>().sub;
+    const int gi = warp * GPW + Lane<GROUP>().sub;   // + m * kConsumerWarps * GPW for sub-tile m
     long long i = 0;
     Tile t;
     for (long long k = blockIdx.x; walker.locate(k, &t); k += gridDim.x, ++i) {
@@ -669,7 +676,11 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
             if ((threadIdx.x & 31) == 0) report_timeout(a, p);
             return;
         }
-        reduce_tile_group<GROUP, BITS>(a, p.stages + (size_t)s * kStageBytes, t, gi, gi < t.count);
+#pragma unroll 1
+        for (int m = 0; m < M; ++m) {
+            const int g = gi + m * kConsumerWarps * GPW;
+            reduce_tile_group<GROUP, BITS, FB>(a, p.stages + (size_t)s * kStageBytes, t, g, g < t.count);
+        }
         __syncwarp();
         if ((threadIdx.x & 31) == 0) mbar_arrive(&p.empty[s]);
     }
