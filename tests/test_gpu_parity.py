@@ -208,3 +208,38 @@ def test_deterministic():
             gpu.close()
     for a, b in zip(*outs):
         assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("P,n,group,bits", [(6, 5000, 32, 8), (2, 4096, 128, 8), (9, 70001, 128, 8), (3, 2 * 2048 * 5 + 300, 256, 4)])
+def test_parity_more_shapes(P, n, group, bits):
+    x = _random_inputs(P, n, 31 * P + n, 1.0)
+    el0, es0 = _seeded_state(P, n, n + 3 * P)
+    _check_full_call(P, n, Params(bits=bits, group=group), x, el0, es0, True, calls=2)
+
+
+@pytest.mark.parametrize("eta,w,aL,aS", [(0.0, 0.5, 0.05, 0.5), (1.5, 0.0, 1.0, 0.0), (0.5, 1.0, 0.0, 1.0), (1.0, 0.25, 0.3, 0.9)])
+def test_parity_feedback_parameters(eta, w, aL, aS):
+    P, n = 4, 3 * 4096 + 77
+    x = _random_inputs(P, n, 17, 1.5)
+    el0, es0 = _seeded_state(P, n, 18, scale=0.2)
+    _check_full_call(P, n, Params(eta=eta, w=w, alpha_long=aL, alpha_short=aS), x, el0, es0, True, calls=3)
+
+
+def test_parity_special_values():
+    """Groups that are constant (s = 0: every code 0), all zero, holding -0,
+    bf16 subnormals, or values close to the fp16 edge after the sum."""
+    P, n, group = 4, 64 * 128, 128
+    g = torch.Generator().manual_seed(21)
+    x = torch.randn(P, n, generator=g)
+    x[:, 0:128] = 0.0                                   # all-zero group on every rank
+    x[:, 128:256] = -0.0                                # negative zeros
+    x[0, 256:384] = 3.25                                # constant on one rank
+    x[:, 384:512] = 1.5                                 # constant on every rank (sum exact)
+    x[1, 512:640] = torch.randn(128, generator=g) * 1e-39   # bf16 subnormals
+    x[:, 640:768] = 16000.0 + torch.randn(P, 128, generator=g)  # sum near 64000 < 65504
+    x[2, 768:896] = -3.0e4                              # large negative on one rank
+    x[:, 896:900] = torch.tensor([1e-30, -1e-30, 2e-38, -2e-38])
+    xb = x.to(torch.bfloat16)
+    for feedback in (True, False):
+        el0, es0 = (np.zeros((P, n), np.float32), np.zeros((P, n), np.float32)) if feedback else (None, None)
+        _check_full_call(P, n, Params(), xb, el0, es0, feedback, calls=2)
