@@ -60,8 +60,11 @@ def _peak_hbm():
 
 
 def algorithmic_bytes(P, n, group, bits, feedback=True):
-    """Minimal bytes each kernel must move per call: every tensor crosses HBM
-    once, each payload is written once and read once."""
+    """Minimal bytes per call: every tensor crosses HBM once, each payload is
+    written once and read once ("total", the roofline of the call). Per
+    kernel: quantize; and the owners' reduce, which also writes the P outputs
+    (it decodes the gathered bits it just produced, so its own bytes omit the
+    re-read of the gather payload that "total" counts)."""
     G = -(-n // group)
     pb = group * bits // 8 + 4                       # payload bytes per group
     st = 16 if feedback else 0                       # two fp32 EMAs read + written
@@ -69,7 +72,7 @@ def algorithmic_bytes(P, n, group, bits, feedback=True):
     q = (P - 1) * G * (xb + st * group + pb)          # non-owned rank-groups
     r = G * (xb + st * group + (P - 1) * pb + pb)      # owners: own x + EMAs, P-1 payloads in, gather out
     g = G * (pb + P * xb)                             # gather payload in, P outputs
-    return {"quantize": q, "reduce": r, "gather": g, "total": q + r + g}
+    return {"quantize": q, "reduce_gather": r + g - G * pb, "total": q + r + g}
 
 
 def _kernel_source_hash():
@@ -241,18 +244,18 @@ def run_gpu(args):
     h = ar.handle
     fb = (w.eta, w.alpha_long, w.alpha_short, w.w)
 
+    # one step = echo_allreduce_sim's two launches, with an event between them
+    # for the per-kernel roofline: quantize, then the owners' reduce, which
+    # also decodes into all P outputs
     def step(evs=None):
         if evs is not None:
             evs[0].record(stream)
         E.echo_phase_quantize(inputs, h, bits, *fb, stream=stream)
         if evs is not None:
             evs[1].record(stream)
-        E.echo_phase_reduce(inputs, None, h, bits, *fb, stream=stream)
+        E.echo_phase_reduce(inputs, outputs, h, bits, *fb, stream=stream)
         if evs is not None:
             evs[2].record(stream)
-        E.echo_phase_gather(outputs, h, bits, stream=stream)
-        if evs is not None:
-            evs[3].record(stream)
 
     def barrier():
         if world > 1:
@@ -263,7 +266,7 @@ def run_gpu(args):
         step()
     barrier()
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     clocks = ClockSampler(local)
     barrier()
     for i in range(args.steps):
@@ -271,12 +274,11 @@ def run_gpu(args):
     barrier()
     clock_info = clocks.stop()
     rc, flags = ar.status()
-    per_phase = {"quantize": 0.0, "reduce": 0.0, "gather": 0.0}
-    total_ms = evs[0][0].elapsed_time(evs[-1][3])
+    per_phase = {"quantize": 0.0, "reduce_gather": 0.0}
+    total_ms = evs[0][0].elapsed_time(evs[-1][2])
     for e in evs:
         per_phase["quantize"] += e[0].elapsed_time(e[1])
-        per_phase["reduce"] += e[1].elapsed_time(e[2])
-        per_phase["gather"] += e[2].elapsed_time(e[3])
+        per_phase["reduce_gather"] += e[1].elapsed_time(e[2])
     max_ms = max_over_ranks(total_ms, world, dev)
 
     # the same message without feedback state (x' = x, no EMA traffic): its
@@ -356,7 +358,7 @@ def run_gpu(args):
                               "frac": ab["total"] / (ms * 1e-3) / 1e9 / peak},
             "phases_ms": {k: v / args.steps for k, v in per_phase.items()},
             "elements_per_s": world * P * n / (ms * 1e-3),
-            "gpu_launches": 3 * args.steps if P >= 2 else args.steps,
+            "gpu_launches": 2 * args.steps if P >= 2 else args.steps,
             "clocks": clock_info, "status": rc, "flags": flags,
             "e2e": e2e,
         }

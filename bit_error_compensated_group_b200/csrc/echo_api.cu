@@ -263,8 +263,8 @@ int echo_phase_reduce(const void* const* inputs, void* const* outputs, echo_stat
     if (!valid_feedback(eta, alpha_long, alpha_short, w)) return ECHO_EINVAL;
     if (st->P == 1 && !outputs) return ECHO_EINVAL;
     echo_dev::Args a;
-    if (!make_args(st, bits, inputs, st->P == 1 ? outputs : nullptr, eta, alpha_long, alpha_short, w, &a))
-        return ECHO_EINVAL;
+    if (!make_args(st, bits, inputs, outputs, eta, alpha_long, alpha_short, w, &a)) return ECHO_EINVAL;
+    a.write_outputs = outputs != nullptr;
     if (int rc = set_device(st)) return rc;
     return launch(Stage::Reduce, bits, a, st, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -288,14 +288,11 @@ int echo_allreduce_sim(const void* const* inputs, void* const* outputs, echo_sta
     if (!make_args(st, bits, inputs, outputs, eta, alpha_long, alpha_short, w, &a)) return ECHO_EINVAL;
     if (int rc = set_device(st)) return rc;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    a.write_outputs = 1;   // the owner's pass decodes into every output (phase 4)
     if (P >= 2) {
         if (int rc = launch(Stage::Quantize, bits, a, st, s)) return rc;
     }
-    if (int rc = launch(Stage::Reduce, bits, a, st, s)) return rc;
-    if (P >= 2) {
-        if (int rc = launch(Stage::Gather, bits, a, st, s)) return rc;
-    }
-    return ECHO_OK;
+    return launch(Stage::Reduce, bits, a, st, s);
 }
 
 int echo_check_watchdog(echo_state* st, uint32_t limit_us, echo_stream_t stream) {
@@ -390,13 +387,11 @@ int echo_allreduce_sim_noalloc(const void* const* inputs, void* const* outputs, 
     if (!make_args(&st, bits, inputs, outputs, eta, alpha_long, alpha_short, w, &a)) return ECHO_EINVAL;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(scratch + L.flags_offset, 0, sizeof(uint32_t), s) != cudaSuccess) return ECHO_ECUDA;
+    a.write_outputs = 1;
     if (P >= 2) {
         if (int rc = launch(Stage::Quantize, bits, a, &st, s)) return rc;
     }
     if (int rc = launch(Stage::Reduce, bits, a, &st, s)) return rc;
-    if (P >= 2) {
-        if (int rc = launch(Stage::Gather, bits, a, &st, s)) return rc;
-    }
     if (flags_out) {
         uint32_t f = 0;
         if (cudaStreamSynchronize(s) != cudaSuccess) return ECHO_ECUDA;

@@ -57,6 +57,7 @@ struct Args {
     float eta, w, one_minus_w;
     float a_long, keep_long, a_short, keep_short;
     float one;   // 1.0f, passed at run time (see add_after_mul2 in echo_pipeline.cuh)
+    int write_outputs;   // reduce: also decode into all P outputs (phase 4 in the owner's pass)
 };
 
 // ------------------------------------------------------------------ helpers
@@ -393,6 +394,9 @@ __device__ __forceinline__ void reduce_range(const Args& a, int o, long long j_b
                         yb[4 * h + k] = f2bf16(decode(q[k], g.s, g.z));
                     }
                     store_chunk_codes<BITS>(codes, ln.chunk(h), pack4<BITS>(q));
+                    if (a.write_outputs) {
+                        for (int r = 0; r < a.P; ++r) store_y4(a.out[r], e, a.n, full, &yb[4 * h]);
+                    }
                 }
                 if (ln.t == 0) a.g_params[j] = g.param;
             }

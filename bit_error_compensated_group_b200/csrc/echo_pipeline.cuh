@@ -623,6 +623,14 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
             yb[2 * h + 1] = bf16x2_rn(y23);
         }
         if (ln.t == 0) a.g_params[j] = g.param;
+        if (a.write_outputs) {
+            // phase 4 in the owner's pass: every rank's output gets the decoded
+            // requantized sum -- the same bits a decode of the gathered payload gives
+            for (int r = 0; r < a.P; ++r) {
+                __stcs(reinterpret_cast<uint2*>(a.out[r] + j * GROUP + c0), make_uint2(yb[0], yb[1]));
+                __stcs(reinterpret_cast<uint2*>(a.out[r] + j * GROUP + c1), make_uint2(yb[2], yb[3]));
+            }
+        }
     } else {
         // a single rank sends nothing: its output is its own x'
         raise_flags(a, act && !(lmin >= -65504.0f && lmax <= 65504.0f));

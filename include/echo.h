@@ -175,17 +175,22 @@ ECHO_API int echo_allreduce_sim(const void* const* inputs, void* const* outputs,
                        echo_stream_t stream);
 
 /*
- * The three kernels of echo_allreduce_sim, callable one by one (same
- * arguments and errors; running them in this order on one stream is exactly
- * echo_allreduce_sim):
+ * The phases one by one (same arguments and errors as echo_allreduce_sim):
  *   echo_phase_quantize  phases 1, 2 and 5 for every rank's non-owned groups:
  *                        writes the all-to-all payload and those EMAs
  *                        (does nothing when P == 1)
  *   echo_phase_reduce    phases 1, 3 and 5 for every group's owner: reads the
  *                        all-to-all payload, writes the all-gather payload
- *                        and the owners' EMAs (P == 1: writes outputs[0])
- *   echo_phase_gather    phase 4: reads the all-gather payload, writes all P
- *                        outputs (does nothing when P == 1)
+ *                        and the owners' EMAs. When `outputs` is given (it is
+ *                        required when P == 1) the same pass also performs
+ *                        phase 4: the owner decodes its requantized sum --
+ *                        the very bits of the all-gather payload -- into all
+ *                        P outputs. echo_allreduce_sim is echo_phase_quantize
+ *                        followed by echo_phase_reduce with outputs.
+ *   echo_phase_gather    phase 4 on its own: decodes the all-gather payload
+ *                        into all P outputs (the same result; for callers
+ *                        that ran echo_phase_reduce without outputs; does
+ *                        nothing when P == 1)
  */
 ECHO_API int echo_phase_quantize(const void* const* inputs, echo_state* st, int bits,
                         float eta, float alpha_long, float alpha_short, float w,

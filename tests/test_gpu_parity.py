@@ -132,6 +132,33 @@ def test_phase_entry_points_compose():
         gpu.close()
 
 
+@pytest.mark.parametrize("P,n,group,bits", [(4, 10000, 128, 4), (3, 5000 + 11, 32, 8), (8, 1 << 18, 128, 4)])
+def test_reduce_with_outputs_equals_reduce_then_gather(P, n, group, bits):
+    """Phase 4 in the owner's pass (echo_phase_reduce given outputs) writes
+    exactly what decoding the all-gather payload afterwards writes."""
+    x = _random_inputs(P, n, 40 + P)
+    el0, es0 = _seeded_state(P, n, 41 + P)
+    fb = (1.0, 0.05, 0.5, 0.5)
+    outs = []
+    for fused in (False, True):
+        gpu = GpuEcho(P, n, group, bits)
+        try:
+            gpu.set_inputs(x)
+            gpu.set_state(el0, es0)
+            h = gpu.ar.handle
+            E.echo_phase_quantize(gpu.inputs, h, bits, *fb)
+            if fused:
+                E.echo_phase_reduce(gpu.inputs, gpu.outputs, h, bits, *fb)
+            else:
+                E.echo_phase_reduce(gpu.inputs, None, h, bits, *fb)
+                E.echo_phase_gather(gpu.outputs, h, bits)
+            outs.append((gpu.outputs_u16(), *gpu.state(), *gpu.payload(bits)[2:]))
+        finally:
+            gpu.close()
+    for a, b in zip(*outs):
+        assert np.array_equal(a, b)
+
+
 def test_in_place_outputs():
     P, n = 4, 50000
     x = _random_inputs(P, n, 9)
