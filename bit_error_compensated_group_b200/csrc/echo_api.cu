@@ -90,34 +90,48 @@ enum class Stage { Quantize, Reduce, Gather };
 
 // One pipelined launch; `grid` caches the grid (and the shared-memory opt-in)
 // of this kernel instantiation.
+// An upper bound on the tiles a pipelined launch walks: the runs (2 per rank
+// for quantize, 1 per owner for reduce) cut into tiles of `tile_groups`.
+int64_t tile_bound(Stage stage, const echo_dev::Args& a, int tile_groups) {
+    const int64_t groups = stage == Stage::Quantize ? (int64_t)(a.P - 1) * a.G : a.G;
+    const int64_t runs = stage == Stage::Quantize ? 2 * (int64_t)a.P : a.P;
+    return groups / tile_groups + runs + 1;
+}
+
+// A persistent launch never needs more CTAs than tiles: small messages then
+// start only the CTAs that have work.
 template <typename K>
-int launch_pipe(K kernel, int* grid, const echo_dev::Args& a, const echo_state* st, cudaStream_t s) {
+int launch_pipe(K kernel, int* grid, int64_t max_tiles, const echo_dev::Args& a, const echo_state* st,
+                cudaStream_t s) {
     if (*grid == 0) *grid = pipe_grid(kernel, st);
     if (*grid == 0) return ECHO_ECUDA;
-    kernel<<<*grid, echo_dev::kPipeThreads, echo_dev::kPipeSmem, s>>>(a);
+    const int g = (int)(max_tiles < (int64_t)*grid ? max_tiles : (int64_t)*grid);
+    kernel<<<g, echo_dev::kPipeThreads, echo_dev::kPipeSmem, s>>>(a);
     return ECHO_OK;
 }
 
 template <int GROUP, int BITS>
 int launch_stage(Stage stage, const echo_dev::Args& a, const echo_state* st, cudaStream_t s) {
     int rc = ECHO_OK;
+    // tiles of 2048 elements with feedback, 5 x 2048 without (see RunWalker)
+    const int64_t tiles = tile_bound(stage, a, (a.state ? 1 : 5) * echo_dev::kTileElems / GROUP);
     switch (stage) {
         case Stage::Quantize:
             if (a.state) {
                 static int grid = 0;
-                rc = launch_pipe(echo_dev::k_quantize_tma<GROUP, BITS, true>, &grid, a, st, s);
+                rc = launch_pipe(echo_dev::k_quantize_tma<GROUP, BITS, true>, &grid, tiles, a, st, s);
             } else {
                 static int grid = 0;
-                rc = launch_pipe(echo_dev::k_quantize_tma<GROUP, BITS, false>, &grid, a, st, s);
+                rc = launch_pipe(echo_dev::k_quantize_tma<GROUP, BITS, false>, &grid, tiles, a, st, s);
             }
             break;
         case Stage::Reduce:
             if (a.state) {
                 static int grid = 0;
-                rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, true>, &grid, a, st, s);
+                rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, true>, &grid, tiles, a, st, s);
             } else {
                 static int grid = 0;
-                rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, false>, &grid, a, st, s);
+                rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, false>, &grid, tiles, a, st, s);
             }
             break;
         case Stage::Gather: {
