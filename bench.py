@@ -211,9 +211,12 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+_FEEDBACK = True   # --feedback off: the main step runs without EMA state (profiling that variant)
+
+
 def _config(w):
     return {"workload": w.name, "P": w.P, "n": w.n, "tokens": w.tokens, "hidden": w.hidden, "group": w.group,
-            "bits": w.bits, "feedback": True, "eta": w.eta, "alpha_long": w.alpha_long,
+            "bits": w.bits, "feedback": _FEEDBACK, "eta": w.eta, "alpha_long": w.alpha_long,
             "alpha_short": w.alpha_short, "w": w.w, "values": "Student-t nu=3 / sqrt(3)",
             "l2": "no flush: each step touches ~90 GB, far larger than the 126 MB L2"}
 
@@ -235,7 +238,7 @@ def run_gpu(args):
 
     w = _workload()
     P, n, group, bits = w.P, w.n, w.group, w.bits
-    ar = E.EchoAllReduce(n, P, group, bits, feedback=True, device=dev)
+    ar = E.EchoAllReduce(n, P, group, bits, feedback=_FEEDBACK, device=dev)
     inputs = []
     for r in range(P):
         inputs.append(W.rank_input(w, r, site=rank, device=dev))   # each GPU its own message
@@ -285,26 +288,33 @@ def run_gpu(args):
     # time and the difference, the cost of compensation (the pages quote
     # 0.90 ms per 1 GB message on 8 A100s, fused into the entry pass)
     variant = None
-    if not args.no_variants:
+    if not args.no_variants and _FEEDBACK:
         nf = E.EchoAllReduce(n, P, group, bits, feedback=False, device=dev)
         nf_steps = max(3, min(args.steps, 10))
 
-        def nf_step():
-            E.echo_allreduce_sim(inputs, outputs, nf.handle, n, P, bits, group, *fb, stream=stream)
+        def nf_step(ev=None):
+            if ev is not None:
+                ev[0].record(stream)
+            E.echo_phase_quantize(inputs, nf.handle, bits, *fb, stream=stream)
+            if ev is not None:
+                ev[1].record(stream)
+            E.echo_phase_reduce(inputs, outputs, nf.handle, bits, *fb, stream=stream)
+            if ev is not None:
+                ev[2].record(stream)
 
         for _ in range(args.warmup):
             nf_step()
         barrier()
-        a0, b0 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a0.record(stream)
-        for _ in range(nf_steps):
-            nf_step()
-        b0.record(stream)
+        nf_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nf_steps)]
+        for i in range(nf_steps):
+            nf_step(nf_evs[i])
         barrier()
-        nf_ms = max_over_ranks(a0.elapsed_time(b0), world, dev) / nf_steps
+        nf_ms = max_over_ranks(nf_evs[0][0].elapsed_time(nf_evs[-1][2]), world, dev) / nf_steps
+        nf_phases = {"quantize": sum(e[0].elapsed_time(e[1]) for e in nf_evs) / nf_steps,
+                     "reduce_gather": sum(e[1].elapsed_time(e[2]) for e in nf_evs) / nf_steps}
         nf.close()
         del nf
-        variant = {"ms_per_step": nf_ms, "steps": nf_steps,
+        variant = {"ms_per_step": nf_ms, "steps": nf_steps, "phases_ms": nf_phases,
                    "value": weak_scaling_gbs(world, P * n * 2, nf_ms),
                    "roofline_frac": algorithmic_bytes(P, n, group, bits, feedback=False)["total"] / (nf_ms * 1e-3)
                    / 1e9 / _peak_hbm()[0]}
@@ -343,10 +353,10 @@ def run_gpu(args):
         ms = max_ms / args.steps
         value = weak_scaling_gbs(world, P * n * 2, ms)
         peak, peak_kind = _peak_hbm()
-        ab = algorithmic_bytes(P, n, group, bits)
+        ab = algorithmic_bytes(P, n, group, bits, feedback=_FEEDBACK)
         q_ms = per_phase["quantize"] / args.steps
         achieved = ab["quantize"] / (q_ms * 1e-3) / 1e9
-        traffic = _measured_traffic()
+        traffic = _measured_traffic() if _FEEDBACK else None
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -386,11 +396,14 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-variants", action="store_true", help="skip the no-feedback timing")
+    ap.add_argument("--feedback", choices=["on", "off"], default="on",
+                    help="off: time the call without EMA state as the main step (profiling)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="tokens per rank (default 131072, the 1 GB message); smaller values are for profiling")
     args = ap.parse_args()
-    global _TOKENS
+    global _TOKENS, _FEEDBACK
     _TOKENS = args.tokens
+    _FEEDBACK = args.feedback == "on"
     if args.impl == "reference":
         run_reference(args)
     else:
