@@ -113,8 +113,12 @@ int launch_pipe(K kernel, int* grid, int64_t max_tiles, const echo_dev::Args& a,
 template <int GROUP, int BITS>
 int launch_stage(Stage stage, const echo_dev::Args& a, const echo_state* st, cudaStream_t s) {
     int rc = ECHO_OK;
-    // tiles of 2048 elements with feedback, 5 x 2048 without (see RunWalker)
-    const int64_t tiles = tile_bound(stage, a, (a.state ? 1 : 5) * echo_dev::kTileElems / GROUP);
+    // tiles of 2048 elements with feedback; without, 4 x 2048 (quantize) and
+    // 5 x 2048 (reduce) -- the sub-tile counts of the kernels' RunWalkers
+    const int subtiles = a.state ? 1
+                         : stage == Stage::Quantize ? echo_dev::kQuantizeSubtilesNF
+                                                    : echo_dev::kReduceSubtilesNF;
+    const int64_t tiles = tile_bound(stage, a, subtiles * echo_dev::kTileElems / GROUP);
     switch (stage) {
         case Stage::Quantize:
             if (a.state) {

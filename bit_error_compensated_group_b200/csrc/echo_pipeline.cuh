@@ -327,14 +327,9 @@ struct GridP {
     bool bad;   // a value outside [-65504, 65504] or a NaN
 };
 
-template <int L, int Q>
-__device__ __forceinline__ GridP make_grid_p(float lane_min, float lane_max) {
-    float mn = lane_min, mx = lane_max;
-#pragma unroll
-    for (int o = L / 2; o > 0; o >>= 1) {
-        mn = nan_min(mn, __shfl_xor_sync(kFull, mn, o));
-        mx = nan_max(mx, __shfl_xor_sync(kFull, mx, o));
-    }
+// fp16 parameters of a group from its range [mn, mx] (same values as make_grid).
+template <int Q>
+__device__ __forceinline__ GridP grid_from_range(float mn, float mx) {
     GridP g;
     g.bad = !(mn >= -65504.0f && mx <= 65504.0f);
     mn = __fadd_rn(mn, 0.0f);   // -0 -> +0
@@ -351,6 +346,17 @@ __device__ __forceinline__ GridP make_grid_p(float lane_min, float lane_max) {
     g.inv = splat(inv);
     g.param = (uint32_t)__half_as_ushort(sh) | ((uint32_t)__half_as_ushort(zh) << 16);
     return g;
+}
+
+template <int L, int Q>
+__device__ __forceinline__ GridP make_grid_p(float lane_min, float lane_max) {
+    float mn = lane_min, mx = lane_max;
+#pragma unroll
+    for (int o = L / 2; o > 0; o >>= 1) {
+        mn = nan_min(mn, __shfl_xor_sync(kFull, mn, o));
+        mx = nan_max(mx, __shfl_xor_sync(kFull, mx, o));
+    }
+    return grid_from_range<Q>(mn, mx);
 }
 
 // p + q where p (or q) is a rounded product: fma(p, one, q), one = 1.0 at run time
@@ -484,10 +490,112 @@ __device__ __forceinline__ void quantize_tile_group(const Args& a, const uint8_t
     if (ln.t == 0) a.a2a_params[(size_t)r * a.G + j] = g.param;
 }
 
+// Without feedback the quantizer reads bf16 values only, and the per-group
+// work (range reduction, fp16 parameters, two divisions) dominates the issue
+// slots. This path gives each lane 16 elements (two 8-element chunks t and
+// t + L16) so that the group work is shared by twice as many elements, and
+// takes the group range on packed bf16 pairs: bf16 -> binary32 is exact and
+// order-preserving, so min/max on bf16 gives the same values. Lane minima and
+// negated maxima travel as one bf16x2 word (min, -max), reduced with a single
+// min per shuffle round (max(x) = -min(-x) exactly, and min.NaN keeps NaNs).
+template <int GROUP>
+struct Lane16 {
+    static constexpr int L = GROUP / 16;     // lanes per group
+    static constexpr int GPW = 32 / L;       // groups per warp
+    int sub, t;
+    __device__ __forceinline__ Lane16() {
+        const int lane = threadIdx.x & 31;
+        sub = lane / L;
+        t = lane % L;
+    }
+    __device__ __forceinline__ int chunk(int h) const { return t + h * L; }   // 8-element chunk
+};
+
+constexpr int kQuantizeSubtilesNF = 4;   // 8192 elements per tile: two passes of 8 warps x 32 lanes x 16
+constexpr int kReduceSubtilesNF = 5;
+
+__device__ __forceinline__ uint32_t bmin2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("min.NaN.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.NaN.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+__device__ __forceinline__ float2 bf16_pair(uint32_t u) { return make_float2(bf16_lo(u), bf16_hi(u)); }
+
+// eight codes (2^23 + code each, in four pairs) -> packed bytes: one word at
+// 4 bits, two at 8 bits. Only the low byte of each float's bit pattern is
+// used; at 4 bits (hi << 4) + lo puts code 2i + 1 above code 2i without a
+// carry out of the byte (both codes <= 15).
+template <int BITS>
+__device__ __forceinline__ uint2 pack_codes8(const float2 t[4]) {
+    uint2 out;
+    if (BITS == 4) {
+        uint32_t b[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) b[k] = (__float_as_uint(t[k].y) << 4) + __float_as_uint(t[k].x);
+        out.x = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+        out.y = 0;
+    } else {
+        const uint32_t p0 = __byte_perm(__float_as_uint(t[0].x), __float_as_uint(t[0].y), 0x0040);
+        const uint32_t p1 = __byte_perm(__float_as_uint(t[1].x), __float_as_uint(t[1].y), 0x0040);
+        const uint32_t p2 = __byte_perm(__float_as_uint(t[2].x), __float_as_uint(t[2].y), 0x0040);
+        const uint32_t p3 = __byte_perm(__float_as_uint(t[3].x), __float_as_uint(t[3].y), 0x0040);
+        out.x = __byte_perm(p0, p1, 0x5410);
+        out.y = __byte_perm(p2, p3, 0x5410);
+    }
+    return out;
+}
+
+template <int GROUP, int BITS>
+__device__ __forceinline__ void quantize_tile_group_nf(const Args& a, const uint8_t* st, const Tile& t, int gi,
+                                                       bool act) {
+    using LN = Lane16<GROUP>;
+    constexpr int L = LN::L, Q = (1 << BITS) - 1, CB = GROUP * BITS / 8;
+    const LN ln;
+    const uint4* xs = reinterpret_cast<const uint4*>(st + (size_t)gi * GROUP * 2);
+    uint4 w[2];
+    uint32_t mm = 0x7F807F80u;   // (+inf, -(-inf)): neutral for an inactive group
+    if (act) {
+        w[0] = xs[ln.chunk(0)];
+        w[1] = xs[ln.chunk(1)];
+        const uint32_t lo = bmin2(bmin2(bmin2(w[0].x, w[0].y), bmin2(w[0].z, w[0].w)),
+                                  bmin2(bmin2(w[1].x, w[1].y), bmin2(w[1].z, w[1].w)));
+        const uint32_t hi = bmax2(bmax2(bmax2(w[0].x, w[0].y), bmax2(w[0].z, w[0].w)),
+                                  bmax2(bmax2(w[1].x, w[1].y), bmax2(w[1].z, w[1].w)));
+        // (lo.even, -hi.even) and (lo.odd, -hi.odd) -> (lane min, -lane max)
+        mm = bmin2(__byte_perm(lo, hi, 0x5410) ^ 0x80000000u, __byte_perm(lo, hi, 0x7632) ^ 0x80000000u);
+    }
+#pragma unroll
+    for (int o = L / 2; o > 0; o >>= 1) mm = bmin2(mm, __shfl_xor_sync(kFull, mm, o));
+    const GridP g = grid_from_range<Q>(__uint_as_float(mm << 16), __uint_as_float((mm & 0xffff0000u) ^ 0x80000000u));
+    raise_flags(a, act && g.bad);
+    if (!act) return;
+    const long long j = t.j0 + gi;
+    uint8_t* codes = a.a2a_codes + ((size_t)t.rank * a.G + j) * CB;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        float2 e[4];
+        e[0] = encode2(bf16_pair(w[h].x), g, a);
+        e[1] = encode2(bf16_pair(w[h].y), g, a);
+        e[2] = encode2(bf16_pair(w[h].z), g, a);
+        e[3] = encode2(bf16_pair(w[h].w), g, a);
+        const uint2 pk = pack_codes8<BITS>(e);
+        if (BITS == 4) *reinterpret_cast<uint32_t*>(codes + 4 * ln.chunk(h)) = pk.x;
+        else *reinterpret_cast<uint2*>(codes + 8 * ln.chunk(h)) = pk;
+    }
+    if (ln.t == 0) a.a2a_params[(size_t)t.rank * a.G + j] = g.param;
+}
+
 template <int GROUP, int BITS, bool FB>
 __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
-    constexpr int M = FB ? 1 : 5;
+    constexpr int M = FB ? 1 : kQuantizeSubtilesNF;
     const PipeShared p = pipe_shared(smem);
     pipe_init(p);
     const int warp = threadIdx.x >> 5;
@@ -497,8 +605,11 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
         if ((threadIdx.x & 31) == 0) produce<GROUP, M>(a, p, walker, FB);
         return;
     }
-    constexpr int GPW = Lane<GROUP>::GPW;
-    const int gi = warp * GPW + Lane<GROUP>().sub;   // + m * kConsumerWarps * GPW for sub-tile m
+    // with feedback: 8 elements per lane, one pass per tile; without: 16 per
+    // lane, two passes over the 4-sub-tile stage
+    constexpr int GPW = FB ? Lane<GROUP>::GPW : Lane16<GROUP>::GPW;
+    constexpr int PASSES = FB ? 1 : M * kTileElems / (kConsumerWarps * 32 * 16);
+    const int gi = warp * GPW + (FB ? Lane<GROUP>().sub : Lane16<GROUP>().sub);
     long long i = 0;
     Tile t;
     for (long long k = blockIdx.x; walker.locate(k, &t); k += gridDim.x, ++i) {
@@ -507,10 +618,15 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
             if ((threadIdx.x & 31) == 0) report_timeout(a, p);
             return;
         }
+        const uint8_t* stage = p.stages + (size_t)s * kStageBytes;
+        if (FB) {
+            quantize_tile_group<GROUP, BITS, true>(a, stage, t, gi, gi < t.count);
+        } else {
 #pragma unroll 1
-        for (int m = 0; m < M; ++m) {
-            const int g = gi + m * kConsumerWarps * GPW;
-            quantize_tile_group<GROUP, BITS, FB>(a, p.stages + (size_t)s * kStageBytes, t, g, g < t.count);
+            for (int m = 0; m < PASSES; ++m) {
+                const int g = gi + m * kConsumerWarps * GPW;
+                quantize_tile_group_nf<GROUP, BITS>(a, stage, t, g, g < t.count);
+            }
         }
         __syncwarp();
         if ((threadIdx.x & 31) == 0) mbar_arrive(&p.empty[s]);
@@ -664,7 +780,7 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
 template <int GROUP, int BITS, bool FB>
 __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
-    constexpr int M = FB ? 1 : 5;
+    constexpr int M = FB ? 1 : kReduceSubtilesNF;
     const PipeShared p = pipe_shared(smem);
     pipe_init(p);
     const int warp = threadIdx.x >> 5;

@@ -175,13 +175,17 @@ def test_in_place_outputs():
 
 
 @pytest.mark.parametrize("feedback", [True, False])
-def test_range_flag_and_recovery(feedback):
-    """A value outside the fp16 parameter range raises the sticky flag;
-    echo_get_status reports and clears it. The EMAs of a flagged group are
-    unspecified, so the recovery call starts from fresh state."""
+@pytest.mark.parametrize("bad", [1e6, -1e6, float("nan"), float("-inf")])
+@pytest.mark.parametrize("rank", [0, 1])
+def test_range_flag_and_recovery(feedback, bad, rank):
+    """A value outside the fp16 parameter range (or a NaN) raises the sticky
+    flag, from a non-owned group (rank 1: the quantize pass) or an owned one
+    (rank 0: the owner's sum); echo_get_status reports and clears it. The EMAs
+    of a flagged group are unspecified, so the recovery call starts from fresh
+    state."""
     P, n = 2, 4096
     x = _random_inputs(P, n, 10)
-    x[1, 1234] = 1e6
+    x[rank, 1234] = bad
     gpu = GpuEcho(P, n, feedback=feedback)
     try:
         gpu.set_inputs(x)
@@ -190,7 +194,7 @@ def test_range_flag_and_recovery(feedback):
         assert rc == E.ECHO_ERANGE and flags & E.ECHO_FLAG_RANGE
         rc, flags = gpu.status()                     # cleared by the read
         assert rc == E.ECHO_OK and flags == 0
-        x[1, 1234] = 0.5
+        x[rank, 1234] = 0.5
         gpu.set_inputs(x)
         if feedback:
             gpu.set_state(np.zeros((P, n), np.float32), np.zeros((P, n), np.float32))
