@@ -512,7 +512,7 @@ struct Lane16 {
 };
 
 constexpr int kQuantizeSubtilesNF = 4;   // 8192 elements per tile: two passes of 8 warps x 32 lanes x 16
-constexpr int kReduceSubtilesNF = 5;
+constexpr int kReduceSubtilesNF = 4;
 
 __device__ __forceinline__ uint32_t bmin2(uint32_t a, uint32_t b) {
     uint32_t r;
@@ -777,6 +777,165 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
     }
 }
 
+// eight packed codes (one word at 4 bits, two at 8) -> four exact float pairs
+template <int BITS>
+__device__ __forceinline__ void unpack_codes8(const uint32_t* w, float2 q[4]) {
+    uint32_t ev[4], od[4];   // 2^23 + code of elements 2p and 2p + 1
+    if (BITS == 4) {
+        const uint32_t lo = w[0] & 0x0F0F0F0Fu;          // codes 0, 2, 4, 6 in bytes 0..3
+        const uint32_t hi = (w[0] >> 4) & 0x0F0F0F0Fu;   // codes 1, 3, 5, 7
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            ev[p] = __byte_perm(lo, 0x4B000000u, 0x7650 + p);
+            od[p] = __byte_perm(hi, 0x4B000000u, 0x7650 + p);
+        }
+    } else {
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            ev[p] = __byte_perm(w[p >> 1], 0x4B000000u, 0x7650 + 2 * (p & 1));
+            od[p] = __byte_perm(w[p >> 1], 0x4B000000u, 0x7651 + 2 * (p & 1));
+        }
+    }
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+        q[p] = add2_rn(make_float2(__uint_as_float(ev[p]), __uint_as_float(od[p])), splat(-kMagic));
+}
+
+__device__ __forceinline__ float nan_min3(float a, float b, float c) {
+    float r;
+    asm("min.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+__device__ __forceinline__ float nan_max3(float a, float b, float c) {
+    float r;
+    asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// The owner's pass without feedback, 16 elements per lane (chunks t and
+// t + L16 of 8 elements): twice the elements per payload load batch and per
+// group-level step of the 8-element path, and 16-byte output stores.
+template <int GROUP, int BITS>
+__device__ __forceinline__ void reduce_tile_group_nf(const Args& a, const uint8_t* st, const Tile& t, int gi,
+                                                     bool act) {
+    using LN = Lane16<GROUP>;
+    constexpr int L = LN::L, Q = (1 << BITS) - 1, CB = GROUP * BITS / 8;
+    constexpr int RB = BITS == 4 ? 8 : 4;   // ranks whose payload loads are issued together
+    constexpr int CW = BITS / 4;            // 32-bit code words per 8-element chunk
+    const LN ln;
+    const int o = t.rank;
+    const long long j = t.j0 + gi;
+    const uint4* xs = reinterpret_cast<const uint4*>(st + (size_t)gi * GROUP * 2);
+    uint4 xw[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+    if (act) {
+        xw[0] = xs[ln.chunk(0)];
+        xw[1] = xs[ln.chunk(1)];
+    }
+    float2 acc[8];
+#pragma unroll
+    for (int p = 0; p < 8; ++p) acc[p] = make_float2(0.0f, 0.0f);
+    // binary32 sum in rank order 0..P-1: own x unquantized, others decoded
+    for (int r0 = 0; r0 < a.P; r0 += RB) {
+        uint32_t cw[RB][2 * CW];
+        uint32_t pw[RB];
+#pragma unroll
+        for (int k = 0; k < RB; ++k) {
+            const int r = r0 + k;
+            pw[k] = 0u;
+#pragma unroll
+            for (int c = 0; c < 2 * CW; ++c) cw[k][c] = 0u;
+            if (act && r < a.P && r != o) {
+                const size_t slot = (size_t)r * a.G + j;
+                const uint8_t* codes = a.a2a_codes + slot * CB;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    if (BITS == 4) {
+                        cw[k][h] = *reinterpret_cast<const uint32_t*>(codes + 4 * ln.chunk(h));
+                    } else {
+                        const uint2 v = *reinterpret_cast<const uint2*>(codes + 8 * ln.chunk(h));
+                        cw[k][2 * h] = v.x;
+                        cw[k][2 * h + 1] = v.y;
+                    }
+                }
+                pw[k] = a.a2a_params[slot];
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < RB; ++k) {
+            const int r = r0 + k;
+            if (r >= a.P) break;
+            float2 term[8];
+            if (r == o) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    term[4 * h] = bf16_pair(xw[h].x);
+                    term[4 * h + 1] = bf16_pair(xw[h].y);
+                    term[4 * h + 2] = bf16_pair(xw[h].z);
+                    term[4 * h + 3] = bf16_pair(xw[h].w);
+                }
+            } else {
+                const float2 s2 = splat(param_s(pw[k]));
+                const float2 z2 = splat(param_z(pw[k]));
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    float2 q[4];
+                    unpack_codes8<BITS>(&cw[k][h * CW], q);
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) term[4 * h + p] = fma2_rn(q[p], s2, z2);
+                }
+            }
+#pragma unroll
+            for (int p = 0; p < 8; ++p) acc[p] = (r == 0) ? term[p] : add2_rn(acc[p], term[p]);
+        }
+    }
+    float lmin = __int_as_float(0x7f800000), lmax = -__int_as_float(0x7f800000);
+    if (act) {
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+            lmin = nan_min3(lmin, acc[p].x, acc[p].y);
+            lmax = nan_max3(lmax, acc[p].x, acc[p].y);
+        }
+    }
+    uint32_t yw[8];   // bf16 pairs of the result
+    if (a.P >= 2) {
+        const GridP g = make_grid_p<L, Q>(lmin, lmax);
+        raise_flags(a, act && g.bad);
+        if (!act) return;
+        uint8_t* codes = a.g_codes + (size_t)j * CB;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float2 e[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) e[p] = encode2(acc[4 * h + p], g, a);
+            const uint2 pk = pack_codes8<BITS>(e);
+            if (BITS == 4) *reinterpret_cast<uint32_t*>(codes + 4 * ln.chunk(h)) = pk.x;
+            else *reinterpret_cast<uint2*>(codes + 8 * ln.chunk(h)) = pk;
+#pragma unroll
+            for (int p = 0; p < 4; ++p) yw[4 * h + p] = bf16x2_rn(fma2_rn(add2_rn(e[p], splat(-kMagic)), g.s, g.z));
+        }
+        if (ln.t == 0) a.g_params[j] = g.param;
+        if (a.write_outputs) {
+            // phase 4 in the owner's pass: every rank's output gets the decoded
+            // requantized sum -- the same bits a decode of the gathered payload gives
+            for (int r = 0; r < a.P; ++r) {
+                uint16_t* y = a.out[r] + j * GROUP;
+                __stcs(reinterpret_cast<uint4*>(y + 8 * ln.chunk(0)), make_uint4(yw[0], yw[1], yw[2], yw[3]));
+                __stcs(reinterpret_cast<uint4*>(y + 8 * ln.chunk(1)), make_uint4(yw[4], yw[5], yw[6], yw[7]));
+            }
+        }
+    } else {
+        // a single rank sends nothing: its output is its own x
+        raise_flags(a, act && !(lmin >= -65504.0f && lmax <= 65504.0f));
+        if (!act) return;
+#pragma unroll
+        for (int p = 0; p < 8; ++p) yw[p] = bf16x2_rn(acc[p]);
+        uint16_t* y = a.out[0] + j * GROUP;
+        *reinterpret_cast<uint4*>(y + 8 * ln.chunk(0)) = make_uint4(yw[0], yw[1], yw[2], yw[3]);
+        *reinterpret_cast<uint4*>(y + 8 * ln.chunk(1)) = make_uint4(yw[4], yw[5], yw[6], yw[7]);
+    }
+}
+
 template <int GROUP, int BITS, bool FB>
 __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -790,8 +949,11 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
         if ((threadIdx.x & 31) == 0) produce<GROUP, M>(a, p, walker, FB);
         return;
     }
-    constexpr int GPW = Lane<GROUP>::GPW;
-    const int gi = warp * GPW + Lane<GROUP>().sub;   // + m * kConsumerWarps * GPW for sub-tile m
+    // with feedback: 8 elements per lane, one pass per tile; without: 16 per
+    // lane, two passes over the 4-sub-tile stage
+    constexpr int GPW = FB ? Lane<GROUP>::GPW : Lane16<GROUP>::GPW;
+    constexpr int PASSES = FB ? 1 : M * kTileElems / (kConsumerWarps * 32 * 16);
+    const int gi = warp * GPW + (FB ? Lane<GROUP>().sub : Lane16<GROUP>().sub);
     long long i = 0;
     Tile t;
     for (long long k = blockIdx.x; walker.locate(k, &t); k += gridDim.x, ++i) {
@@ -800,10 +962,15 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
             if ((threadIdx.x & 31) == 0) report_timeout(a, p);
             return;
         }
+        const uint8_t* stage = p.stages + (size_t)s * kStageBytes;
+        if (FB) {
+            reduce_tile_group<GROUP, BITS, true>(a, stage, t, gi, gi < t.count);
+        } else {
 #pragma unroll 1
-        for (int m = 0; m < M; ++m) {
-            const int g = gi + m * kConsumerWarps * GPW;
-            reduce_tile_group<GROUP, BITS, FB>(a, p.stages + (size_t)s * kStageBytes, t, g, g < t.count);
+            for (int m = 0; m < PASSES; ++m) {
+                const int g = gi + m * kConsumerWarps * GPW;
+                reduce_tile_group_nf<GROUP, BITS>(a, stage, t, g, g < t.count);
+            }
         }
         __syncwarp();
         if ((threadIdx.x & 31) == 0) mbar_arrive(&p.empty[s]);
