@@ -218,7 +218,8 @@ def _config(w):
     return {"workload": w.name, "P": w.P, "n": w.n, "tokens": w.tokens, "hidden": w.hidden, "group": w.group,
             "bits": w.bits, "feedback": _FEEDBACK, "eta": w.eta, "alpha_long": w.alpha_long,
             "alpha_short": w.alpha_short, "w": w.w, "values": "Student-t nu=3 / sqrt(3)",
-            "l2": "no flush: each step touches ~90 GB, far larger than the 126 MB L2"}
+            "l2": "no flush: each step touches %.0f GB, far larger than the 126 MB L2"
+                  % (algorithmic_bytes(w.P, w.n, w.group, w.bits, _FEEDBACK)["total"] / 1e9)}
 
 
 def run_gpu(args):

@@ -436,7 +436,9 @@ __device__ __forceinline__ void store_f4_pair(float* p, float2 lo, float2 hi) {
 
 // ------------------------------------------------------------ quantize
 
-template <int GROUP, int BITS, bool FB>
+// One non-owned group of a tile with feedback (x, e_long, e_short staged):
+// 8 elements per lane, chunks t and t + L of 4.
+template <int GROUP, int BITS>
 __device__ __forceinline__ void quantize_tile_group(const Args& a, const uint8_t* st, const Tile& t, int gi,
                                                     bool act) {
     using LN = Lane<GROUP>;
@@ -452,12 +454,10 @@ __device__ __forceinline__ void quantize_tile_group(const Args& a, const uint8_t
     float lmin = __int_as_float(0x7f800000), lmax = -__int_as_float(0x7f800000);
     if (act) {
         load_x8_smem(xs, c0, c1, v);
-        if (FB) {
-            load_f8_smem(els, c0, c1, el);
-            load_f8_smem(ess, c0, c1, es);
+        load_f8_smem(els, c0, c1, el);
+        load_f8_smem(ess, c0, c1, es);
 #pragma unroll
-            for (int p = 0; p < 4; ++p) v[p] = inject2(v[p], el[p], es[p], a);
-        }
+        for (int p = 0; p < 4; ++p) v[p] = inject2(v[p], el[p], es[p], a);
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
             lmin = nan_min(lmin, nan_min(v[p].x, v[p].y));
@@ -468,50 +468,54 @@ __device__ __forceinline__ void quantize_tile_group(const Args& a, const uint8_t
     raise_flags(a, act && g.bad);
     if (!act) return;
     uint8_t* codes = a.a2a_codes + ((size_t)r * a.G + j) * CB;
-    float* el_g = FB ? a.state + (size_t)r * 2 * a.S + j * GROUP : nullptr;
+    float* el_g = a.state + (size_t)r * 2 * a.S + j * GROUP;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const float2 t01 = encode2(v[2 * h], g, a);
         const float2 t23 = encode2(v[2 * h + 1], g, a);
         store_chunk_codes<BITS>(codes, ln.chunk(h), pack_codes4<BITS>(t01, t23));
-        if (FB) {
-            // residual x' - x_hat with x_hat = code*s + z (fused: code*s is exact)
-            const float2 q01 = add2_rn(t01, splat(-kMagic));
-            const float2 q23 = add2_rn(t23, splat(-kMagic));
-            const float2 rho01 = add2_rn(v[2 * h], fma2_rn(q01, g.ns, g.nz));
-            const float2 rho23 = add2_rn(v[2 * h + 1], fma2_rn(q23, g.ns, g.nz));
-            const int c = h ? c1 : c0;
-            store_f4_pair(el_g + c, ema2(el[2 * h], rho01, a.keep_long, a.a_long, a),
-                          ema2(el[2 * h + 1], rho23, a.keep_long, a.a_long, a));
-            store_f4_pair(el_g + a.S + c, ema2(es[2 * h], rho01, a.keep_short, a.a_short, a),
-                          ema2(es[2 * h + 1], rho23, a.keep_short, a.a_short, a));
-        }
+        // residual x' - x_hat with x_hat = code*s + z (fused: code*s is exact)
+        const float2 q01 = add2_rn(t01, splat(-kMagic));
+        const float2 q23 = add2_rn(t23, splat(-kMagic));
+        const float2 rho01 = add2_rn(v[2 * h], fma2_rn(q01, g.ns, g.nz));
+        const float2 rho23 = add2_rn(v[2 * h + 1], fma2_rn(q23, g.ns, g.nz));
+        const int c = h ? c1 : c0;
+        store_f4_pair(el_g + c, ema2(el[2 * h], rho01, a.keep_long, a.a_long, a),
+                      ema2(el[2 * h + 1], rho23, a.keep_long, a.a_long, a));
+        store_f4_pair(el_g + a.S + c, ema2(es[2 * h], rho01, a.keep_short, a.a_short, a),
+                      ema2(es[2 * h + 1], rho23, a.keep_short, a.a_short, a));
     }
     if (ln.t == 0) a.a2a_params[(size_t)r * a.G + j] = g.param;
 }
 
 // Without feedback the quantizer reads bf16 values only, and the per-group
 // work (range reduction, fp16 parameters, two divisions) dominates the issue
-// slots. This path gives each lane 16 elements (two 8-element chunks t and
-// t + L16) so that the group work is shared by twice as many elements, and
-// takes the group range on packed bf16 pairs: bf16 -> binary32 is exact and
-// order-preserving, so min/max on bf16 gives the same values. Lane minima and
-// negated maxima travel as one bf16x2 word (min, -max), reduced with a single
-// min per shuffle round (max(x) = -min(-x) exactly, and min.NaN keeps NaNs).
-template <int GROUP>
-struct Lane16 {
-    static constexpr int L = GROUP / 16;     // lanes per group
+// slots. These paths give each lane E = 16 or 32 elements (E/8 chunks of 8:
+// t, t + L, t + 2L, ...) so that the group work is shared by more elements,
+// and the quantizer takes the group range on packed bf16 pairs: bf16 ->
+// binary32 is exact and order-preserving, so min/max on bf16 gives the same
+// values. Lane minima and negated maxima travel as one bf16x2 word (min, -max),
+// reduced with a single min per shuffle round (max(x) = -min(-x) exactly, and
+// min.NaN keeps NaNs).
+template <int GROUP, int E>
+struct LaneE {
+    static constexpr int L = GROUP / E;      // lanes per group
     static constexpr int GPW = 32 / L;       // groups per warp
+    static constexpr int H = E / 8;          // 8-element chunks per lane
     int sub, t;
-    __device__ __forceinline__ Lane16() {
+    __device__ __forceinline__ LaneE() {
         const int lane = threadIdx.x & 31;
         sub = lane / L;
         t = lane % L;
     }
-    __device__ __forceinline__ int chunk(int h) const { return t + h * L; }   // 8-element chunk
+    __device__ __forceinline__ int chunk(int h) const { return t + h * L; }
 };
 
-constexpr int kQuantizeSubtilesNF = 4;   // 8192 elements per tile: two passes of 8 warps x 32 lanes x 16
+template <int GROUP>
+using Lane16 = LaneE<GROUP, 16>;
+
+constexpr int kQuantizeLaneElemsNF = 32;
+constexpr int kQuantizeSubtilesNF = 4;   // 8192 elements per tile: one pass of 8 warps x 32 lanes x 32
 constexpr int kReduceSubtilesNF = 4;
 
 __device__ __forceinline__ uint32_t bmin2(uint32_t a, uint32_t b) {
@@ -555,19 +559,28 @@ __device__ __forceinline__ uint2 pack_codes8(const float2 t[4]) {
 template <int GROUP, int BITS>
 __device__ __forceinline__ void quantize_tile_group_nf(const Args& a, const uint8_t* st, const Tile& t, int gi,
                                                        bool act) {
-    using LN = Lane16<GROUP>;
-    constexpr int L = LN::L, Q = (1 << BITS) - 1, CB = GROUP * BITS / 8;
+    using LN = LaneE<GROUP, kQuantizeLaneElemsNF>;
+    constexpr int L = LN::L, H = LN::H, Q = (1 << BITS) - 1, CB = GROUP * BITS / 8;
     const LN ln;
+    // Chunk order per group (h ^ flip): when a quarter-warp spans several
+    // groups, each takes a different chunk at a time, so that the 16-byte
+    // shared-memory reads of those 8 lanes fall in distinct banks (groups of
+    // 32 elements at an odd index are 16 banks apart already).
+    constexpr int QG = L >= 8 ? 1 : 8 / L;   // groups per quarter-warp
+    const int flip = (GROUP == 32 ? (ln.sub >> 1) : (ln.sub & (QG - 1))) & (H - 1);
     const uint4* xs = reinterpret_cast<const uint4*>(st + (size_t)gi * GROUP * 2);
-    uint4 w[2];
+    uint4 w[H];
     uint32_t mm = 0x7F807F80u;   // (+inf, -(-inf)): neutral for an inactive group
     if (act) {
-        w[0] = xs[ln.chunk(0)];
-        w[1] = xs[ln.chunk(1)];
-        const uint32_t lo = bmin2(bmin2(bmin2(w[0].x, w[0].y), bmin2(w[0].z, w[0].w)),
-                                  bmin2(bmin2(w[1].x, w[1].y), bmin2(w[1].z, w[1].w)));
-        const uint32_t hi = bmax2(bmax2(bmax2(w[0].x, w[0].y), bmax2(w[0].z, w[0].w)),
-                                  bmax2(bmax2(w[1].x, w[1].y), bmax2(w[1].z, w[1].w)));
+#pragma unroll
+        for (int h = 0; h < H; ++h) w[h] = xs[ln.chunk(h ^ flip)];
+        uint32_t lo = bmin2(bmin2(w[0].x, w[0].y), bmin2(w[0].z, w[0].w));
+        uint32_t hi = bmax2(bmax2(w[0].x, w[0].y), bmax2(w[0].z, w[0].w));
+#pragma unroll
+        for (int h = 1; h < H; ++h) {
+            lo = bmin2(lo, bmin2(bmin2(w[h].x, w[h].y), bmin2(w[h].z, w[h].w)));
+            hi = bmax2(hi, bmax2(bmax2(w[h].x, w[h].y), bmax2(w[h].z, w[h].w)));
+        }
         // (lo.even, -hi.even) and (lo.odd, -hi.odd) -> (lane min, -lane max)
         mm = bmin2(__byte_perm(lo, hi, 0x5410) ^ 0x80000000u, __byte_perm(lo, hi, 0x7632) ^ 0x80000000u);
     }
@@ -579,15 +592,16 @@ __device__ __forceinline__ void quantize_tile_group_nf(const Args& a, const uint
     const long long j = t.j0 + gi;
     uint8_t* codes = a.a2a_codes + ((size_t)t.rank * a.G + j) * CB;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
+    for (int h = 0; h < H; ++h) {
         float2 e[4];
         e[0] = encode2(bf16_pair(w[h].x), g, a);
         e[1] = encode2(bf16_pair(w[h].y), g, a);
         e[2] = encode2(bf16_pair(w[h].z), g, a);
         e[3] = encode2(bf16_pair(w[h].w), g, a);
         const uint2 pk = pack_codes8<BITS>(e);
-        if (BITS == 4) *reinterpret_cast<uint32_t*>(codes + 4 * ln.chunk(h)) = pk.x;
-        else *reinterpret_cast<uint2*>(codes + 8 * ln.chunk(h)) = pk;
+        const int c = ln.chunk(h ^ flip);
+        if (BITS == 4) *reinterpret_cast<uint32_t*>(codes + 4 * c) = pk.x;
+        else *reinterpret_cast<uint2*>(codes + 8 * c) = pk;
     }
     if (ln.t == 0) a.a2a_params[(size_t)t.rank * a.G + j] = g.param;
 }
@@ -605,11 +619,13 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
         if ((threadIdx.x & 31) == 0) produce<GROUP, M>(a, p, walker, FB);
         return;
     }
-    // with feedback: 8 elements per lane, one pass per tile; without: 16 per
-    // lane, two passes over the 4-sub-tile stage
-    constexpr int GPW = FB ? Lane<GROUP>::GPW : Lane16<GROUP>::GPW;
-    constexpr int PASSES = FB ? 1 : M * kTileElems / (kConsumerWarps * 32 * 16);
-    const int gi = warp * GPW + (FB ? Lane<GROUP>().sub : Lane16<GROUP>().sub);
+    // with feedback: 8 elements per lane, one pass per tile; without: 32 per
+    // lane, one pass over the 4-sub-tile stage
+    using LNF = LaneE<GROUP, kQuantizeLaneElemsNF>;
+    constexpr int GPW = FB ? Lane<GROUP>::GPW : LNF::GPW;
+    constexpr int PASSES = FB ? 1 : M * kTileElems / (kConsumerWarps * 32 * kQuantizeLaneElemsNF);
+    static_assert(FB || PASSES * kConsumerWarps * 32 * kQuantizeLaneElemsNF == M * kTileElems, "tile split");
+    const int gi = warp * GPW + (FB ? Lane<GROUP>().sub : LNF().sub);
     long long i = 0;
     Tile t;
     for (long long k = blockIdx.x; walker.locate(k, &t); k += gridDim.x, ++i) {
@@ -620,7 +636,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
         }
         const uint8_t* stage = p.stages + (size_t)s * kStageBytes;
         if (FB) {
-            quantize_tile_group<GROUP, BITS, true>(a, stage, t, gi, gi < t.count);
+            quantize_tile_group<GROUP, BITS>(a, stage, t, gi, gi < t.count);
         } else {
 #pragma unroll 1
             for (int m = 0; m < PASSES; ++m) {
@@ -643,7 +659,9 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
 
 // ------------------------------------------------------------ reduce
 
-template <int GROUP, int BITS, bool FB>
+// One owned group of a tile with feedback (x, e_long, e_short staged): 8
+// elements per lane, chunks t and t + L of 4.
+template <int GROUP, int BITS>
 __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* st, const Tile& t, int gi,
                                                   bool act) {
     using LN = Lane<GROUP>;
@@ -661,13 +679,11 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
     for (int p = 0; p < 4; ++p) xo[p] = acc[p] = make_float2(0.0f, 0.0f);
     if (act) {
         load_x8_smem(xs, c0, c1, xo);
-        if (FB) {
-            float2 el[4], es[4];
-            load_f8_smem(els, c0, c1, el);
-            load_f8_smem(ess, c0, c1, es);
+        float2 el[4], es[4];
+        load_f8_smem(els, c0, c1, el);
+        load_f8_smem(ess, c0, c1, es);
 #pragma unroll
-            for (int p = 0; p < 4; ++p) xo[p] = inject2(xo[p], el[p], es[p], a);
-        }
+        for (int p = 0; p < 4; ++p) xo[p] = inject2(xo[p], el[p], es[p], a);
     }
     // binary32 sum in rank order 0..P-1: own x' unquantized, others decoded
     for (int r0 = 0; r0 < a.P; r0 += RB) {
@@ -756,25 +772,23 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
         *reinterpret_cast<uint2*>(a.out[0] + j * GROUP + c0) = make_uint2(yb[0], yb[1]);
         *reinterpret_cast<uint2*>(a.out[0] + j * GROUP + c1) = make_uint2(yb[2], yb[3]);
     }
-    if (FB) {
-        float2 el[4], es[4];
-        load_f8_smem(els, c0, c1, el);
-        load_f8_smem(ess, c0, c1, es);
-        float* el_g = a.state + (size_t)o * 2 * a.S + j * GROUP;
-        float2 rho[4];
+    float2 el[4], es[4];
+    load_f8_smem(els, c0, c1, el);
+    load_f8_smem(ess, c0, c1, es);
+    float* el_g = a.state + (size_t)o * 2 * a.S + j * GROUP;
+    float2 rho[4];
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            // -float(y): flip the sign bits of the bf16 pair, then widen exactly
-            const uint32_t ny = yb[p] ^ 0x80008000u;
-            rho[p] = add2_rn(acc[p], make_float2(__uint_as_float(ny << 16), __uint_as_float(ny & 0xffff0000u)));
-        }
-        store_f4_pair(el_g + c0, ema2(el[0], rho[0], a.keep_long, a.a_long, a), ema2(el[1], rho[1], a.keep_long, a.a_long, a));
-        store_f4_pair(el_g + c1, ema2(el[2], rho[2], a.keep_long, a.a_long, a), ema2(el[3], rho[3], a.keep_long, a.a_long, a));
-        store_f4_pair(el_g + a.S + c0, ema2(es[0], rho[0], a.keep_short, a.a_short, a),
-                      ema2(es[1], rho[1], a.keep_short, a.a_short, a));
-        store_f4_pair(el_g + a.S + c1, ema2(es[2], rho[2], a.keep_short, a.a_short, a),
-                      ema2(es[3], rho[3], a.keep_short, a.a_short, a));
+    for (int p = 0; p < 4; ++p) {
+        // -float(y): flip the sign bits of the bf16 pair, then widen exactly
+        const uint32_t ny = yb[p] ^ 0x80008000u;
+        rho[p] = add2_rn(acc[p], make_float2(__uint_as_float(ny << 16), __uint_as_float(ny & 0xffff0000u)));
     }
+    store_f4_pair(el_g + c0, ema2(el[0], rho[0], a.keep_long, a.a_long, a), ema2(el[1], rho[1], a.keep_long, a.a_long, a));
+    store_f4_pair(el_g + c1, ema2(el[2], rho[2], a.keep_long, a.a_long, a), ema2(el[3], rho[3], a.keep_long, a.a_long, a));
+    store_f4_pair(el_g + a.S + c0, ema2(es[0], rho[0], a.keep_short, a.a_short, a),
+                  ema2(es[1], rho[1], a.keep_short, a.a_short, a));
+    store_f4_pair(el_g + a.S + c1, ema2(es[2], rho[2], a.keep_short, a.a_short, a),
+                  ema2(es[3], rho[3], a.keep_short, a.a_short, a));
 }
 
 // eight packed codes (one word at 4 bits, two at 8) -> four exact float pairs
@@ -964,7 +978,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
         }
         const uint8_t* stage = p.stages + (size_t)s * kStageBytes;
         if (FB) {
-            reduce_tile_group<GROUP, BITS, true>(a, stage, t, gi, gi < t.count);
+            reduce_tile_group<GROUP, BITS>(a, stage, t, gi, gi < t.count);
         } else {
 #pragma unroll 1
             for (int m = 0; m < PASSES; ++m) {
