@@ -234,8 +234,6 @@ __device__ __forceinline__ void produce(const Args& a, const PipeShared& p, RunW
     }
 }
 
-// ------------------------------------------------------------ quantize
-
 // ------------------------------------------------------------ packed math
 //
 // The tile paths compute two elements per instruction with the sm_100 paired
@@ -320,6 +318,18 @@ __device__ __forceinline__ float nan_max(float a, float b) {
     return r;
 }
 
+__device__ __forceinline__ float nan_min3(float a, float b, float c) {
+    float r;
+    asm("min.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+__device__ __forceinline__ float nan_max3(float a, float b, float c) {
+    float r;
+    asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // Packed quantization grid of one group (same values as make_grid).
 struct GridP {
     float2 s, z, ns, nz, inv;
@@ -370,36 +380,56 @@ __device__ __forceinline__ float2 encode2(float2 v, const GridP& g, const Args& 
     return add_after_mul2(u, splat(kMagic), a);
 }
 
-// four codes (2^23 + code each) -> one chunk of packed codes
+
+
+// eight codes (2^23 + code each, in four pairs) -> packed bytes: one word at
+// 4 bits, two at 8 bits. Only the low byte of each float's bit pattern is
+// used; at 4 bits (hi << 4) + lo puts code 2i + 1 above code 2i without a
+// carry out of the byte (both codes <= 15).
 template <int BITS>
-__device__ __forceinline__ uint32_t pack_codes4(float2 t01, float2 t23) {
-    constexpr uint32_t Q = (1u << BITS) - 1u;
-    const uint32_t c0 = __float_as_uint(t01.x) & Q, c1 = __float_as_uint(t01.y) & Q;
-    const uint32_t c2 = __float_as_uint(t23.x) & Q, c3 = __float_as_uint(t23.y) & Q;
-    if (BITS == 4) return c0 | (c1 << 4) | (c2 << 8) | (c3 << 12);
-    return c0 | (c1 << 8) | (c2 << 16) | (c3 << 24);
+__device__ __forceinline__ uint2 pack_codes8(const float2 t[4]) {
+    uint2 out;
+    if (BITS == 4) {
+        uint32_t b[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) b[k] = (__float_as_uint(t[k].y) << 4) + __float_as_uint(t[k].x);
+        out.x = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+        out.y = 0;
+    } else {
+        const uint32_t p0 = __byte_perm(__float_as_uint(t[0].x), __float_as_uint(t[0].y), 0x0040);
+        const uint32_t p1 = __byte_perm(__float_as_uint(t[1].x), __float_as_uint(t[1].y), 0x0040);
+        const uint32_t p2 = __byte_perm(__float_as_uint(t[2].x), __float_as_uint(t[2].y), 0x0040);
+        const uint32_t p3 = __byte_perm(__float_as_uint(t[3].x), __float_as_uint(t[3].y), 0x0040);
+        out.x = __byte_perm(p0, p1, 0x5410);
+        out.y = __byte_perm(p2, p3, 0x5410);
+    }
+    return out;
 }
 
-// one chunk of packed codes -> the four codes as exact floats
+// eight packed codes (one word at 4 bits, two at 8) -> four exact float pairs
 template <int BITS>
-__device__ __forceinline__ void unpack_codes4(uint32_t w, float2& q01, float2& q23) {
-    uint32_t m0, m1, m2, m3;
+__device__ __forceinline__ void unpack_codes8(const uint32_t* w, float2 q[4]) {
+    uint32_t ev[4], od[4];   // 2^23 + code of elements 2p and 2p + 1
     if (BITS == 4) {
-        const uint32_t lo = w & 0x0F0Fu;          // codes 0 and 2 in bytes 0 and 1
-        const uint32_t hi = (w >> 4) & 0x0F0Fu;   // codes 1 and 3
-        m0 = __byte_perm(lo, 0x4B000000u, 0x7650);
-        m1 = __byte_perm(hi, 0x4B000000u, 0x7650);
-        m2 = __byte_perm(lo, 0x4B000000u, 0x7651);
-        m3 = __byte_perm(hi, 0x4B000000u, 0x7651);
+        const uint32_t lo = w[0] & 0x0F0F0F0Fu;          // codes 0, 2, 4, 6 in bytes 0..3
+        const uint32_t hi = (w[0] >> 4) & 0x0F0F0F0Fu;   // codes 1, 3, 5, 7
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            ev[p] = __byte_perm(lo, 0x4B000000u, 0x7650 + p);
+            od[p] = __byte_perm(hi, 0x4B000000u, 0x7650 + p);
+        }
     } else {
-        m0 = __byte_perm(w, 0x4B000000u, 0x7650);
-        m1 = __byte_perm(w, 0x4B000000u, 0x7651);
-        m2 = __byte_perm(w, 0x4B000000u, 0x7652);
-        m3 = __byte_perm(w, 0x4B000000u, 0x7653);
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            ev[p] = __byte_perm(w[p >> 1], 0x4B000000u, 0x7650 + 2 * (p & 1));
+            od[p] = __byte_perm(w[p >> 1], 0x4B000000u, 0x7651 + 2 * (p & 1));
+        }
     }
-    q01 = add2_rn(make_float2(__uint_as_float(m0), __uint_as_float(m1)), splat(-kMagic));
-    q23 = add2_rn(make_float2(__uint_as_float(m2), __uint_as_float(m3)), splat(-kMagic));
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+        q[p] = add2_rn(make_float2(__uint_as_float(ev[p]), __uint_as_float(od[p])), splat(-kMagic));
 }
+
 
 // x' = x + eta * (w * e_short + (1 - w) * e_long), two elements
 __device__ __forceinline__ float2 inject2(float2 x, float2 el, float2 es, const Args& a) {
@@ -412,14 +442,6 @@ __device__ __forceinline__ float2 ema2(float2 e, float2 rho, float keep, float a
     return add_after_mul2(mul2_rn(splat(keep), e), mul2_rn(splat(alpha), rho), a);
 }
 
-__device__ __forceinline__ void load_x8_smem(const uint16_t* xs, int c0, int c1, float2 v[4]) {
-    const uint2 u0 = *reinterpret_cast<const uint2*>(xs + c0);
-    const uint2 u1 = *reinterpret_cast<const uint2*>(xs + c1);
-    v[0] = make_float2(bf16_lo(u0.x), bf16_hi(u0.x));
-    v[1] = make_float2(bf16_lo(u0.y), bf16_hi(u0.y));
-    v[2] = make_float2(bf16_lo(u1.x), bf16_hi(u1.x));
-    v[3] = make_float2(bf16_lo(u1.y), bf16_hi(u1.y));
-}
 
 __device__ __forceinline__ void load_f8_smem(const float* p, int c0, int c1, float2 v[4]) {
     const float4 a = *reinterpret_cast<const float4*>(p + c0);
@@ -434,10 +456,28 @@ __device__ __forceinline__ void store_f4_pair(float* p, float2 lo, float2 hi) {
     __stcs(reinterpret_cast<float4*>(p), make_float4(lo.x, lo.y, hi.x, hi.y));
 }
 
+// 8 consecutive bf16 values (16 bytes) from shared memory
+__device__ __forceinline__ void load_x8c_smem(const uint16_t* xs, float2 v[4]) {
+    const uint4 u = *reinterpret_cast<const uint4*>(xs);
+    v[0] = make_float2(bf16_lo(u.x), bf16_hi(u.x));
+    v[1] = make_float2(bf16_lo(u.y), bf16_hi(u.y));
+    v[2] = make_float2(bf16_lo(u.z), bf16_hi(u.z));
+    v[3] = make_float2(bf16_lo(u.w), bf16_hi(u.w));
+}
+
+// 8 consecutive fp32 values to global memory in one 32-byte streaming store
+// (sm_100 vector width; p must be 32-byte aligned).
+__device__ __forceinline__ void store_f8_cs(float* p, const float2 v[4]) {
+    asm volatile("st.global.cs.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "f"(v[0].x),
+                 "f"(v[0].y), "f"(v[1].x), "f"(v[1].y), "f"(v[2].x), "f"(v[2].y), "f"(v[3].x), "f"(v[3].y)
+                 : "memory");
+}
+
 // ------------------------------------------------------------ quantize
 
 // One non-owned group of a tile with feedback (x, e_long, e_short staged):
-// 8 elements per lane, chunks t and t + L of 4.
+// 8 consecutive elements per lane (lane t of the group's L takes elements
+// [8t, 8t + 8)).
 template <int GROUP, int BITS>
 __device__ __forceinline__ void quantize_tile_group(const Args& a, const uint8_t* st, const Tile& t, int gi,
                                                     bool act) {
@@ -446,45 +486,48 @@ __device__ __forceinline__ void quantize_tile_group(const Args& a, const uint8_t
     const LN ln;
     const int r = t.rank;
     const long long j = t.j0 + gi;
-    const int c0 = 4 * ln.chunk(0), c1 = 4 * ln.chunk(1);
+    const int e0 = 8 * ln.t;
     const uint16_t* xs = reinterpret_cast<const uint16_t*>(st) + gi * GROUP;
     const float* els = reinterpret_cast<const float*>(st + kTileElems * 2) + gi * GROUP;
     const float* ess = reinterpret_cast<const float*>(st + kTileElems * 6) + gi * GROUP;
     float2 v[4], el[4], es[4];
     float lmin = __int_as_float(0x7f800000), lmax = -__int_as_float(0x7f800000);
     if (act) {
-        load_x8_smem(xs, c0, c1, v);
-        load_f8_smem(els, c0, c1, el);
-        load_f8_smem(ess, c0, c1, es);
-#pragma unroll
-        for (int p = 0; p < 4; ++p) v[p] = inject2(v[p], el[p], es[p], a);
+        load_x8c_smem(xs + e0, v);
+        load_f8_smem(els, e0, e0 + 4, el);
+        load_f8_smem(ess, e0, e0 + 4, es);
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
-            lmin = nan_min(lmin, nan_min(v[p].x, v[p].y));
-            lmax = nan_max(lmax, nan_max(v[p].x, v[p].y));
+            v[p] = inject2(v[p], el[p], es[p], a);
+            lmin = nan_min3(lmin, v[p].x, v[p].y);
+            lmax = nan_max3(lmax, v[p].x, v[p].y);
         }
     }
     const GridP g = make_grid_p<L, Q>(lmin, lmax);
     raise_flags(a, act && g.bad);
     if (!act) return;
-    uint8_t* codes = a.a2a_codes + ((size_t)r * a.G + j) * CB;
-    float* el_g = a.state + (size_t)r * 2 * a.S + j * GROUP;
+    float2 e[4];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const float2 t01 = encode2(v[2 * h], g, a);
-        const float2 t23 = encode2(v[2 * h + 1], g, a);
-        store_chunk_codes<BITS>(codes, ln.chunk(h), pack_codes4<BITS>(t01, t23));
-        // residual x' - x_hat with x_hat = code*s + z (fused: code*s is exact)
-        const float2 q01 = add2_rn(t01, splat(-kMagic));
-        const float2 q23 = add2_rn(t23, splat(-kMagic));
-        const float2 rho01 = add2_rn(v[2 * h], fma2_rn(q01, g.ns, g.nz));
-        const float2 rho23 = add2_rn(v[2 * h + 1], fma2_rn(q23, g.ns, g.nz));
-        const int c = h ? c1 : c0;
-        store_f4_pair(el_g + c, ema2(el[2 * h], rho01, a.keep_long, a.a_long, a),
-                      ema2(el[2 * h + 1], rho23, a.keep_long, a.a_long, a));
-        store_f4_pair(el_g + a.S + c, ema2(es[2 * h], rho01, a.keep_short, a.a_short, a),
-                      ema2(es[2 * h + 1], rho23, a.keep_short, a.a_short, a));
+    for (int p = 0; p < 4; ++p) e[p] = encode2(v[p], g, a);
+    uint8_t* codes = a.a2a_codes + ((size_t)r * a.G + j) * CB;
+    const uint2 pk = pack_codes8<BITS>(e);
+    if (BITS == 4) *reinterpret_cast<uint32_t*>(codes + 4 * ln.t) = pk.x;
+    else *reinterpret_cast<uint2*>(codes + 8 * ln.t) = pk;
+    // residual x' - x_hat with x_hat = code*s + z (fused: code*s is exact)
+    float2 nl[4], ns[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const float2 rho = add2_rn(v[p], fma2_rn(add2_rn(e[p], splat(-kMagic)), g.ns, g.nz));
+        nl[p] = ema2(el[p], rho, a.keep_long, a.a_long, a);
+        ns[p] = ema2(es[p], rho, a.keep_short, a.a_short, a);
     }
+    float* el_g = a.state + (size_t)r * 2 * a.S + j * GROUP + e0;
+    // 16-byte stores here: measured on B200, 32-byte ones made this pass ~2 %
+    // slower (the owner's pass gains from them)
+    store_f4_pair(el_g, nl[0], nl[1]);
+    store_f4_pair(el_g + 4, nl[2], nl[3]);
+    store_f4_pair(el_g + a.S, ns[0], ns[1]);
+    store_f4_pair(el_g + a.S + 4, ns[2], ns[3]);
     if (ln.t == 0) a.a2a_params[(size_t)r * a.G + j] = g.param;
 }
 
@@ -531,30 +574,6 @@ __device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
 }
 
 __device__ __forceinline__ float2 bf16_pair(uint32_t u) { return make_float2(bf16_lo(u), bf16_hi(u)); }
-
-// eight codes (2^23 + code each, in four pairs) -> packed bytes: one word at
-// 4 bits, two at 8 bits. Only the low byte of each float's bit pattern is
-// used; at 4 bits (hi << 4) + lo puts code 2i + 1 above code 2i without a
-// carry out of the byte (both codes <= 15).
-template <int BITS>
-__device__ __forceinline__ uint2 pack_codes8(const float2 t[4]) {
-    uint2 out;
-    if (BITS == 4) {
-        uint32_t b[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) b[k] = (__float_as_uint(t[k].y) << 4) + __float_as_uint(t[k].x);
-        out.x = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
-        out.y = 0;
-    } else {
-        const uint32_t p0 = __byte_perm(__float_as_uint(t[0].x), __float_as_uint(t[0].y), 0x0040);
-        const uint32_t p1 = __byte_perm(__float_as_uint(t[1].x), __float_as_uint(t[1].y), 0x0040);
-        const uint32_t p2 = __byte_perm(__float_as_uint(t[2].x), __float_as_uint(t[2].y), 0x0040);
-        const uint32_t p3 = __byte_perm(__float_as_uint(t[3].x), __float_as_uint(t[3].y), 0x0040);
-        out.x = __byte_perm(p0, p1, 0x5410);
-        out.y = __byte_perm(p2, p3, 0x5410);
-    }
-    return out;
-}
 
 template <int GROUP, int BITS>
 __device__ __forceinline__ void quantize_tile_group_nf(const Args& a, const uint8_t* st, const Tile& t, int gi,
@@ -660,17 +679,18 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
 // ------------------------------------------------------------ reduce
 
 // One owned group of a tile with feedback (x, e_long, e_short staged): 8
-// elements per lane, chunks t and t + L of 4.
+// consecutive elements per lane, like the quantize pass.
 template <int GROUP, int BITS>
 __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* st, const Tile& t, int gi,
                                                   bool act) {
     using LN = Lane<GROUP>;
     constexpr int L = LN::L, Q = (1 << BITS) - 1, CB = GROUP * BITS / 8;
-    constexpr int RB = 8;   // ranks whose payload loads are issued together
+    constexpr int RB = 8;          // ranks whose payload loads are issued together
+    constexpr int CW = BITS / 4;   // 32-bit code words per lane (8 codes)
     const LN ln;
     const int o = t.rank;
     const long long j = t.j0 + gi;
-    const int c0 = 4 * ln.chunk(0), c1 = 4 * ln.chunk(1);
+    const int e0 = 8 * ln.t;
     const uint16_t* xs = reinterpret_cast<const uint16_t*>(st) + gi * GROUP;
     const float* els = reinterpret_cast<const float*>(st + kTileElems * 2) + gi * GROUP;
     const float* ess = reinterpret_cast<const float*>(st + kTileElems * 6) + gi * GROUP;
@@ -678,27 +698,33 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
 #pragma unroll
     for (int p = 0; p < 4; ++p) xo[p] = acc[p] = make_float2(0.0f, 0.0f);
     if (act) {
-        load_x8_smem(xs, c0, c1, xo);
+        load_x8c_smem(xs + e0, xo);
         float2 el[4], es[4];
-        load_f8_smem(els, c0, c1, el);
-        load_f8_smem(ess, c0, c1, es);
+        load_f8_smem(els, e0, e0 + 4, el);
+        load_f8_smem(ess, e0, e0 + 4, es);
 #pragma unroll
         for (int p = 0; p < 4; ++p) xo[p] = inject2(xo[p], el[p], es[p], a);
     }
     // binary32 sum in rank order 0..P-1: own x' unquantized, others decoded
     for (int r0 = 0; r0 < a.P; r0 += RB) {
-        uint32_t cw[RB][2];
+        uint32_t cw[RB][CW];
         uint32_t pw[RB];
 #pragma unroll
         for (int k = 0; k < RB; ++k) {
             const int r = r0 + k;
-            cw[k][0] = cw[k][1] = 0u;
+#pragma unroll
+            for (int c = 0; c < CW; ++c) cw[k][c] = 0u;
             pw[k] = 0u;
             if (act && r < a.P && r != o) {
                 const size_t slot = (size_t)r * a.G + j;
                 const uint8_t* codes = a.a2a_codes + slot * CB;
-                cw[k][0] = load_chunk_codes<BITS>(codes, ln.chunk(0));
-                cw[k][1] = load_chunk_codes<BITS>(codes, ln.chunk(1));
+                if (BITS == 4) {
+                    cw[k][0] = *reinterpret_cast<const uint32_t*>(codes + 4 * ln.t);
+                } else {
+                    const uint2 v = *reinterpret_cast<const uint2*>(codes + 8 * ln.t);
+                    cw[k][0] = v.x;
+                    cw[k][CW - 1] = v.y;
+                }
                 pw[k] = a.a2a_params[slot];
             }
         }
@@ -713,29 +739,21 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
             } else {
                 const float2 s2 = splat(param_s(pw[k]));
                 const float2 z2 = splat(param_z(pw[k]));
+                float2 q[4];
+                unpack_codes8<BITS>(cw[k], q);
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    float2 q01, q23;
-                    unpack_codes4<BITS>(cw[k][h], q01, q23);
-                    term[2 * h] = fma2_rn(q01, s2, z2);
-                    term[2 * h + 1] = fma2_rn(q23, s2, z2);
-                }
+                for (int p = 0; p < 4; ++p) term[p] = fma2_rn(q[p], s2, z2);
             }
-            if (r == 0) {
 #pragma unroll
-                for (int p = 0; p < 4; ++p) acc[p] = term[p];
-            } else {
-#pragma unroll
-                for (int p = 0; p < 4; ++p) acc[p] = add2_rn(acc[p], term[p]);
-            }
+            for (int p = 0; p < 4; ++p) acc[p] = (r == 0) ? term[p] : add2_rn(acc[p], term[p]);
         }
     }
     float lmin = __int_as_float(0x7f800000), lmax = -__int_as_float(0x7f800000);
     if (act) {
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
-            lmin = nan_min(lmin, nan_min(acc[p].x, acc[p].y));
-            lmax = nan_max(lmax, nan_max(acc[p].x, acc[p].y));
+            lmin = nan_min3(lmin, acc[p].x, acc[p].y);
+            lmax = nan_max3(lmax, acc[p].x, acc[p].y);
         }
     }
     uint32_t yb[4];   // bf16 pairs of the result
@@ -743,25 +761,22 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
         const GridP g = make_grid_p<L, Q>(lmin, lmax);
         raise_flags(a, act && g.bad);
         if (!act) return;
-        uint8_t* codes = a.g_codes + (size_t)j * CB;
+        float2 e[4];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const float2 t01 = encode2(acc[2 * h], g, a);
-            const float2 t23 = encode2(acc[2 * h + 1], g, a);
-            store_chunk_codes<BITS>(codes, ln.chunk(h), pack_codes4<BITS>(t01, t23));
-            const float2 y01 = fma2_rn(add2_rn(t01, splat(-kMagic)), g.s, g.z);
-            const float2 y23 = fma2_rn(add2_rn(t23, splat(-kMagic)), g.s, g.z);
-            yb[2 * h] = bf16x2_rn(y01);
-            yb[2 * h + 1] = bf16x2_rn(y23);
+        for (int p = 0; p < 4; ++p) {
+            e[p] = encode2(acc[p], g, a);
+            yb[p] = bf16x2_rn(fma2_rn(add2_rn(e[p], splat(-kMagic)), g.s, g.z));
         }
+        uint8_t* codes = a.g_codes + (size_t)j * CB;
+        const uint2 pk = pack_codes8<BITS>(e);
+        if (BITS == 4) *reinterpret_cast<uint32_t*>(codes + 4 * ln.t) = pk.x;
+        else *reinterpret_cast<uint2*>(codes + 8 * ln.t) = pk;
         if (ln.t == 0) a.g_params[j] = g.param;
         if (a.write_outputs) {
             // phase 4 in the owner's pass: every rank's output gets the decoded
             // requantized sum -- the same bits a decode of the gathered payload gives
-            for (int r = 0; r < a.P; ++r) {
-                __stcs(reinterpret_cast<uint2*>(a.out[r] + j * GROUP + c0), make_uint2(yb[0], yb[1]));
-                __stcs(reinterpret_cast<uint2*>(a.out[r] + j * GROUP + c1), make_uint2(yb[2], yb[3]));
-            }
+            const uint4 y4 = make_uint4(yb[0], yb[1], yb[2], yb[3]);
+            for (int r = 0; r < a.P; ++r) __stcs(reinterpret_cast<uint4*>(a.out[r] + j * GROUP + e0), y4);
         }
     } else {
         // a single rank sends nothing: its output is its own x'
@@ -769,62 +784,22 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
         if (!act) return;
 #pragma unroll
         for (int p = 0; p < 4; ++p) yb[p] = bf16x2_rn(acc[p]);
-        *reinterpret_cast<uint2*>(a.out[0] + j * GROUP + c0) = make_uint2(yb[0], yb[1]);
-        *reinterpret_cast<uint2*>(a.out[0] + j * GROUP + c1) = make_uint2(yb[2], yb[3]);
+        *reinterpret_cast<uint4*>(a.out[0] + j * GROUP + e0) = make_uint4(yb[0], yb[1], yb[2], yb[3]);
     }
-    float2 el[4], es[4];
-    load_f8_smem(els, c0, c1, el);
-    load_f8_smem(ess, c0, c1, es);
-    float* el_g = a.state + (size_t)o * 2 * a.S + j * GROUP;
-    float2 rho[4];
+    float2 el[4], es[4], nl[4], ns[4];
+    load_f8_smem(els, e0, e0 + 4, el);
+    load_f8_smem(ess, e0, e0 + 4, es);
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
-        // -float(y): flip the sign bits of the bf16 pair, then widen exactly
+        // rho = acc - float(y): flip the sign bits of the bf16 pair, then widen exactly
         const uint32_t ny = yb[p] ^ 0x80008000u;
-        rho[p] = add2_rn(acc[p], make_float2(__uint_as_float(ny << 16), __uint_as_float(ny & 0xffff0000u)));
+        const float2 rho = add2_rn(acc[p], make_float2(__uint_as_float(ny << 16), __uint_as_float(ny & 0xffff0000u)));
+        nl[p] = ema2(el[p], rho, a.keep_long, a.a_long, a);
+        ns[p] = ema2(es[p], rho, a.keep_short, a.a_short, a);
     }
-    store_f4_pair(el_g + c0, ema2(el[0], rho[0], a.keep_long, a.a_long, a), ema2(el[1], rho[1], a.keep_long, a.a_long, a));
-    store_f4_pair(el_g + c1, ema2(el[2], rho[2], a.keep_long, a.a_long, a), ema2(el[3], rho[3], a.keep_long, a.a_long, a));
-    store_f4_pair(el_g + a.S + c0, ema2(es[0], rho[0], a.keep_short, a.a_short, a),
-                  ema2(es[1], rho[1], a.keep_short, a.a_short, a));
-    store_f4_pair(el_g + a.S + c1, ema2(es[2], rho[2], a.keep_short, a.a_short, a),
-                  ema2(es[3], rho[3], a.keep_short, a.a_short, a));
-}
-
-// eight packed codes (one word at 4 bits, two at 8) -> four exact float pairs
-template <int BITS>
-__device__ __forceinline__ void unpack_codes8(const uint32_t* w, float2 q[4]) {
-    uint32_t ev[4], od[4];   // 2^23 + code of elements 2p and 2p + 1
-    if (BITS == 4) {
-        const uint32_t lo = w[0] & 0x0F0F0F0Fu;          // codes 0, 2, 4, 6 in bytes 0..3
-        const uint32_t hi = (w[0] >> 4) & 0x0F0F0F0Fu;   // codes 1, 3, 5, 7
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            ev[p] = __byte_perm(lo, 0x4B000000u, 0x7650 + p);
-            od[p] = __byte_perm(hi, 0x4B000000u, 0x7650 + p);
-        }
-    } else {
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            ev[p] = __byte_perm(w[p >> 1], 0x4B000000u, 0x7650 + 2 * (p & 1));
-            od[p] = __byte_perm(w[p >> 1], 0x4B000000u, 0x7651 + 2 * (p & 1));
-        }
-    }
-#pragma unroll
-    for (int p = 0; p < 4; ++p)
-        q[p] = add2_rn(make_float2(__uint_as_float(ev[p]), __uint_as_float(od[p])), splat(-kMagic));
-}
-
-__device__ __forceinline__ float nan_min3(float a, float b, float c) {
-    float r;
-    asm("min.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-    return r;
-}
-
-__device__ __forceinline__ float nan_max3(float a, float b, float c) {
-    float r;
-    asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-    return r;
+    float* el_g = a.state + (size_t)o * 2 * a.S + j * GROUP + e0;
+    store_f8_cs(el_g, nl);
+    store_f8_cs(el_g + a.S, ns);
 }
 
 // The owner's pass without feedback, 16 elements per lane (chunks t and
@@ -1035,13 +1010,8 @@ __device__ __forceinline__ uint4 decode8_bf16(uint2 w, uint32_t param) {
     const float2 s2 = splat(param_s(param));
     const float2 z2 = splat(param_z(param));
     float2 q[4];
-    if (BITS == 4) {
-        unpack_codes4<4>(w.x & 0xffffu, q[0], q[1]);
-        unpack_codes4<4>(w.x >> 16, q[2], q[3]);
-    } else {
-        unpack_codes4<8>(w.x, q[0], q[1]);
-        unpack_codes4<8>(w.y, q[2], q[3]);
-    }
+    const uint32_t cw[2] = {w.x, w.y};
+    unpack_codes8<BITS>(cw, q);
     return make_uint4(bf16x2_rn(fma2_rn(q[0], s2, z2)), bf16x2_rn(fma2_rn(q[1], s2, z2)),
                       bf16x2_rn(fma2_rn(q[2], s2, z2)), bf16x2_rn(fma2_rn(q[3], s2, z2)));
 }
