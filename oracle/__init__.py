@@ -20,6 +20,7 @@ from . import build as _build
 
 RN, RD, RU = 0, 1, 2
 FLAG_RANGE = 1
+Q_DIRECTED, Q_NEAREST, Q_INT_ZERO = 0, 1, 2   # quantizer forms (readings R4, R10, R11)
 
 _lib = None
 
@@ -62,6 +63,16 @@ def lib() -> ctypes.CDLL:
             P, P, P, P, P, P, P, P,
         ]
         L.oracle_echo_allreduce.restype = ctypes.c_int
+        L.oracle_quantize_group_q.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P, P]
+        L.oracle_quantize_group_q.restype = ctypes.c_uint32
+        L.oracle_echo_allreduce_q.argtypes = [
+            ctypes.c_int, ctypes.c_longlong, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_longlong, ctypes.c_longlong,
+            P, P, P, P,
+            ctypes.c_float, ctypes.c_float, ctypes.c_float, ctypes.c_float,
+            P, P, P, P, P, P, P, P,
+        ]
+        L.oracle_echo_allreduce_q.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -117,15 +128,22 @@ class GroupQuant:
     flag: int
 
 
-def quantize_group(v: np.ndarray, bits: int) -> GroupQuant:
+def quantize_group(v: np.ndarray, bits: int, quantizer: int = Q_DIRECTED) -> GroupQuant:
+    """One group through the quantizer form ``quantizer`` (Q_DIRECTED: fp16
+    zero rounded down and step rounded up; Q_NEAREST: both rounded to
+    nearest; Q_INT_ZERO: integer zero point, ``z_bits`` then holds zp)."""
     v = np.ascontiguousarray(v, dtype=np.float32)
     m = v.size
     codes = np.zeros(m, np.uint8)
     vhat = np.zeros(m, np.float32)
     s = ctypes.c_uint16()
     z = ctypes.c_uint16()
-    flag = lib().oracle_quantize_group(_ptr(v), m, bits, _ptr(codes), ctypes.byref(s),
-                                       ctypes.byref(z), _ptr(vhat))
+    if quantizer == Q_DIRECTED:
+        flag = lib().oracle_quantize_group(_ptr(v), m, bits, _ptr(codes), ctypes.byref(s),
+                                           ctypes.byref(z), _ptr(vhat))
+    else:
+        flag = lib().oracle_quantize_group_q(_ptr(v), m, bits, quantizer, _ptr(codes), ctypes.byref(s),
+                                             ctypes.byref(z), _ptr(vhat))
     return GroupQuant(codes, int(s.value), int(z.value), vhat, int(flag))
 
 
@@ -162,12 +180,12 @@ def echo_allreduce(x: np.ndarray, *, n_total: int, group: int, bits: int,
                    e_long: Optional[np.ndarray] = None, e_short: Optional[np.ndarray] = None,
                    eta: float = 1.0, alpha_long: float = 0.05, alpha_short: float = 0.5,
                    w: float = 0.5, j0: int = 0, jc: Optional[int] = None,
-                   debug: bool = False) -> CallResult:
+                   debug: bool = False, quantizer: int = Q_DIRECTED) -> CallResult:
     """Run one oracle call on the columns ``[j0, j0 + jc)``.
 
     ``x`` is ``[P][jc*group]`` uint16 (bf16 bit patterns). ``e_long`` and
     ``e_short`` (``[P][jc*group]`` float32) are updated in place; pass both or
-    neither.
+    neither. ``quantizer`` selects the quantizer form (see quantize_group).
     """
     x = np.ascontiguousarray(x, dtype=np.uint16)
     P, ld = x.shape
@@ -189,10 +207,16 @@ def echo_allreduce(x: np.ndarray, *, n_total: int, group: int, bits: int,
     rho = np.zeros((P, ld), np.float32) if debug else None
     passes = np.zeros((P, ld), np.uint8) if debug else None
     flags = ctypes.c_uint32(0)
-    rc = lib().oracle_echo_allreduce(
-        P, n_total, group, bits, j0, jc, _ptr(x), _ptr(y), _ptr(e_long), _ptr(e_short),
-        eta, alpha_long, alpha_short, w, _ptr(a2a_c), _ptr(a2a_p), _ptr(g_c), _ptr(g_p),
-        _ptr(xp), _ptr(rho), _ptr(passes), ctypes.byref(flags))
+    if quantizer == Q_DIRECTED:
+        rc = lib().oracle_echo_allreduce(
+            P, n_total, group, bits, j0, jc, _ptr(x), _ptr(y), _ptr(e_long), _ptr(e_short),
+            eta, alpha_long, alpha_short, w, _ptr(a2a_c), _ptr(a2a_p), _ptr(g_c), _ptr(g_p),
+            _ptr(xp), _ptr(rho), _ptr(passes), ctypes.byref(flags))
+    else:
+        rc = lib().oracle_echo_allreduce_q(
+            P, n_total, group, bits, quantizer, j0, jc, _ptr(x), _ptr(y), _ptr(e_long), _ptr(e_short),
+            eta, alpha_long, alpha_short, w, _ptr(a2a_c), _ptr(a2a_p), _ptr(g_c), _ptr(g_p),
+            _ptr(xp), _ptr(rho), _ptr(passes), ctypes.byref(flags))
     if rc != 0:
         raise ValueError("oracle_echo_allreduce rejected its arguments")
     return CallResult(y, a2a_c, a2a_p, g_c, g_p, xp, rho, passes, int(flags.value))

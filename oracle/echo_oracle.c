@@ -64,6 +64,19 @@
  *      sum - float(y), y being the bf16 value every rank receives.
  *   R9 values outside [-65504, 65504] (or NaN) in a group that is quantized,
  *      or in a P == 1 output, raise the sticky RANGE flag.
+ *
+ * Quantizer variants for the ablations (the pages name the asymmetric
+ * zero-point form but fix neither the rounding of the half-precision
+ * parameters nor whether the zero is a float or an integer):
+ *   R10 "nearest": z = fp16_nearest(mn); s = fp16_nearest((mx - mn) / Q);
+ *      codes clamp(rint((v - z) * (1/s)), 0, Q) -- the clamp now matters,
+ *      because [z, z + Q*s] need not cover [mn, mx]; dequantization as R4.
+ *   R11 "integer zero point": the range is widened to include zero,
+ *      lo = min(mn, 0), hi = max(mx, 0); s = fp16_up((hi - lo) / Q);
+ *      inv = 1/s; zp = clamp(rint(-lo * inv), 0, Q) (0 when s == 0);
+ *      codes clamp(rint(v * inv) + zp, 0, Q); dequantization (code - zp) * s,
+ *      exact in binary32. The parameter pair carries {s, zp} with zp as an
+ *      unsigned 16-bit integer in place of z.
  */
 #include <math.h>
 #include <stdint.h>
@@ -71,6 +84,9 @@
 #include <string.h>
 
 #define ORACLE_FLAG_RANGE 1u
+
+/* quantizer forms: R4 (default), R10, R11 */
+enum { ORACLE_Q_DIRECTED = 0, ORACLE_Q_NEAREST = 1, ORACLE_Q_INT_ZERO = 2 };
 
 enum { ORACLE_RN = 0, ORACLE_RD = 1, ORACLE_RU = 2 };
 
@@ -232,14 +248,39 @@ static int outside_domain(float v)
     return !(v >= -65504.0f && v <= 65504.0f);
 }
 
+/* clamp(rint(u) + add, 0, Q) with rint half to even (the default rounding mode) */
+static int round_clamp(float u, int add, int Q)
+{
+    float r = rintf(u);
+    int c;
+    if (r != r) {
+        c = -1024;      /* NaN: only in a group already flagged out of range */
+    } else if (r < -1024.0f) {
+        c = -1024;
+    } else if (r > 1024.0f) {
+        c = 1024;
+    } else {
+        c = (int)r;
+    }
+    c = c + add;
+    if (c < 0) {
+        c = 0;
+    }
+    if (c > Q) {
+        c = Q;
+    }
+    return c;
+}
+
 /*
- * Quantize m values of one group to codes in [0, Q]. Writes one code per
- * element (unpacked), the fp16 bit patterns of s and z, and the dequantized
- * values. Returns ORACLE_FLAG_RANGE when a value lies outside the fp16
- * parameter domain, 0 otherwise.
+ * Quantize m values of one group to codes in [0, Q] with quantizer form
+ * `qmode` (R4, R10 or R11). Writes one code per element (unpacked), the two
+ * 16-bit parameter words (fp16 s, and fp16 z or the integer zero point), and
+ * the dequantized values. Returns ORACLE_FLAG_RANGE when a value lies outside
+ * the fp16 parameter domain, 0 otherwise.
  */
-uint32_t oracle_quantize_group(const float* v, int m, int bits, uint8_t* codes,
-                               uint16_t* s_bits, uint16_t* z_bits, float* vhat)
+uint32_t oracle_quantize_group_q(const float* v, int m, int bits, int qmode, uint8_t* codes,
+                                 uint16_t* s_bits, uint16_t* z_bits, float* vhat)
 {
     int Q = (1 << bits) - 1;
     uint32_t flag = 0;
@@ -258,11 +299,50 @@ uint32_t oracle_quantize_group(const float* v, int m, int bits, uint8_t* codes,
     }
     mn = mn + 0.0f;
     mx = mx + 0.0f;
-    uint16_t zh = oracle_f32_to_f16(mn, ORACLE_RD);
+    if (qmode == ORACLE_Q_INT_ZERO) {
+        float lo = mn < 0.0f ? mn : 0.0f;
+        float hi = mx > 0.0f ? mx : 0.0f;
+        float d = hi - lo;
+        float step = d / (float)Q;
+        uint16_t sh = oracle_f32_to_f16(step, ORACLE_RU);
+        float s = oracle_f16_to_f32(sh);
+        int zp = 0;
+        float inv = 0.0f;
+        if (s != 0.0f) {
+            inv = 1.0f / s;
+            float nlo = -lo;
+            float t = nlo * inv;
+            zp = round_clamp(t, 0, Q);
+        }
+        for (int i = 0; i < m; i++) {
+            int c = 0;
+            if (s != 0.0f) {
+                float u = v[i] * inv;
+                c = round_clamp(u, zp, Q);
+            }
+            codes[i] = (uint8_t)c;
+            int k = c - zp;
+            vhat[i] = (float)k * s;       /* exact: |k| <= 255, s has 11 bits */
+        }
+        *s_bits = sh;
+        *z_bits = (uint16_t)zp;
+        return flag;
+    }
+    uint16_t zh;
+    uint16_t sh;
+    if (qmode == ORACLE_Q_NEAREST) {
+        zh = oracle_f32_to_f16(mn, ORACLE_RN);
+        float d = mx - mn;
+        float step = d / (float)Q;
+        sh = oracle_f32_to_f16(step, ORACLE_RN);
+    } else {
+        zh = oracle_f32_to_f16(mn, ORACLE_RD);
+        float zd = oracle_f16_to_f32(zh);
+        float d = mx - zd;
+        float step = d / (float)Q;
+        sh = oracle_f32_to_f16(step, ORACLE_RU);
+    }
     float z = oracle_f16_to_f32(zh);
-    float d = mx - z;
-    float step = d / (float)Q;
-    uint16_t sh = oracle_f32_to_f16(step, ORACLE_RU);
     float s = oracle_f16_to_f32(sh);
     float inv = 0.0f;
     if (s != 0.0f) {
@@ -273,14 +353,7 @@ uint32_t oracle_quantize_group(const float* v, int m, int bits, uint8_t* codes,
         if (s != 0.0f) {
             float t = v[i] - z;
             float u = t * inv;
-            float r = rintf(u);     /* default rounding mode: half to even */
-            if (r < 0.0f) {
-                r = 0.0f;
-            }
-            if (r > (float)Q) {
-                r = (float)Q;
-            }
-            c = (int)r;
+            c = round_clamp(u, 0, Q);
         }
         codes[i] = (uint8_t)c;
         float cs = (float)c * s;
@@ -291,10 +364,21 @@ uint32_t oracle_quantize_group(const float* v, int m, int bits, uint8_t* codes,
     return flag;
 }
 
-/* dequantize one code with the fp16 parameters of its group */
-static float dequant(int code, uint16_t s_bits, uint16_t z_bits)
+/* the default form (R4) */
+uint32_t oracle_quantize_group(const float* v, int m, int bits, uint8_t* codes,
+                               uint16_t* s_bits, uint16_t* z_bits, float* vhat)
+{
+    return oracle_quantize_group_q(v, m, bits, ORACLE_Q_DIRECTED, codes, s_bits, z_bits, vhat);
+}
+
+/* dequantize one code with the parameter words of its group */
+static float dequant(int code, uint16_t s_bits, uint16_t z_bits, int qmode)
 {
     float s = oracle_f16_to_f32(s_bits);
+    if (qmode == ORACLE_Q_INT_ZERO) {
+        int k = code - (int)z_bits;
+        return (float)k * s;
+    }
     float z = oracle_f16_to_f32(z_bits);
     float cs = (float)code * s;
     return cs + z;
@@ -389,7 +473,7 @@ void oracle_ema_update(float* e, const float* rho, long long count, float alpha)
  *            means "no feedback state" (x' = x, no update)
  *   a2a_codes   [P][jc][group*bits/8] packed all-to-all payload; the slot
  *            of a group's owner is left untouched          (may be NULL)
- *   a2a_params  [P][jc][2] fp16 {s, z} of that payload      (may be NULL)
+ *   a2a_params  [P][jc][2] {s, z} (or {s, zp}, R11) of that payload (may be NULL)
  *   gather_codes [jc][group*bits/8], gather_params [jc][2]: the owner's
  *            requantized sum, sent to every rank            (may be NULL;
  *            untouched when P == 1)
@@ -399,17 +483,18 @@ void oracle_ema_update(float* e, const float* rho, long long count, float alpha)
  *   flags    sticky flag word, ORACLE_FLAG_RANGE on a domain violation
  * Returns 0, or -1 on invalid arguments / allocation failure.
  */
-int oracle_echo_allreduce(int P, long long n_total, int group, int bits,
-                          long long j0, long long jc,
-                          const uint16_t* x, uint16_t* y,
-                          float* e_long, float* e_short,
-                          float eta, float alpha_long, float alpha_short, float w,
-                          uint8_t* a2a_codes, uint16_t* a2a_params,
-                          uint8_t* gather_codes, uint16_t* gather_params,
-                          float* xprime, float* rho, uint8_t* passes,
-                          uint32_t* flags)
+int oracle_echo_allreduce_q(int P, long long n_total, int group, int bits, int qmode,
+                            long long j0, long long jc,
+                            const uint16_t* x, uint16_t* y,
+                            float* e_long, float* e_short,
+                            float eta, float alpha_long, float alpha_short, float w,
+                            uint8_t* a2a_codes, uint16_t* a2a_params,
+                            uint8_t* gather_codes, uint16_t* gather_params,
+                            float* xprime, float* rho, uint8_t* passes,
+                            uint32_t* flags)
 {
-    if (P < 1 || n_total < 1 || group < 2 || (bits != 4 && bits != 8) || jc < 0 || j0 < 0) {
+    if (P < 1 || n_total < 1 || group < 2 || (bits != 4 && bits != 8) || jc < 0 || j0 < 0 ||
+        qmode < ORACLE_Q_DIRECTED || qmode > ORACLE_Q_INT_ZERO) {
         return -1;
     }
     long long G = (n_total + group - 1) / group;
@@ -496,7 +581,7 @@ int oracle_echo_allreduce(int P, long long n_total, int group, int bits,
             size_t base = (size_t)r * (size_t)ld + (size_t)(jl * group);
             uint16_t sb;
             uint16_t zb;
-            flag |= oracle_quantize_group(&xp[base], m, bits, codes, &sb, &zb, vhat);
+            flag |= oracle_quantize_group_q(&xp[base], m, bits, qmode, codes, &sb, &zb, vhat);
             for (int i = m; i < group; i++) {
                 codes[i] = 0;                       /* padding of a partial group */
             }
@@ -534,7 +619,7 @@ int oracle_echo_allreduce(int P, long long n_total, int group, int bits,
                 size_t slot = (size_t)r * (size_t)jc + (size_t)jl;
                 oracle_unpack_codes(&a2a_c[slot * (size_t)cb], group, bits, codes);
                 for (int i = 0; i < m; i++) {
-                    vtmp[i] = dequant(codes[i], a2a_p[2 * slot], a2a_p[2 * slot + 1]);
+                    vtmp[i] = dequant(codes[i], a2a_p[2 * slot], a2a_p[2 * slot + 1], qmode);
                 }
             }
             for (int i = 0; i < m; i++) {
@@ -549,7 +634,7 @@ int oracle_echo_allreduce(int P, long long n_total, int group, int bits,
         if (P >= 2) {
             uint16_t sb;
             uint16_t zb;
-            flag |= oracle_quantize_group(sum, m, bits, codes, &sb, &zb, vhat);
+            flag |= oracle_quantize_group_q(sum, m, bits, qmode, codes, &sb, &zb, vhat);
             for (int i = m; i < group; i++) {
                 codes[i] = 0;
             }
@@ -592,7 +677,7 @@ int oracle_echo_allreduce(int P, long long n_total, int group, int bits,
             for (int r = 0; r < P; r++) {
                 size_t base = (size_t)r * (size_t)ld + (size_t)(jl * group);
                 for (int i = 0; i < m; i++) {
-                    float v = dequant(codes[i], g_p[2 * jl], g_p[2 * jl + 1]);
+                    float v = dequant(codes[i], g_p[2 * jl], g_p[2 * jl + 1], qmode);
                     y[base + (size_t)i] = oracle_f32_to_bf16(v);
                 }
             }
@@ -624,4 +709,20 @@ int oracle_echo_allreduce(int P, long long n_total, int group, int bits,
     free(xp); free(res); free(own_a2a_c); free(own_a2a_p); free(own_g_c); free(own_g_p);
     free(sum); free(vtmp); free(vhat); free(codes); free(y_owner);
     return 0;
+}
+
+/* the default quantizer form (R4) */
+int oracle_echo_allreduce(int P, long long n_total, int group, int bits,
+                          long long j0, long long jc,
+                          const uint16_t* x, uint16_t* y,
+                          float* e_long, float* e_short,
+                          float eta, float alpha_long, float alpha_short, float w,
+                          uint8_t* a2a_codes, uint16_t* a2a_params,
+                          uint8_t* gather_codes, uint16_t* gather_params,
+                          float* xprime, float* rho, uint8_t* passes,
+                          uint32_t* flags)
+{
+    return oracle_echo_allreduce_q(P, n_total, group, bits, ORACLE_Q_DIRECTED, j0, jc, x, y, e_long, e_short,
+                                   eta, alpha_long, alpha_short, w, a2a_codes, a2a_params, gather_codes,
+                                   gather_params, xprime, rho, passes, flags);
 }

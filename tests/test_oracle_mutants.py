@@ -34,10 +34,21 @@ MUTANTS = {
     "nibbles_swapped": [("out[i] = (uint8_t)(lo | (hi << 4));", "out[i] = (uint8_t)(hi | (lo << 4));"),
                         ("codes[2 * i] = (uint8_t)(packed[i] & 0xF);\n        codes[2 * i + 1] = (uint8_t)(packed[i] >> 4);",
                          "codes[2 * i + 1] = (uint8_t)(packed[i] & 0xF);\n        codes[2 * i] = (uint8_t)(packed[i] >> 4);")],
-    "zero_rounded_to_nearest": [("uint16_t zh = oracle_f32_to_f16(mn, ORACLE_RD);",
-                                 "uint16_t zh = oracle_f32_to_f16(mn, ORACLE_RN);")],
-    "scale_rounded_down": [("uint16_t sh = oracle_f32_to_f16(step, ORACLE_RU);",
-                            "uint16_t sh = oracle_f32_to_f16(step, ORACLE_RD);")],
+    "zero_rounded_to_nearest": [("zh = oracle_f32_to_f16(mn, ORACLE_RD);",
+                                 "zh = oracle_f32_to_f16(mn, ORACLE_RN);")],
+    "scale_rounded_down": [("float d = mx - zd;\n        float step = d / (float)Q;\n        sh = oracle_f32_to_f16(step, ORACLE_RU);",
+                            "float d = mx - zd;\n        float step = d / (float)Q;\n        sh = oracle_f32_to_f16(step, ORACLE_RD);")],
+    # the quantizer forms of the ablations
+    "nearest_zero_rounded_down": [("zh = oracle_f32_to_f16(mn, ORACLE_RN);", "zh = oracle_f32_to_f16(mn, ORACLE_RD);")],
+    "nearest_scale_rounded_up": [("sh = oracle_f32_to_f16(step, ORACLE_RN);", "sh = oracle_f32_to_f16(step, ORACLE_RU);")],
+    "nearest_scale_from_rounded_zero": [("        float d = mx - mn;\n", "        float d = mx - oracle_f16_to_f32(zh);\n")],
+    "codes_not_clamped_above": [("    if (c > Q) {\n        c = Q;\n    }\n", "")],
+    "int_zero_scale_rounded_down": [("uint16_t sh = oracle_f32_to_f16(step, ORACLE_RU);",
+                                     "uint16_t sh = oracle_f32_to_f16(step, ORACLE_RD);")],
+    "int_zero_range_not_widened": [("float lo = mn < 0.0f ? mn : 0.0f;", "float lo = mn;")],
+    "int_zero_point_sign": [("float nlo = -lo;", "float nlo = lo;")],
+    "int_zero_codes_without_zero_point": [("c = round_clamp(u, zp, Q);", "c = round_clamp(u, 0, Q);")],
+    "int_zero_dequant_drops_zero_point": [("        int k = code - (int)z_bits;", "        int k = code;")],
     "codes_truncated": [("float r = rintf(u);", "float r = floorf(u);")],
     "segment_off_by_one": [("if (j >= oracle_segment_begin(s, G, P) && j < oracle_segment_begin(s + 1, G, P)) {",
                             "if (j >= oracle_segment_begin(s, G, P) && j <= oracle_segment_begin(s + 1, G, P)) {")],
@@ -46,7 +57,7 @@ MUTANTS = {
     "no_feedback_add": [("                xp[idx] = xv + c;", "                xp[idx] = xv;")],
 }
 
-PIN_FILES = ["tests/test_oracle_call.py", "tests/test_oracle_quantizer.py",
+PIN_FILES = ["tests/test_oracle_call.py", "tests/test_oracle_quantizer.py", "tests/test_oracle_variants.py",
              "tests/test_oracle_chain.py", "tests/test_oracle_convert.py"]
 
 
