@@ -24,6 +24,7 @@ struct echo_state {
     uint8_t* workspace;
     int device;
     int sm_count;
+    int quantizer;         // ECHO_QUANT_*; ECHO_QUANT_DIRECTED unless set
 };
 
 namespace {
@@ -110,7 +111,7 @@ int launch_pipe(K kernel, int* grid, int64_t max_tiles, const echo_dev::Args& a,
     return ECHO_OK;
 }
 
-template <int GROUP, int BITS>
+template <int GROUP, int BITS, int QM>
 int launch_stage(Stage stage, const echo_dev::Args& a, const echo_state* st, cudaStream_t s) {
     int rc = ECHO_OK;
     // tiles of 2048 elements with feedback; without, 4 x 2048 (quantize) and
@@ -123,23 +124,23 @@ int launch_stage(Stage stage, const echo_dev::Args& a, const echo_state* st, cud
         case Stage::Quantize:
             if (a.state) {
                 static int grid = 0;
-                rc = launch_pipe(echo_dev::k_quantize_tma<GROUP, BITS, true>, &grid, tiles, a, st, s);
+                rc = launch_pipe(echo_dev::k_quantize_tma<GROUP, BITS, true, QM>, &grid, tiles, a, st, s);
             } else {
                 static int grid = 0;
-                rc = launch_pipe(echo_dev::k_quantize_tma<GROUP, BITS, false>, &grid, tiles, a, st, s);
+                rc = launch_pipe(echo_dev::k_quantize_tma<GROUP, BITS, false, QM>, &grid, tiles, a, st, s);
             }
             break;
         case Stage::Reduce:
             if (a.state) {
                 static int grid = 0;
-                rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, true>, &grid, tiles, a, st, s);
+                rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, true, QM>, &grid, tiles, a, st, s);
             } else {
                 static int grid = 0;
-                rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, false>, &grid, tiles, a, st, s);
+                rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, false, QM>, &grid, tiles, a, st, s);
             }
             break;
         case Stage::Gather: {
-            auto k = echo_dev::k_gather_tma<GROUP, BITS>;
+            auto k = echo_dev::k_gather_tma<GROUP, BITS, QM>;
             static int grid = 0;
             if (grid == 0) grid = grid_for(k, st, echo_dev::kGatherThreads, echo_dev::kGatherSmem);
             k<<<grid, echo_dev::kGatherThreads, echo_dev::kGatherSmem, s>>>(a);
@@ -152,7 +153,18 @@ int launch_stage(Stage stage, const echo_dev::Args& a, const echo_state* st, cud
 
 template <int GROUP>
 int launch_bits(Stage stage, int bits, const echo_dev::Args& a, const echo_state* st, cudaStream_t s) {
-    return bits == 4 ? launch_stage<GROUP, 4>(stage, a, st, s) : launch_stage<GROUP, 8>(stage, a, st, s);
+    switch (st->quantizer) {
+        case ECHO_QUANT_DIRECTED:
+            return bits == 4 ? launch_stage<GROUP, 4, echo_dev::kQuantDirected>(stage, a, st, s)
+                             : launch_stage<GROUP, 8, echo_dev::kQuantDirected>(stage, a, st, s);
+        case ECHO_QUANT_NEAREST:
+            return bits == 4 ? launch_stage<GROUP, 4, echo_dev::kQuantNearest>(stage, a, st, s)
+                             : launch_stage<GROUP, 8, echo_dev::kQuantNearest>(stage, a, st, s);
+        case ECHO_QUANT_INT_ZERO:
+            return bits == 4 ? launch_stage<GROUP, 4, echo_dev::kQuantIntZero>(stage, a, st, s)
+                             : launch_stage<GROUP, 8, echo_dev::kQuantIntZero>(stage, a, st, s);
+    }
+    return ECHO_EINVAL;
 }
 
 int launch(Stage stage, int bits, const echo_dev::Args& a, const echo_state* st, cudaStream_t s) {
@@ -260,7 +272,16 @@ int echo_init_state(echo_state** out, int64_t n, int P, int group, int max_bits,
     st->workspace = static_cast<uint8_t*>(workspace_dev);
     st->device = dev;
     st->sm_count = sms;
+    st->quantizer = ECHO_QUANT_DIRECTED;
     *out = st;
+    return ECHO_OK;
+}
+
+int echo_set_quantizer(echo_state* st, int quantizer) {
+    if (!st) return ECHO_EINVAL;
+    if (quantizer != ECHO_QUANT_DIRECTED && quantizer != ECHO_QUANT_NEAREST && quantizer != ECHO_QUANT_INT_ZERO)
+        return ECHO_EINVAL;
+    st->quantizer = quantizer;
     return ECHO_OK;
 }
 
@@ -401,6 +422,7 @@ int echo_allreduce_sim_noalloc(const void* const* inputs, void* const* outputs, 
     st.workspace = scratch;
     st.device = dev;
     st.sm_count = sms;
+    st.quantizer = ECHO_QUANT_DIRECTED;
     echo_dev::Args a;
     if (!make_args(&st, bits, inputs, outputs, eta, alpha_long, alpha_short, w, &a)) return ECHO_EINVAL;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

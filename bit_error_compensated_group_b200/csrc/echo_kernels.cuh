@@ -73,12 +73,53 @@ __device__ __forceinline__ bool outside_fp16_domain(float v) {
     return !(v >= -65504.0f && v <= 65504.0f);   // NaN fails both
 }
 
-// Quantization grid of one group: fp16 zero z (rounded toward -inf from the
-// minimum) and step s (rounded toward +inf from (max - z) / Q).
+// Quantizer forms (template parameter QM): 0 = fp16 zero rounded toward -inf
+// from the minimum and step rounded toward +inf from (max - z) / Q (the
+// default); 1 = zero and step (max - min) / Q both rounded to nearest, codes
+// clamped; 2 = integer zero point: range widened to include 0, step rounded
+// up, zp = rint(-lo / s), code = rint(v / s) + zp, value (code - zp) * s.
+constexpr int kQuantDirected = 0, kQuantNearest = 1, kQuantIntZero = 2;
+
+// Quantization grid of one group. A code c decodes to c * s + zf (c * s is
+// exact); encoding rounds (v - zsub) * inv to an integer and adds zq.
 struct Grid {
-    float s, z, inv;
-    uint32_t param;   // fp16 bits: s | z << 16
+    float s, zf, zsub, inv;
+    int zq;
+    uint32_t param;   // s | z << 16 (fp16 bits), or s | zp << 16 for the integer zero point
 };
+
+// Parameters of a group from its range [mn, mx] (both already +0-canonical).
+template <int Q, int QM>
+__device__ __forceinline__ Grid group_grid(float mn, float mx) {
+    Grid g;
+    if (QM == kQuantIntZero) {
+        const float lo = mn < 0.0f ? mn : 0.0f, hi = mx > 0.0f ? mx : 0.0f;
+        const __half sh = __float2half_ru(__fdiv_rn(__fsub_rn(hi, lo), (float)Q));
+        g.s = __half2float(sh);
+        g.inv = (g.s != 0.0f) ? __fdiv_rn(1.0f, g.s) : 0.0f;
+        int zp = 0;
+        if (g.s != 0.0f) zp = min(max(__float2int_rn(__fmul_rn(-lo, g.inv)), 0), Q);
+        g.zq = zp;
+        g.zsub = 0.0f;
+        g.zf = __fmul_rn(__int2float_rn(-zp), g.s);   // exact: |zp| <= 255, s has 11 bits
+        g.param = (uint32_t)__half_as_ushort(sh) | ((uint32_t)zp << 16);
+        return g;
+    }
+    __half zh, sh;
+    if (QM == kQuantNearest) {
+        zh = __float2half_rn(mn);
+        sh = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), (float)Q));
+    } else {
+        zh = __float2half_rd(mn);
+        sh = __float2half_ru(__fdiv_rn(__fsub_rn(mx, __half2float(zh)), (float)Q));
+    }
+    g.s = __half2float(sh);
+    g.zf = g.zsub = __half2float(zh);
+    g.zq = 0;
+    g.inv = (g.s != 0.0f) ? __fdiv_rn(1.0f, g.s) : 0.0f;   // s == 0 -> every code 0
+    g.param = (uint32_t)__half_as_ushort(sh) | ((uint32_t)__half_as_ushort(zh) << 16);
+    return g;
+}
 
 template <int L>
 __device__ __forceinline__ float group_min(float v) {
@@ -96,36 +137,33 @@ __device__ __forceinline__ float group_max(float v) {
 
 // All 32 lanes must call this (it shuffles); lanes of an inactive group pass
 // neutral values and ignore the result.
-template <int L, int Q>
+template <int L, int Q, int QM>
 __device__ __forceinline__ Grid make_grid(float lane_min, float lane_max) {
-    float mn = group_min<L>(lane_min);
-    float mx = group_max<L>(lane_max);
-    mn = __fadd_rn(mn, 0.0f);   // -0 -> +0
-    mx = __fadd_rn(mx, 0.0f);
-    const __half zh = __float2half_rd(mn);
-    const float z = __half2float(zh);
-    const float d = __fsub_rn(mx, z);
-    const __half sh = __float2half_ru(__fdiv_rn(d, (float)Q));
-    Grid g;
-    g.s = __half2float(sh);
-    g.z = z;
-    g.inv = (g.s != 0.0f) ? __fdiv_rn(1.0f, g.s) : 0.0f;   // s == 0 -> every code 0
-    g.param = (uint32_t)__half_as_ushort(sh) | ((uint32_t)__half_as_ushort(zh) << 16);
-    return g;
+    const float mn = __fadd_rn(group_min<L>(lane_min), 0.0f);   // -0 -> +0
+    const float mx = __fadd_rn(group_max<L>(lane_max), 0.0f);
+    return group_grid<Q, QM>(mn, mx);
 }
 
-template <int Q>
+template <int Q, int QM>
 __device__ __forceinline__ int encode(float v, const Grid& g) {
-    const int q = __float2int_rn(__fmul_rn(__fsub_rn(v, g.z), g.inv));   // half to even
+    float u = __fmul_rn(__fsub_rn(v, g.zsub), g.inv);
+    if (QM != kQuantDirected) u = fminf(fmaxf(u, -(float)(Q + 1)), (float)(Q + 1));   // rint, then clamp, agree
+    const int q = __float2int_rn(u) + g.zq;   // half to even
     return min(max(q, 0), Q);
 }
 
-__device__ __forceinline__ float decode(int q, float s, float z) {
-    return __fadd_rn(__fmul_rn(__int2float_rn(q), s), z);   // q*s is exact
+__device__ __forceinline__ float decode(int q, float s, float zf) {
+    return __fadd_rn(__fmul_rn(__int2float_rn(q), s), zf);   // q*s is exact
 }
 
 __device__ __forceinline__ float param_s(uint32_t p) { return __half2float(__ushort_as_half((unsigned short)(p & 0xffffu))); }
 __device__ __forceinline__ float param_z(uint32_t p) { return __half2float(__ushort_as_half((unsigned short)(p >> 16))); }
+// the additive term of a group's decode, c * s + zf, from its parameter word
+template <int QM>
+__device__ __forceinline__ float param_zf(uint32_t p, float s) {
+    if (QM == kQuantIntZero) return __fmul_rn(__int2float_rn(-(int)(p >> 16)), s);   // -zp * s, exact
+    return param_z(p);
+}
 
 // codes of one 4-element chunk: 4 nibbles in 16 bits, or 4 bytes in 32 bits
 template <int BITS>
@@ -225,7 +263,7 @@ struct Lane {
 };
 
 // Stage 1: quantize the groups [j_begin, j_end) of rank r (none owned by r).
-template <int GROUP, int BITS>
+template <int GROUP, int BITS, int QM>
 __device__ __forceinline__ void quantize_range(const Args& a, int r, long long j_begin, long long j_end,
                                                long long warp, long long nwarps) {
     using LN = Lane<GROUP>;
@@ -267,7 +305,7 @@ __device__ __forceinline__ void quantize_range(const Args& a, int r, long long j
             }
         }
         raise_flags(a, bad);
-        const Grid g = make_grid<L, Q>(lmin, lmax);
+        const Grid g = make_grid<L, Q, QM>(lmin, lmax);
         if (act) {
             uint8_t* codes = a.a2a_codes + ((size_t)r * a.G + j) * CB;
 #pragma unroll
@@ -278,9 +316,9 @@ __device__ __forceinline__ void quantize_range(const Args& a, int r, long long j
                 for (int k = 0; k < 4; ++k) {
                     const int i = 4 * h + k;
                     const bool valid = full || e + k < a.n;
-                    q[k] = valid ? encode<Q>(v[i], g) : 0;
+                    q[k] = valid ? encode<Q, QM>(v[i], g) : 0;
                     if (a.state) {
-                        const float rho = __fsub_rn(v[i], decode(q[k], g.s, g.z));
+                        const float rho = __fsub_rn(v[i], decode(q[k], g.s, g.zf));
                         el[i] = ema(el[i], rho, a.keep_long, a.a_long);
                         es[i] = ema(es[i], rho, a.keep_short, a.a_short);
                     }
@@ -297,7 +335,7 @@ __device__ __forceinline__ void quantize_range(const Args& a, int r, long long j
 }
 
 // Stage 2: owner o sums and requantizes its groups [j_begin, j_end).
-template <int GROUP, int BITS>
+template <int GROUP, int BITS, int QM>
 __device__ __forceinline__ void reduce_range(const Args& a, int o, long long j_begin, long long j_end,
                                              long long warp, long long nwarps) {
     using LN = Lane<GROUP>;
@@ -351,7 +389,7 @@ __device__ __forceinline__ void reduce_range(const Args& a, int o, long long j_b
                 const int r = r0 + k;
                 if (r < a.P) {
                     const float s = param_s(pw[k]);
-                    const float z = param_z(pw[k]);
+                    const float z = param_zf<QM>(pw[k], s);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         const float term = (r == o) ? xo[i] : decode(unpack1<BITS>(cw[k][i >> 2], i & 3), s, z);
@@ -380,7 +418,7 @@ __device__ __forceinline__ void reduce_range(const Args& a, int o, long long j_b
         raise_flags(a, bad);
         uint32_t yb[8];
         if (a.P >= 2) {
-            const Grid g = make_grid<L, Q>(lmin, lmax);
+            const Grid g = make_grid<L, Q, QM>(lmin, lmax);
             if (act) {
                 uint8_t* codes = a.g_codes + (size_t)j * CB;
 #pragma unroll
@@ -390,8 +428,8 @@ __device__ __forceinline__ void reduce_range(const Args& a, int o, long long j_b
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
                         const bool valid = full || e + k < a.n;
-                        q[k] = valid ? encode<Q>(acc[4 * h + k], g) : 0;
-                        yb[4 * h + k] = f2bf16(decode(q[k], g.s, g.z));
+                        q[k] = valid ? encode<Q, QM>(acc[4 * h + k], g) : 0;
+                        yb[4 * h + k] = f2bf16(decode(q[k], g.s, g.zf));
                     }
                     store_chunk_codes<BITS>(codes, ln.chunk(h), pack4<BITS>(q));
                     if (a.write_outputs) {

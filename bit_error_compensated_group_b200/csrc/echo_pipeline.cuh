@@ -330,35 +330,34 @@ __device__ __forceinline__ float nan_max3(float a, float b, float c) {
     return r;
 }
 
-// Packed quantization grid of one group (same values as make_grid).
+// Packed quantization grid of one group (same values as make_grid). A code
+// decodes to code * s + z (z is the additive term zf of the scalar Grid).
 struct GridP {
     float2 s, z, ns, nz, inv;
+    float2 nzs;   // -zsub (nearest form)
+    int C;        // 0x4B400000 - zq: signed-magic bits of code 0 (nearest and integer-zero forms)
     uint32_t param;
     bool bad;   // a value outside [-65504, 65504] or a NaN
 };
 
 // fp16 parameters of a group from its range [mn, mx] (same values as make_grid).
-template <int Q>
+template <int Q, int QM>
 __device__ __forceinline__ GridP grid_from_range(float mn, float mx) {
-    GridP g;
-    g.bad = !(mn >= -65504.0f && mx <= 65504.0f);
-    mn = __fadd_rn(mn, 0.0f);   // -0 -> +0
-    mx = __fadd_rn(mx, 0.0f);
-    const __half zh = __float2half_rd(mn);
-    const float z = __half2float(zh);
-    const __half sh = __float2half_ru(__fdiv_rn(__fsub_rn(mx, z), (float)Q));
-    const float s = __half2float(sh);
-    const float inv = (s != 0.0f) ? __fdiv_rn(1.0f, s) : 0.0f;
-    g.s = splat(s);
-    g.z = splat(z);
-    g.ns = splat(-s);
-    g.nz = splat(-z);
-    g.inv = splat(inv);
-    g.param = (uint32_t)__half_as_ushort(sh) | ((uint32_t)__half_as_ushort(zh) << 16);
-    return g;
+    GridP gp;
+    gp.bad = !(mn >= -65504.0f && mx <= 65504.0f);
+    const Grid g = group_grid<Q, QM>(__fadd_rn(mn, 0.0f), __fadd_rn(mx, 0.0f));   // -0 -> +0
+    gp.s = splat(g.s);
+    gp.z = splat(g.zf);
+    gp.ns = splat(-g.s);
+    gp.nz = splat(-g.zf);
+    gp.inv = splat(g.inv);
+    gp.nzs = splat(-g.zsub);
+    gp.C = 0x4B400000 - g.zq;
+    gp.param = g.param;
+    return gp;
 }
 
-template <int L, int Q>
+template <int L, int Q, int QM>
 __device__ __forceinline__ GridP make_grid_p(float lane_min, float lane_max) {
     float mn = lane_min, mx = lane_max;
 #pragma unroll
@@ -366,7 +365,7 @@ __device__ __forceinline__ GridP make_grid_p(float lane_min, float lane_max) {
         mn = nan_min(mn, __shfl_xor_sync(kFull, mn, o));
         mx = nan_max(mx, __shfl_xor_sync(kFull, mx, o));
     }
-    return grid_from_range<Q>(mn, mx);
+    return grid_from_range<Q, QM>(mn, mx);
 }
 
 // p + q where p (or q) is a rounded product: fma(p, one, q), one = 1.0 at run time
@@ -374,10 +373,29 @@ __device__ __forceinline__ float2 add_after_mul2(float2 p, float2 q, const Args&
     return fma2_rn(p, splat(a.one), q);
 }
 
-// 2^23 + code for a pair of values: code = round_half_even((v - z) * inv)
+// 2^23 + code for a pair of values (the code sits in the low mantissa bits).
+// Default form: code = round_half_even((v - z) * inv), in [0, Q] without a
+// clamp because the directed parameters make [z, z + Q s] cover the group.
+// Other forms: u = (v - z) * inv (nearest) or v * inv (integer zero), clamped
+// to [-(Q+1), Q+1] (then rint-and-clamp agrees with clamping first); adding
+// 1.5 * 2^23 rounds u to an integer with ties to even (the magic is even and
+// the spacing there is 1), leaving bits 0x4B400000 + rint(u); subtracting
+// C = 0x4B400000 - zq gives rint(u) + zq, clamped to [0, Q].
+constexpr float kMagicSigned = 12582912.0f;   // 1.5 * 2^23
+
+template <int QM, int Q>
 __device__ __forceinline__ float2 encode2(float2 v, const GridP& g, const Args& a) {
-    const float2 u = mul2_rn(add2_rn(v, g.nz), g.inv);   // (v - z) * inv
-    return add_after_mul2(u, splat(kMagic), a);
+    if (QM == kQuantDirected) {
+        const float2 u = mul2_rn(add2_rn(v, g.nz), g.inv);   // (v - z) * inv
+        return add_after_mul2(u, splat(kMagic), a);
+    }
+    float2 u = (QM == kQuantNearest) ? mul2_rn(add2_rn(v, g.nzs), g.inv) : mul2_rn(v, g.inv);
+    u.x = fminf(fmaxf(u.x, -(float)(Q + 1)), (float)(Q + 1));
+    u.y = fminf(fmaxf(u.y, -(float)(Q + 1)), (float)(Q + 1));
+    const float2 t = add_after_mul2(u, splat(kMagicSigned), a);
+    const int cx = min(max((int)__float_as_uint(t.x) - g.C, 0), Q);
+    const int cy = min(max((int)__float_as_uint(t.y) - g.C, 0), Q);
+    return make_float2(__uint_as_float(0x4B000000u | (uint32_t)cx), __uint_as_float(0x4B000000u | (uint32_t)cy));
 }
 
 
@@ -478,7 +496,7 @@ __device__ __forceinline__ void store_f8_cs(float* p, const float2 v[4]) {
 // One non-owned group of a tile with feedback (x, e_long, e_short staged):
 // 8 consecutive elements per lane (lane t of the group's L takes elements
 // [8t, 8t + 8)).
-template <int GROUP, int BITS>
+template <int GROUP, int BITS, int QM>
 __device__ __forceinline__ void quantize_tile_group(const Args& a, const uint8_t* st, const Tile& t, int gi,
                                                     bool act) {
     using LN = Lane<GROUP>;
@@ -503,12 +521,12 @@ __device__ __forceinline__ void quantize_tile_group(const Args& a, const uint8_t
             lmax = nan_max3(lmax, v[p].x, v[p].y);
         }
     }
-    const GridP g = make_grid_p<L, Q>(lmin, lmax);
+    const GridP g = make_grid_p<L, Q, QM>(lmin, lmax);
     raise_flags(a, act && g.bad);
     if (!act) return;
     float2 e[4];
 #pragma unroll
-    for (int p = 0; p < 4; ++p) e[p] = encode2(v[p], g, a);
+    for (int p = 0; p < 4; ++p) e[p] = encode2<QM, Q>(v[p], g, a);
     uint8_t* codes = a.a2a_codes + ((size_t)r * a.G + j) * CB;
     const uint2 pk = pack_codes8<BITS>(e);
     if (BITS == 4) *reinterpret_cast<uint32_t*>(codes + 4 * ln.t) = pk.x;
@@ -575,7 +593,7 @@ __device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
 
 __device__ __forceinline__ float2 bf16_pair(uint32_t u) { return make_float2(bf16_lo(u), bf16_hi(u)); }
 
-template <int GROUP, int BITS>
+template <int GROUP, int BITS, int QM>
 __device__ __forceinline__ void quantize_tile_group_nf(const Args& a, const uint8_t* st, const Tile& t, int gi,
                                                        bool act) {
     using LN = LaneE<GROUP, kQuantizeLaneElemsNF>;
@@ -605,7 +623,7 @@ __device__ __forceinline__ void quantize_tile_group_nf(const Args& a, const uint
     }
 #pragma unroll
     for (int o = L / 2; o > 0; o >>= 1) mm = bmin2(mm, __shfl_xor_sync(kFull, mm, o));
-    const GridP g = grid_from_range<Q>(__uint_as_float(mm << 16), __uint_as_float((mm & 0xffff0000u) ^ 0x80000000u));
+    const GridP g = grid_from_range<Q, QM>(__uint_as_float(mm << 16), __uint_as_float((mm & 0xffff0000u) ^ 0x80000000u));
     raise_flags(a, act && g.bad);
     if (!act) return;
     const long long j = t.j0 + gi;
@@ -613,10 +631,10 @@ __device__ __forceinline__ void quantize_tile_group_nf(const Args& a, const uint
 #pragma unroll
     for (int h = 0; h < H; ++h) {
         float2 e[4];
-        e[0] = encode2(bf16_pair(w[h].x), g, a);
-        e[1] = encode2(bf16_pair(w[h].y), g, a);
-        e[2] = encode2(bf16_pair(w[h].z), g, a);
-        e[3] = encode2(bf16_pair(w[h].w), g, a);
+        e[0] = encode2<QM, Q>(bf16_pair(w[h].x), g, a);
+        e[1] = encode2<QM, Q>(bf16_pair(w[h].y), g, a);
+        e[2] = encode2<QM, Q>(bf16_pair(w[h].z), g, a);
+        e[3] = encode2<QM, Q>(bf16_pair(w[h].w), g, a);
         const uint2 pk = pack_codes8<BITS>(e);
         const int c = ln.chunk(h ^ flip);
         if (BITS == 4) *reinterpret_cast<uint32_t*>(codes + 4 * c) = pk.x;
@@ -625,7 +643,7 @@ __device__ __forceinline__ void quantize_tile_group_nf(const Args& a, const uint
     if (ln.t == 0) a.a2a_params[(size_t)t.rank * a.G + j] = g.param;
 }
 
-template <int GROUP, int BITS, bool FB>
+template <int GROUP, int BITS, bool FB, int QM>
 __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
     constexpr int M = FB ? 1 : kQuantizeSubtilesNF;
@@ -655,12 +673,12 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
         }
         const uint8_t* stage = p.stages + (size_t)s * kStageBytes;
         if (FB) {
-            quantize_tile_group<GROUP, BITS>(a, stage, t, gi, gi < t.count);
+            quantize_tile_group<GROUP, BITS, QM>(a, stage, t, gi, gi < t.count);
         } else {
 #pragma unroll 1
             for (int m = 0; m < PASSES; ++m) {
                 const int g = gi + m * kConsumerWarps * GPW;
-                quantize_tile_group_nf<GROUP, BITS>(a, stage, t, g, g < t.count);
+                quantize_tile_group_nf<GROUP, BITS, QM>(a, stage, t, g, g < t.count);
             }
         }
         __syncwarp();
@@ -671,7 +689,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
         const long long j = a.G - 1;
         for (int r = 0; r < a.P; ++r) {
             const long long lo = (long long)r * a.G / a.P, hi = (long long)(r + 1) * a.G / a.P;
-            if (j < lo || j >= hi) quantize_range<GROUP, BITS>(a, r, j, j + 1, 0, 1);
+            if (j < lo || j >= hi) quantize_range<GROUP, BITS, QM>(a, r, j, j + 1, 0, 1);
         }
     }
 }
@@ -680,7 +698,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
 
 // One owned group of a tile with feedback (x, e_long, e_short staged): 8
 // consecutive elements per lane, like the quantize pass.
-template <int GROUP, int BITS>
+template <int GROUP, int BITS, int QM>
 __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* st, const Tile& t, int gi,
                                                   bool act) {
     using LN = Lane<GROUP>;
@@ -737,8 +755,9 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
 #pragma unroll
                 for (int p = 0; p < 4; ++p) term[p] = xo[p];
             } else {
-                const float2 s2 = splat(param_s(pw[k]));
-                const float2 z2 = splat(param_z(pw[k]));
+                const float sk = param_s(pw[k]);
+                const float2 s2 = splat(sk);
+                const float2 z2 = splat(param_zf<QM>(pw[k], sk));
                 float2 q[4];
                 unpack_codes8<BITS>(cw[k], q);
 #pragma unroll
@@ -758,13 +777,13 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
     }
     uint32_t yb[4];   // bf16 pairs of the result
     if (a.P >= 2) {
-        const GridP g = make_grid_p<L, Q>(lmin, lmax);
+        const GridP g = make_grid_p<L, Q, QM>(lmin, lmax);
         raise_flags(a, act && g.bad);
         if (!act) return;
         float2 e[4];
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
-            e[p] = encode2(acc[p], g, a);
+            e[p] = encode2<QM, Q>(acc[p], g, a);
             yb[p] = bf16x2_rn(fma2_rn(add2_rn(e[p], splat(-kMagic)), g.s, g.z));
         }
         uint8_t* codes = a.g_codes + (size_t)j * CB;
@@ -805,7 +824,7 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
 // The owner's pass without feedback, 16 elements per lane (chunks t and
 // t + L16 of 8 elements): twice the elements per payload load batch and per
 // group-level step of the 8-element path, and 16-byte output stores.
-template <int GROUP, int BITS>
+template <int GROUP, int BITS, int QM>
 __device__ __forceinline__ void reduce_tile_group_nf(const Args& a, const uint8_t* st, const Tile& t, int gi,
                                                      bool act) {
     using LN = Lane16<GROUP>;
@@ -864,8 +883,9 @@ __device__ __forceinline__ void reduce_tile_group_nf(const Args& a, const uint8_
                     term[4 * h + 3] = bf16_pair(xw[h].w);
                 }
             } else {
-                const float2 s2 = splat(param_s(pw[k]));
-                const float2 z2 = splat(param_z(pw[k]));
+                const float sk = param_s(pw[k]);
+                const float2 s2 = splat(sk);
+                const float2 z2 = splat(param_zf<QM>(pw[k], sk));
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     float2 q[4];
@@ -888,7 +908,7 @@ __device__ __forceinline__ void reduce_tile_group_nf(const Args& a, const uint8_
     }
     uint32_t yw[8];   // bf16 pairs of the result
     if (a.P >= 2) {
-        const GridP g = make_grid_p<L, Q>(lmin, lmax);
+        const GridP g = make_grid_p<L, Q, QM>(lmin, lmax);
         raise_flags(a, act && g.bad);
         if (!act) return;
         uint8_t* codes = a.g_codes + (size_t)j * CB;
@@ -896,7 +916,7 @@ __device__ __forceinline__ void reduce_tile_group_nf(const Args& a, const uint8_
         for (int h = 0; h < 2; ++h) {
             float2 e[4];
 #pragma unroll
-            for (int p = 0; p < 4; ++p) e[p] = encode2(acc[4 * h + p], g, a);
+            for (int p = 0; p < 4; ++p) e[p] = encode2<QM, Q>(acc[4 * h + p], g, a);
             const uint2 pk = pack_codes8<BITS>(e);
             if (BITS == 4) *reinterpret_cast<uint32_t*>(codes + 4 * ln.chunk(h)) = pk.x;
             else *reinterpret_cast<uint2*>(codes + 8 * ln.chunk(h)) = pk;
@@ -925,7 +945,7 @@ __device__ __forceinline__ void reduce_tile_group_nf(const Args& a, const uint8_
     }
 }
 
-template <int GROUP, int BITS, bool FB>
+template <int GROUP, int BITS, bool FB, int QM>
 __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
     constexpr int M = FB ? 1 : kReduceSubtilesNF;
@@ -953,12 +973,12 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
         }
         const uint8_t* stage = p.stages + (size_t)s * kStageBytes;
         if (FB) {
-            reduce_tile_group<GROUP, BITS>(a, stage, t, gi, gi < t.count);
+            reduce_tile_group<GROUP, BITS, QM>(a, stage, t, gi, gi < t.count);
         } else {
 #pragma unroll 1
             for (int m = 0; m < PASSES; ++m) {
                 const int g = gi + m * kConsumerWarps * GPW;
-                reduce_tile_group_nf<GROUP, BITS>(a, stage, t, g, g < t.count);
+                reduce_tile_group_nf<GROUP, BITS, QM>(a, stage, t, g, g < t.count);
             }
         }
         __syncwarp();
@@ -967,7 +987,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
     if (G_full < a.G && blockIdx.x == gridDim.x - 1 && warp == 0) {
         const long long j = a.G - 1;
         const int o = (int)((j * a.P + a.P - 1) / a.G);
-        reduce_range<GROUP, BITS>(a, o, j, j + 1, 0, 1);
+        reduce_range<GROUP, BITS, QM>(a, o, j, j + 1, 0, 1);
     }
 }
 
@@ -1005,10 +1025,11 @@ __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wa
 
 // eight contiguous decoded elements of a group as bf16 (codes word w: 4-bit in
 // w.x, 8-bit in w.x and w.y)
-template <int BITS>
+template <int BITS, int QM>
 __device__ __forceinline__ uint4 decode8_bf16(uint2 w, uint32_t param) {
-    const float2 s2 = splat(param_s(param));
-    const float2 z2 = splat(param_z(param));
+    const float s = param_s(param);
+    const float2 s2 = splat(s);
+    const float2 z2 = splat(param_zf<QM>(param, s));
     float2 q[4];
     const uint32_t cw[2] = {w.x, w.y};
     unpack_codes8<BITS>(cw, q);
@@ -1016,7 +1037,7 @@ __device__ __forceinline__ uint4 decode8_bf16(uint2 w, uint32_t param) {
                       bf16x2_rn(fma2_rn(q[2], s2, z2)), bf16x2_rn(fma2_rn(q[3], s2, z2)));
 }
 
-template <int GROUP, int BITS>
+template <int GROUP, int BITS, int QM>
 __global__ void __launch_bounds__(kGatherThreads) k_gather_tma(const Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
     constexpr int L = GROUP / 8, CB = GROUP * BITS / 8, T = kGatherTileElems / GROUP;
@@ -1038,7 +1059,7 @@ __global__ void __launch_bounds__(kGatherThreads) k_gather_tma(const Args a) {
         if (gi < cnt) {
             const long long j = j0 + gi;
             const uint2 w = load_codes8<BITS>(a.g_codes + (size_t)j * CB, t);
-            *reinterpret_cast<uint4*>(buf + gi * GROUP + 8 * t) = decode8_bf16<BITS>(w, a.g_params[j]);
+            *reinterpret_cast<uint4*>(buf + gi * GROUP + 8 * t) = decode8_bf16<BITS, QM>(w, a.g_params[j]);
         }
         fence_proxy_async_smem();
         __syncthreads();
@@ -1053,7 +1074,7 @@ __global__ void __launch_bounds__(kGatherThreads) k_gather_tma(const Args a) {
     if (G_full < a.G && blockIdx.x == gridDim.x - 1 && tid < L) {
         const long long j = a.G - 1;
         const uint2 w = load_codes8<BITS>(a.g_codes + (size_t)j * CB, tid);
-        const uint4 v = decode8_bf16<BITS>(w, a.g_params[j]);
+        const uint4 v = decode8_bf16<BITS, QM>(w, a.g_params[j]);
         const uint32_t yb[4] = {v.x, v.y, v.z, v.w};
         const long long e = j * GROUP + 8 * tid;
         for (int r = 0; r < a.P; ++r) {

@@ -20,6 +20,7 @@ ECHO_NOALLOC_SCRATCH_BYTES = 16 << 20
 ECHO_FLAG_RANGE = 1
 ECHO_FLAG_TIMEOUT = 2
 ECHO_MAX_RANKS = 64
+ECHO_QUANT_DIRECTED, ECHO_QUANT_NEAREST, ECHO_QUANT_INT_ZERO = 0, 1, 2
 
 LIB_PATH = _build.LIB
 
@@ -77,6 +78,8 @@ def lib() -> ctypes.CDLL:
         L.echo_check_watchdog.restype = I
         L.echo_get_status.argtypes = [V, V, ctypes.POINTER(ctypes.c_uint32)]
         L.echo_get_status.restype = I
+        L.echo_set_quantizer.argtypes = [V, I]
+        L.echo_set_quantizer.restype = I
         L.echo_free.argtypes = [V]
         L.echo_free.restype = I
         L.echo_status_string.argtypes = [I]
@@ -197,6 +200,11 @@ def echo_allreduce_sim_noalloc(inputs: Sequence, outputs: Sequence, state, n: in
     return int(flags.value) if read_flags else None
 
 
+def echo_set_quantizer(st, quantizer: int) -> None:
+    """Quantizer form for the handle's later calls (ECHO_QUANT_*)."""
+    _check(lib().echo_set_quantizer(st, quantizer), "echo_set_quantizer")
+
+
 def echo_free(st) -> None:
     lib().echo_free(st)
 
@@ -208,7 +216,7 @@ class EchoAllReduce:
     and the library handle; ``__call__`` runs echo_allreduce_sim."""
 
     def __init__(self, n: int, P: int, group: int = 128, max_bits: int = 4, feedback: bool = True,
-                 device=None, stream=None):
+                 device=None, stream=None, quantizer: int = ECHO_QUANT_DIRECTED):
         device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
         self.n, self.P, self.group, self.max_bits = n, P, group, max_bits
         self.layout = echo_query_layout(n, P, group, max_bits, max_bits)
@@ -217,6 +225,8 @@ class EchoAllReduce:
         if feedback:
             self.state = torch.empty(int(self.layout.state_bytes) // 4, dtype=torch.float32, device=device)
         self.handle = echo_init_state(n, P, group, max_bits, self.state, self.workspace, stream)
+        if quantizer != ECHO_QUANT_DIRECTED:
+            echo_set_quantizer(self.handle, quantizer)
 
     def __call__(self, inputs, outputs, bits: int = 4, eta: float = 1.0, alpha_long: float = 0.05,
                  alpha_short: float = 0.5, w: float = 0.5, stream=None) -> None:

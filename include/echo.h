@@ -142,6 +142,38 @@ ECHO_API int echo_init_state(echo_state** out, int64_t n, int P, int group, int 
                     void* state_dev, void* workspace_dev, echo_stream_t stream);
 
 /*
+ * Quantizer forms. The Echo explainer (section "Echoの仕組み①", mechanism 1)
+ * names an asymmetric, zero-point-aware group quantizer with half-precision
+ * parameters (section "よくある質問", FAQ) and fixes neither how those
+ * parameters round nor whether the zero is a float or an integer; the
+ * ablations compare three readings. Every form ships `bits`-bit codes plus
+ * one 32-bit parameter word per group (low half: fp16 step s).
+ *   ECHO_QUANT_DIRECTED  (default) z = fp16 rounded toward -inf from the
+ *        group minimum, s = fp16 rounded toward +inf from (max - z) / Q;
+ *        code = rint((v - z) / s); value = code * s + z. High half: fp16 z.
+ *   ECHO_QUANT_NEAREST   z and s = (max - min) / Q both rounded to nearest;
+ *        codes clamped to [0, Q]; value = code * s + z. High half: fp16 z.
+ *   ECHO_QUANT_INT_ZERO  integer zero point: the range is widened to include
+ *        0 (lo = min(min, 0), hi = max(max, 0)); s = fp16 rounded up from
+ *        (hi - lo) / Q; zp = clamp(rint(-lo / s), 0, Q);
+ *        code = clamp(rint(v / s) + zp, 0, Q); value = (code - zp) * s, so 0
+ *        is always exactly representable. High half: zp as an integer.
+ * (Divisions are binary32 multiplications by 1/s rounded to nearest; rint
+ * rounds half to even.)
+ */
+#define ECHO_QUANT_DIRECTED 0
+#define ECHO_QUANT_NEAREST 1
+#define ECHO_QUANT_INT_ZERO 2
+
+/*
+ * Select the quantizer form for the calls that use `st` from now on (the
+ * handle starts with ECHO_QUANT_DIRECTED; echo_allreduce_sim_noalloc always
+ * uses it). Both stages of a call use the same form. Host-only: enqueues
+ * nothing. ECHO_EINVAL for a NULL handle or an unknown form.
+ */
+ECHO_API int echo_set_quantizer(echo_state* st, int quantizer);
+
+/*
  * One all-reduce call over the P virtual ranks (phases 1-5 above).
  *   inputs     host array of P device pointers, each to n bf16 values
  *              (16-byte aligned): rank r's partial sum

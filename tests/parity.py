@@ -25,6 +25,7 @@ class Params:
     alpha_long: float = 0.05
     alpha_short: float = 0.5
     w: float = 0.5
+    quantizer: int = O.Q_DIRECTED   # the oracle's and the library's form numbers agree (0, 1, 2)
 
 
 def u16(t: torch.Tensor) -> np.ndarray:
@@ -39,9 +40,10 @@ class GpuEcho:
     """The CUDA path for one message shape: per-rank input/output buffers and
     the library handle (state and workspace owned by torch)."""
 
-    def __init__(self, P: int, n: int, group: int = 128, max_bits: int = 4, feedback: bool = True):
+    def __init__(self, P: int, n: int, group: int = 128, max_bits: int = 4, feedback: bool = True,
+                 quantizer: int = O.Q_DIRECTED):
         self.P, self.n, self.group = P, n, group
-        self.ar = E.EchoAllReduce(n, P, group, max_bits, feedback)
+        self.ar = E.EchoAllReduce(n, P, group, max_bits, feedback, quantizer=quantizer)
         self.G = int(self.ar.layout.groups)
         self.inputs = [torch.empty(n, dtype=torch.bfloat16, device="cuda") for _ in range(P)]
         self.outputs = [torch.empty(n, dtype=torch.bfloat16, device="cuda") for _ in range(P)]
@@ -129,3 +131,47 @@ def column_ranges(G: int, P: int, width: int) -> List[Tuple[int, int]]:
             continue
         out.append((s, jc))
     return out
+
+
+def seeded_state(P, n, seed, scale=0.05):
+    rng = np.random.default_rng(seed)
+    return ((rng.standard_normal((P, n)) * scale).astype(np.float32),
+            (rng.standard_normal((P, n)) * scale).astype(np.float32))
+
+
+def random_inputs(P, n, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(P, n, generator=g) * scale).to(torch.bfloat16)
+
+
+def check_full_call(P, n, p: Params, x, el0=None, es0=None, feedback=True, calls=1):
+    """Run `calls` consecutive calls on both sides (state carried) and compare
+    everything after each call."""
+    G = -(-n // p.group)
+    ld = G * p.group
+    gpu = GpuEcho(P, n, p.group, max(p.bits, 4), feedback, p.quantizer)
+    try:
+        gpu.set_inputs(x)
+        xb = padded(u16(x), ld)
+        if feedback:
+            el = padded(el0, ld) if el0 is not None else np.zeros((P, ld), np.float32)
+            es = padded(es0, ld) if es0 is not None else np.zeros((P, ld), np.float32)
+            gpu.set_state(el, es)
+        else:
+            el = es = None
+        for c in range(calls):
+            gpu.call(p)
+            orc = O.echo_allreduce(xb, n_total=n, group=p.group, bits=p.bits, e_long=el, e_short=es,
+                                   eta=p.eta, alpha_long=p.alpha_long, alpha_short=p.alpha_short, w=p.w,
+                                   quantizer=p.quantizer)
+            rc, flags = gpu.status()
+            assert flags == orc.flags
+            assert np.array_equal(gpu.outputs_u16(), orc.y[:, :n]), f"outputs differ (call {c})"
+            assert_payload_equal(gpu.payload(p.bits), orc, G, P, what=f"call {c}")
+            if feedback:
+                gl, gs = gpu.state()
+                assert_state_close(gl, el[:, :n], f"e_long call {c}")
+                assert_state_close(gs, es[:, :n], f"e_short call {c}")
+                assert np.array_equal(gl, el[:, :n]) and np.array_equal(gs, es[:, :n])  # expected bit-exact
+    finally:
+        gpu.close()

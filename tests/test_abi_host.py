@@ -94,6 +94,7 @@ def test_calls_reject_missing_handle(L):
     assert L.echo_phase_reduce(arr, arr, None, 4, 1.0, 0.05, 0.5, 0.5, None) == E.ECHO_EINVAL
     assert L.echo_phase_gather(arr, None, 4, None) == E.ECHO_EINVAL
     assert L.echo_get_status(None, None, None) == E.ECHO_EINVAL
+    assert L.echo_set_quantizer(None, E.ECHO_QUANT_NEAREST) == E.ECHO_EINVAL
     assert L.echo_free(None) == E.ECHO_OK
 
 

@@ -12,52 +12,11 @@ import torch
 import oracle as O
 import workloads as W
 import bit_error_compensated_group_b200 as E
-from parity import GpuEcho, Params, assert_payload_equal, assert_state_close, column_ranges, padded, u16
+from parity import (GpuEcho, Params, assert_payload_equal, assert_state_close, column_ranges, padded, u16,
+                    check_full_call as _check_full_call, random_inputs as _random_inputs,
+                    seeded_state as _seeded_state)
 
 pytestmark = pytest.mark.gpu
-
-
-def _seeded_state(P, n, seed, scale=0.05):
-    rng = np.random.default_rng(seed)
-    return ((rng.standard_normal((P, n)) * scale).astype(np.float32),
-            (rng.standard_normal((P, n)) * scale).astype(np.float32))
-
-
-def _random_inputs(P, n, seed, scale=1.0):
-    g = torch.Generator().manual_seed(seed)
-    return (torch.randn(P, n, generator=g) * scale).to(torch.bfloat16)
-
-
-def _check_full_call(P, n, p: Params, x, el0=None, es0=None, feedback=True, calls=1):
-    """Run `calls` consecutive calls on both sides (state carried) and compare
-    everything after each call."""
-    G = -(-n // p.group)
-    ld = G * p.group
-    gpu = GpuEcho(P, n, p.group, max(p.bits, 4), feedback)
-    try:
-        gpu.set_inputs(x)
-        xb = padded(u16(x), ld)
-        if feedback:
-            el = padded(el0, ld) if el0 is not None else np.zeros((P, ld), np.float32)
-            es = padded(es0, ld) if es0 is not None else np.zeros((P, ld), np.float32)
-            gpu.set_state(el, es)
-        else:
-            el = es = None
-        for c in range(calls):
-            gpu.call(p)
-            orc = O.echo_allreduce(xb, n_total=n, group=p.group, bits=p.bits, e_long=el, e_short=es,
-                                   eta=p.eta, alpha_long=p.alpha_long, alpha_short=p.alpha_short, w=p.w)
-            rc, flags = gpu.status()
-            assert flags == orc.flags
-            assert np.array_equal(gpu.outputs_u16(), orc.y[:, :n]), f"outputs differ (call {c})"
-            assert_payload_equal(gpu.payload(p.bits), orc, G, P, what=f"call {c}")
-            if feedback:
-                gl, gs = gpu.state()
-                assert_state_close(gl, el[:, :n], f"e_long call {c}")
-                assert_state_close(gs, es[:, :n], f"e_short call {c}")
-                assert np.array_equal(gl, el[:, :n]) and np.array_equal(gs, es[:, :n])  # expected bit-exact
-    finally:
-        gpu.close()
 
 
 def test_tiny_workload():

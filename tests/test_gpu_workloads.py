@@ -72,21 +72,21 @@ def _compare_sampled(ar, outputs, S: Sampled, orcs, bits, site):
             assert_state_close(es_v[:, c].cpu().numpy(), S.es[j0][:, :m], f"site {site} e_short")
 
 
-def _oracle_step(S: Sampled, x_by_range, bits):
+def _oracle_step(S: Sampled, x_by_range, bits, quantizer=O.Q_DIRECTED):
     w = S.w
     out = []
     for (j0, jc) in S.ranges:
         out.append(O.echo_allreduce(x_by_range[j0], n_total=w.n, group=w.group, bits=bits,
                                     e_long=S.el[j0], e_short=S.es[j0], eta=w.eta, alpha_long=w.alpha_long,
-                                    alpha_short=w.alpha_short, w=w.w, j0=j0, jc=jc))
+                                    alpha_short=w.alpha_short, w=w.w, j0=j0, jc=jc, quantizer=quantizer))
     return out
 
 
-def _run_chain(w: W.Workload, feedback: bool, width: int = 32):
+def run_chain(w: W.Workload, feedback: bool, width: int = 32, quantizer: int = O.Q_DIRECTED):
     """Full chain on the GPU, sampled chain on the oracle, compared per site.
     Returns the GPU's accumulated error S_T = sum_t (y_t - sum_r x_t,r)."""
     P, n = w.P, w.n
-    ar = E.EchoAllReduce(n, P, w.group, 8 if w.int8_sites else 4, feedback)
+    ar = E.EchoAllReduce(n, P, w.group, 8 if w.int8_sites else 4, feedback, quantizer=quantizer)
     S = Sampled(w, width, feedback)
     x_cpu = W.inputs(w, 0)
     inputs = [x_cpu[r].cuda() for r in range(P)]
@@ -97,7 +97,7 @@ def _run_chain(w: W.Workload, feedback: bool, width: int = 32):
         for t in range(w.sites):
             bits = w.bits_at(t)
             ar(inputs, outputs, bits, w.eta, w.alpha_long, w.alpha_short, w.w)
-            orcs = _oracle_step(S, x_orc, bits)
+            orcs = _oracle_step(S, x_orc, bits, quantizer)
             rc, flags = ar.status()
             assert rc == E.ECHO_OK and all(o.flags == 0 for o in orcs)
             _compare_sampled(ar, outputs, S, orcs, bits, t)
@@ -122,30 +122,49 @@ def _run_chain(w: W.Workload, feedback: bool, width: int = 32):
 
 def test_chain_56_sites_p8():
     w = W.CHAIN56
-    with_fb = _run_chain(w, True)
-    without = _run_chain(w, False)
+    with_fb = run_chain(w, True)
+    without = run_chain(w, False)
     rms_fb = float(np.sqrt(np.mean(with_fb ** 2)))
     rms_no = float(np.sqrt(np.mean(without ** 2)))
     # the explainer's theory section: bounded with feedback, growing without
     assert rms_no > 2.5 * rms_fb, (rms_no, rms_fb)
 
 
+def test_chain_ablation_quantizer_forms():
+    """The ablation of the quantizer form on the 56-site chain (P = 8): each
+    form, with and without feedback, run in full on the GPU and checked site
+    by site against the oracle on sampled columns. Reported: RMS of the
+    accumulated error S_T over the last site, in units of q, the RMS per-site
+    error of the default form without feedback. Feedback keeps S_T bounded
+    for every form (the explainer's theory section)."""
+    w = W.CHAIN56
+    res = {}
+    for q in (O.Q_DIRECTED, O.Q_NEAREST, O.Q_INT_ZERO):
+        for fb in (True, False):
+            res[(q, fb)] = float(np.sqrt(np.mean(run_chain(w, fb, width=16, quantizer=q) ** 2)))
+    names = {O.Q_DIRECTED: "directed", O.Q_NEAREST: "nearest", O.Q_INT_ZERO: "int_zero"}
+    print("\nablation RMS(S_56):", {f"{names[q]}/{'fb' if fb else 'nofb'}": round(v, 5) for (q, fb), v in res.items()})
+    for q in names:
+        assert res[(q, False)] > 2.5 * res[(q, True)], (names[q], res[(q, False)], res[(q, True)])
+
+
 def test_chain_48_sites_p4_early_int8():
     w = W.CHAIN48_MIXED
-    _run_chain(w, True)
+    run_chain(w, True)
 
 
-def test_headline_1gb_sampled_columns():
-    """P = 8, 1 GB per rank, two calls with the state carried, in the exact
-    launch sequence the benchmark times (quantize, then the owners' reduce
-    writing the outputs)."""
+@pytest.mark.parametrize("feedback", [True, False])
+def test_headline_1gb_sampled_columns(feedback):
+    """P = 8, 1 GB per rank, two calls (state carried when there is one), in
+    the exact launch sequence the benchmark times (quantize, then the owners'
+    reduce writing the outputs)."""
     w = W.HEADLINE
     P, n = w.P, w.n
     free, _ = torch.cuda.mem_get_info()
     if free < 60e9:
         pytest.skip("needs ~55 GB of free device memory")
-    ar = E.EchoAllReduce(n, P, w.group, 4, True)
-    S = Sampled(w, 256)
+    ar = E.EchoAllReduce(n, P, w.group, 4, feedback)
+    S = Sampled(w, 256, feedback)
     try:
         inputs = [W.rank_input(w, r, 0, "cuda") for r in range(P)]
         outputs = [torch.empty_like(t) for t in inputs]
