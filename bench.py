@@ -320,6 +320,27 @@ def run_gpu(args):
                    "roofline_frac": algorithmic_bytes(P, n, group, bits, feedback=False)["total"] / (nf_ms * 1e-3)
                    / 1e9 / _peak_hbm()[0]}
 
+    # the other quantizer forms (the ablations' variants) on the same call,
+    # feedback on: the nearest and integer-zero forms clamp each code
+    forms = None
+    if not args.no_variants and _FEEDBACK:
+        forms = {}
+        q_steps = max(3, min(args.steps, 10))
+        for name, q in (("nearest", E.ECHO_QUANT_NEAREST), ("int_zero", E.ECHO_QUANT_INT_ZERO)):
+            E.echo_set_quantizer(h, q)
+            for _ in range(args.warmup):
+                step()
+            barrier()
+            q_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(q_steps)]
+            for i in range(q_steps):
+                step(q_evs[i])
+            barrier()
+            q_ms = max_over_ranks(q_evs[0][0].elapsed_time(q_evs[-1][2]), world, dev) / q_steps
+            forms[name] = {"ms_per_step": q_ms, "steps": q_steps,
+                           "roofline_frac": algorithmic_bytes(P, n, group, bits)["total"] / (q_ms * 1e-3)
+                           / 1e9 / _peak_hbm()[0]}
+        E.echo_set_quantizer(h, E.ECHO_QUANT_DIRECTED)
+
     # end to end through the public call with host buffers: pinned inputs
     # copied in, the call, the reduced result copied out, every step
     e2e = None
@@ -376,6 +397,8 @@ def run_gpu(args):
         if variant is not None:
             line["no_feedback"] = variant
             line["compensation_ms"] = ms - variant["ms_per_step"]
+        if forms is not None:
+            line["quantizer_forms"] = forms
         if world == 1 and not args.no_cpu_baseline:
             gbs, dt, er = cpu_sample_rate(CPU_BASELINE_COLS)
             line["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
@@ -386,6 +409,77 @@ def run_gpu(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def run_ablation(args):
+    """Accuracy ablations on the synthetic chains, through the public API on
+    one GPU (the oracle's agreement with these runs is the GPU test suite's
+    job). Each entry: RMS and max over elements of the accumulated error
+    S_T = sum_t (y_t - sum_r x_t,r) after the last site, in units of q and
+    q_max, the RMS and max of the per-site error of the default form at the
+    same bits without feedback (the quantizer's own error scale)."""
+    import torch
+    import workloads as W
+    import bit_error_compensated_group_b200 as E
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+
+    noise = {}   # per chain: every site's noise, drawn once and kept on the device
+
+    def site_noise(w, t):
+        if w.name not in noise:
+            noise[w.name] = [W.chain_noise(w, k + 1).to(dev) for k in range(w.sites)]
+        return noise[w.name][t]
+
+    def chain(w, feedback=True, quantizer=E.ECHO_QUANT_DIRECTED, group=None, int8_sites=None, wt=None):
+        group = group or w.group
+        int8 = w.int8_sites if int8_sites is None else int8_sites
+        ar = E.EchoAllReduce(w.n, w.P, group, 8 if int8 else 4, feedback, device=dev, quantizer=quantizer)
+        x = W.inputs(w, 0, "cpu")
+        inputs = [x[r].to(dev) for r in range(w.P)]
+        outputs = [torch.empty_like(t) for t in inputs]
+        acc = torch.zeros(w.n, dtype=torch.float64, device=dev)
+        site_rms, site_max = [], []
+        try:
+            for t in range(w.sites):
+                bits = 8 if t < int8 else w.bits
+                ar(inputs, outputs, bits, w.eta, w.alpha_long, w.alpha_short, w.w if wt is None else wt)
+                err = outputs[0].double() - torch.stack([i.double() for i in inputs]).sum(0)
+                acc += err
+                site_rms.append(float(err.pow(2).mean().sqrt()))
+                site_max.append(float(err.abs().max()))
+                # the chain rule of workloads.chain_next_input, evaluated on the device
+                xn = (outputs[0].float() * w.decay / w.P + site_noise(w, t)).to(torch.bfloat16)
+                for r in range(w.P):
+                    inputs[r].copy_(xn[r])
+            rc, _ = ar.status()
+            assert rc == E.ECHO_OK, rc
+        finally:
+            ar.close()
+        return float(acc.pow(2).mean().sqrt()), float(acc.abs().max()), site_rms, site_max
+
+    out = {}
+    for w, key in ((W.CHAIN56, "chain56_p8_int4"), (W.CHAIN48_MIXED, "chain48_p4")):
+        _, _, q_rms, q_max = chain(w, feedback=False, int8_sites=0)
+        q, qm = sum(q_rms) / len(q_rms), sum(q_max) / len(q_max)
+        runs = {}
+        if w is W.CHAIN56:
+            for name, qf in (("directed", E.ECHO_QUANT_DIRECTED), ("nearest", E.ECHO_QUANT_NEAREST),
+                             ("int_zero", E.ECHO_QUANT_INT_ZERO)):
+                runs[f"form={name}"] = chain(w, quantizer=qf)
+                runs[f"form={name},no_feedback"] = chain(w, feedback=False, quantizer=qf)
+            for g in (64, 256):
+                runs[f"group={g}"] = chain(w, group=g)
+            runs["ema=long_only(w=0)"] = chain(w, wt=0.0)
+            runs["ema=short_only(w=1)"] = chain(w, wt=1.0)
+        else:
+            for k8, name in ((0, "none"), (12, "first_quarter(12)"), (24, "first_half(24)"), (48, "all")):
+                runs[f"int8_sites={name}"] = chain(w, int8_sites=k8)
+                runs[f"int8_sites={name},no_feedback"] = chain(w, feedback=False, int8_sites=k8)
+        out[key] = {"q": q, "q_max": qm,
+                    "runs": {k: {"rms_S_T/q": v[0] / q, "max_S_T/q_max": v[1] / qm} for k, v in runs.items()}}
+    print(json.dumps({"ablation": out, "data": "synthetic chains (workloads.CHAIN56, workloads.CHAIN48_MIXED)"}),
+          flush=True)
 
 
 def main():
@@ -399,6 +493,8 @@ def main():
     ap.add_argument("--no-variants", action="store_true", help="skip the no-feedback timing")
     ap.add_argument("--feedback", choices=["on", "off"], default="on",
                     help="off: time the call without EMA state as the main step (profiling)")
+    ap.add_argument("--ablation", action="store_true",
+                    help="print the accuracy ablations on the synthetic chains instead of timing")
     ap.add_argument("--tokens", type=int, default=None,
                     help="tokens per rank (default 131072, the 1 GB message); smaller values are for profiling")
     args = ap.parse_args()
@@ -407,6 +503,8 @@ def main():
     _FEEDBACK = args.feedback == "on"
     if args.impl == "reference":
         run_reference(args)
+    elif args.ablation:
+        run_ablation(args)
     else:
         run_gpu(args)
 
