@@ -3,8 +3,9 @@ virtual ranks on one B200, on the 1 GB-per-rank message (131072 x 4096 bf16,
 Student-t nu=3 values scaled to unit variance, groups of 128, INT4, feedback
 on: alpha_long 0.05, alpha_short 0.5, w 0.5, eta 1).
 
-One step = one full call (the three kernels: non-owner quantize with fused
-feedback, owner reduce/requantize, gather dequantize), inputs resident in HBM.
+One step = one full call (two kernels: the non-owners' quantize with fused
+feedback and EMA update; the owners' reduce/requantize, which also decodes the
+gathered result into all P outputs), inputs resident in HBM.
 Metric: GB/s of bf16 input (all P ranks' inputs) per second.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
@@ -98,49 +99,101 @@ def _measured_traffic():
 
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and throttle reasons sampled during the timed region: NVML read
+    every 20 ms from a thread (falls back to `nvidia-smi -lms 200`). Reads
+    only; no setting of the GPU is touched."""
+    PERIOD_S = 0.02
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    SMI_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index):
+        import threading
         import torch
+        self.rows = []          # (sm_mhz, set of reason names)
+        self.max_mhz = None
         self.proc = None
-        self.path = None
+        self.thread = None
+        self.kind = None
         try:
             uuid = str(torch.cuda.get_device_properties(device_index).uuid)
-            sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+        except Exception:
+            return
+        self.uuid = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+        try:
+            import pynvml as N
+            N.nvmlInit()
+            self.N = N
+            self.h = N.nvmlDeviceGetHandleByUUID(self.uuid)
+            self.max_mhz = float(N.nvmlDeviceGetMaxClockInfo(self.h, N.NVML_CLOCK_SM))
+            self.bits = {"hw_slowdown": N.nvmlClocksEventReasonHwSlowdown,
+                         "hw_thermal_slowdown": N.nvmlClocksEventReasonHwThermalSlowdown,
+                         "sw_thermal_slowdown": N.nvmlClocksEventReasonSwThermalSlowdown,
+                         "sw_power_cap": N.nvmlClocksEventReasonSwPowerCap}
+            self.done = threading.Event()
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.kind = "nvml"
+            self.thread.start()
+        except Exception:
+            self.thread = None
+            self._start_smi()
+
+    def _poll(self):
+        N = self.N
+        while not self.done.is_set():
+            try:
+                mhz = float(N.nvmlDeviceGetClockInfo(self.h, N.NVML_CLOCK_SM))
+                r = N.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.rows.append((mhz, {k for k, b in self.bits.items() if r & b}))
+            except Exception:
+                pass
+            self.done.wait(self.PERIOD_S)
+
+    def _start_smi(self):
+        try:
             self.path = f"/tmp/echo_clocks_{os.getpid()}.csv"
             self.fh = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", sel, f"--query-gpu={self.FIELDS}",
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.uuid, f"--query-gpu={self.SMI_FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "200"],
                                          stdout=self.fh, stderr=subprocess.DEVNULL)
+            self.kind = "nvidia-smi"
         except Exception:
             self.proc = None
 
-    def stop(self):
-        if self.proc is None:
-            return None
+    def _stop_smi(self):
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
         self.fh.close()
-        rows = []
         with open(self.path) as f:
             for line in f:
                 parts = [p.strip() for p in line.split(",")]
-                if len(parts) == 9:
-                    rows.append(parts)
+                if len(parts) != 9 or not parts[1].replace(".", "").isdigit():
+                    continue
+                if parts[2].replace(".", "").isdigit():
+                    self.max_mhz = float(parts[2])
+                self.rows.append((float(parts[1]),
+                                  {self.REASONS[i] for i in range(4) if parts[5 + i].lower() == "active"}))
         os.unlink(self.path)
-        if not rows:
+
+    def stop(self):
+        if self.thread is not None:
+            self.done.set()
+            self.thread.join(timeout=5)
+            try:
+                self.N.nvmlShutdown()
+            except Exception:
+                pass
+        elif self.proc is not None:
+            self._stop_smi()
+        if not self.rows:
             return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
-                "reasons": reasons, "samples": len(rows)}
+        return {"sm_mhz": statistics.median(r[0] for r in self.rows), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(set().union(*(r[1] for r in self.rows))), "samples": len(self.rows),
+                "sampler": f"{self.kind}, every {int(self.PERIOD_S * 1000) if self.kind == 'nvml' else 200} ms"}
 
 
 def max_over_ranks(value: float, world: int, device) -> float:
@@ -341,8 +394,47 @@ def run_gpu(args):
                            / 1e9 / _peak_hbm()[0]}
         E.echo_set_quantizer(h, E.ECHO_QUANT_DIRECTED)
 
-    # end to end through the public call with host buffers: pinned inputs
-    # copied in, the call, the reduced result copied out, every step
+    # the early-site 8-bit mode on the same message, feedback on (one code
+    # per byte: 22.06 algorithmic bytes per element-rank instead of 21.06)
+    int8 = None
+    if not args.no_variants and _FEEDBACK:
+        a8 = E.EchoAllReduce(n, P, group, 8, feedback=True, device=dev)
+        i8_steps = max(3, min(args.steps, 10))
+
+        def i8_step(ev=None):
+            if ev is not None:
+                ev[0].record(stream)
+            E.echo_phase_quantize(inputs, a8.handle, 8, *fb, stream=stream)
+            if ev is not None:
+                ev[1].record(stream)
+            E.echo_phase_reduce(inputs, outputs, a8.handle, 8, *fb, stream=stream)
+            if ev is not None:
+                ev[2].record(stream)
+
+        for _ in range(args.warmup):
+            i8_step()
+        barrier()
+        i8_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(i8_steps)]
+        for i in range(i8_steps):
+            i8_step(i8_evs[i])
+        barrier()
+        i8_ms = max_over_ranks(i8_evs[0][0].elapsed_time(i8_evs[-1][2]), world, dev) / i8_steps
+        i8_q = sum(e[0].elapsed_time(e[1]) for e in i8_evs) / i8_steps
+        i8_r = sum(e[1].elapsed_time(e[2]) for e in i8_evs) / i8_steps
+        ab8 = algorithmic_bytes(P, n, group, 8)
+        a8_rc, a8_flags = a8.status()
+        a8.close()
+        del a8
+        torch.cuda.empty_cache()
+        int8 = {"ms_per_step": i8_ms, "steps": i8_steps, "phases_ms": {"quantize": i8_q, "reduce_gather": i8_r},
+                "value": weak_scaling_gbs(world, P * n * 2, i8_ms),
+                "roofline_frac": ab8["total"] / (i8_ms * 1e-3) / 1e9 / _peak_hbm()[0],
+                "quantize_frac": ab8["quantize"] / (i8_q * 1e-3) / 1e9 / _peak_hbm()[0],
+                "status": a8_rc, "flags": a8_flags}
+
+    # end to end through the public host-buffer call: every step, pinned
+    # inputs copied in and the reduced result copied out, chunk by chunk on
+    # two copy streams overlapping the kernels (echo_allreduce_sim_host)
     e2e = None
     if not args.no_e2e:
         e2e_steps = max(1, min(args.steps, 4))
@@ -350,12 +442,11 @@ def run_gpu(args):
         for r in range(P):
             host_in[r].copy_(inputs[r])
         host_out = torch.empty(n, dtype=torch.bfloat16, pin_memory=True)
+        cin, cout = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
         def e2e_step():
-            for r in range(P):
-                inputs[r].copy_(host_in[r], non_blocking=True)
-            E.echo_allreduce_sim(inputs, outputs, h, n, P, bits, group, *fb, stream=stream)
-            host_out.copy_(outputs[0], non_blocking=True)
+            E.echo_allreduce_sim_host(host_in, host_out, inputs, outputs, h, n, P, bits, group, *fb,
+                                      args.e2e_chunk, stream=stream, copy_in=cin, copy_out=cout)
 
         e2e_step()
         barrier()
@@ -366,9 +457,12 @@ def run_gpu(args):
         b.record(stream)
         barrier()
         e2e_ms = max_over_ranks(a.elapsed_time(b), world, dev) / e2e_steps
+        G = -(-n // group)
+        chunk = args.e2e_chunk if args.e2e_chunk > 0 else -(-G // 16)
         e2e = {"value": weak_scaling_gbs(world, P * n * 2, e2e_ms), "unit": "GB/s",
                "h2d_bytes_per_step": P * n * 2, "d2h_bytes_per_step": n * 2,
-               "ms_per_step": e2e_ms, "steps": e2e_steps}
+               "ms_per_step": e2e_ms, "steps": e2e_steps, "call": "echo_allreduce_sim_host",
+               "chunks": -(-G // chunk)}
         del host_in, host_out
 
     if rank == 0:
@@ -399,6 +493,8 @@ def run_gpu(args):
             line["compensation_ms"] = ms - variant["ms_per_step"]
         if forms is not None:
             line["quantizer_forms"] = forms
+        if int8 is not None:
+            line["int8"] = int8
         if world == 1 and not args.no_cpu_baseline:
             gbs, dt, er = cpu_sample_rate(CPU_BASELINE_COLS)
             line["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
@@ -490,7 +586,9 @@ def main():
     ap.add_argument("--impl", default="echo", choices=["echo", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-variants", action="store_true", help="skip the no-feedback timing")
+    ap.add_argument("--e2e-chunk", type=int, default=0,
+                    help="group columns per chunk of the host-buffer call (0: the library's default, G/16)")
+    ap.add_argument("--no-variants", action="store_true", help="skip the no-feedback, quantizer-form and 8-bit timings")
     ap.add_argument("--feedback", choices=["on", "off"], default="on",
                     help="off: time the call without EMA state as the main step (profiling)")
     ap.add_argument("--ablation", action="store_true",

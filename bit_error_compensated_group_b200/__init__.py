@@ -8,7 +8,8 @@ and raises if the library is missing.
 from .echo import (  # noqa: F401
     ECHO_EINVAL, ECHO_ECUDA, ECHO_ERANGE, ECHO_ETIMEOUT, ECHO_FLAG_RANGE, ECHO_FLAG_TIMEOUT, ECHO_MAX_RANKS, ECHO_OK,
     ECHO_QUANT_DIRECTED, ECHO_QUANT_INT_ZERO, ECHO_QUANT_NEAREST,
-    EchoAllReduce, EchoError, EchoLayout, echo_allreduce_sim, echo_check_watchdog, echo_free, echo_get_status, echo_init_state,
+    EchoAllReduce, EchoError, EchoLayout, echo_allreduce_sim, echo_allreduce_sim_host, echo_allreduce_sim_range,
+    echo_check_watchdog, echo_free, echo_get_status, echo_init_state,
     echo_phase_gather, echo_phase_quantize, echo_phase_reduce, echo_query_layout, echo_set_quantizer, echo_state_bytes,
     echo_status_string, echo_workspace_bytes, lib,
 )

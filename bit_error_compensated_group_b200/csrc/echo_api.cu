@@ -25,6 +25,10 @@ struct echo_state {
     int device;
     int sm_count;
     int quantizer;         // ECHO_QUANT_*; ECHO_QUANT_DIRECTED unless set
+    // echo_allreduce_sim_host: ordering events between the caller's stream and
+    // the two copy streams, created on first use, destroyed by echo_free
+    cudaEvent_t ev[3];
+    bool have_events;
 };
 
 namespace {
@@ -94,7 +98,8 @@ enum class Stage { Quantize, Reduce, Gather };
 // An upper bound on the tiles a pipelined launch walks: the runs (2 per rank
 // for quantize, 1 per owner for reduce) cut into tiles of `tile_groups`.
 int64_t tile_bound(Stage stage, const echo_dev::Args& a, int tile_groups) {
-    const int64_t groups = stage == Stage::Quantize ? (int64_t)(a.P - 1) * a.G : a.G;
+    const int64_t cols = a.c1 - a.c0;   // the call's group-column window
+    const int64_t groups = stage == Stage::Quantize ? (int64_t)(a.P - 1) * cols : cols;
     const int64_t runs = stage == Stage::Quantize ? 2 * (int64_t)a.P : a.P;
     return groups / tile_groups + runs + 1;
 }
@@ -177,6 +182,15 @@ int launch(Stage stage, int bits, const echo_dev::Args& a, const echo_state* st,
     return ECHO_EINVAL;
 }
 
+// The call's group columns [c0, c1) as the kernels take them: the full
+// groups of the window, and whether it holds the partial last group.
+void set_window(echo_dev::Args* a, const echo_state* st, int64_t c0, int64_t c1) {
+    const int64_t full = st->n / st->group;
+    a->c0 = c0;
+    a->c1 = c1 < full ? c1 : full;
+    a->tail = (full < st->G && c1 == st->G) ? 1 : 0;
+}
+
 bool valid_feedback(float eta, float aL, float aS, float w) {
     return std::isfinite(eta) && in_unit(aL) && in_unit(aS) && in_unit(w);
 }
@@ -205,6 +219,7 @@ bool make_args(const echo_state* st, int bits, const void* const* inputs, void* 
     a->flags = reinterpret_cast<uint32_t*>(st->workspace + L.flags_offset);
     a->n = st->n;
     a->G = st->G;
+    set_window(a, st, 0, st->G);
     a->S = st->S;
     a->P = st->P;
     a->eta = eta;
@@ -273,6 +288,7 @@ int echo_init_state(echo_state** out, int64_t n, int P, int group, int max_bits,
     st->device = dev;
     st->sm_count = sms;
     st->quantizer = ECHO_QUANT_DIRECTED;
+    st->have_events = false;
     *out = st;
     return ECHO_OK;
 }
@@ -334,6 +350,92 @@ int echo_allreduce_sim(const void* const* inputs, void* const* outputs, echo_sta
     return launch(Stage::Reduce, bits, a, st, s);
 }
 
+int echo_allreduce_sim_range(const void* const* inputs, void* const* outputs, echo_state* st, int64_t n, int P,
+                             int bits, int group, float eta, float alpha_long, float alpha_short, float w,
+                             int64_t group_begin, int64_t group_end, echo_stream_t stream) {
+    if (!st || !inputs || !outputs) return ECHO_EINVAL;
+    if (n != st->n || P != st->P || group != st->group) return ECHO_EINVAL;
+    if (!valid_bits(bits) || bits > st->max_bits) return ECHO_EINVAL;
+    if (!valid_feedback(eta, alpha_long, alpha_short, w)) return ECHO_EINVAL;
+    if (group_begin < 0 || group_end < group_begin || group_end > st->G) return ECHO_EINVAL;
+    echo_dev::Args a;
+    if (!make_args(st, bits, inputs, outputs, eta, alpha_long, alpha_short, w, &a)) return ECHO_EINVAL;
+    if (group_begin == group_end) return ECHO_OK;
+    if (int rc = set_device(st)) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    set_window(&a, st, group_begin, group_end);
+    a.write_outputs = 1;
+    if (P >= 2) {
+        if (int rc = launch(Stage::Quantize, bits, a, st, s)) return rc;
+    }
+    return launch(Stage::Reduce, bits, a, st, s);
+}
+
+int echo_allreduce_sim_host(const void* const* host_inputs, void* host_output, void* const* inputs,
+                            void* const* outputs, echo_state* st, int64_t n, int P, int bits, int group, float eta,
+                            float alpha_long, float alpha_short, float w, int64_t chunk_groups,
+                            echo_stream_t stream, echo_stream_t copy_in, echo_stream_t copy_out) {
+    if (!st || !host_inputs || !inputs || !outputs) return ECHO_EINVAL;
+    if (n != st->n || P != st->P || group != st->group) return ECHO_EINVAL;
+    if (!valid_bits(bits) || bits > st->max_bits) return ECHO_EINVAL;
+    if (!valid_feedback(eta, alpha_long, alpha_short, w)) return ECHO_EINVAL;
+    if (chunk_groups < 0) return ECHO_EINVAL;
+    for (int r = 0; r < P; ++r)
+        if (!host_inputs[r]) return ECHO_EINVAL;
+    echo_dev::Args probe;
+    if (!make_args(st, bits, inputs, outputs, eta, alpha_long, alpha_short, w, &probe)) return ECHO_EINVAL;
+    if (int rc = set_device(st)) return rc;
+    if (!st->have_events) {
+        for (int i = 0; i < 3; ++i) {
+            if (cudaEventCreateWithFlags(&st->ev[i], cudaEventDisableTiming) != cudaSuccess) {
+                for (int k = 0; k < i; ++k) cudaEventDestroy(st->ev[k]);
+                return ECHO_ECUDA;
+            }
+        }
+        st->have_events = true;
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaStream_t cin = reinterpret_cast<cudaStream_t>(copy_in);
+    cudaStream_t cout = reinterpret_cast<cudaStream_t>(copy_out);
+    cudaEvent_t ev_start = st->ev[0], ev_in = st->ev[1], ev_done = st->ev[2];
+    const int64_t G = st->G;
+    const int64_t chunk = chunk_groups > 0 ? chunk_groups : (G + 15) / 16;
+    // the copy streams start after everything already on `stream`
+    if (cudaEventRecord(ev_start, s) != cudaSuccess) return ECHO_ECUDA;
+    if (cudaStreamWaitEvent(cin, ev_start, 0) != cudaSuccess) return ECHO_ECUDA;
+    if (host_output && cudaStreamWaitEvent(cout, ev_start, 0) != cudaSuccess) return ECHO_ECUDA;
+    for (int64_t c0 = 0; c0 < G; c0 += chunk) {
+        const int64_t c1 = c0 + chunk < G ? c0 + chunk : G;
+        const int64_t e0 = c0 * group, e1 = c1 * group < n ? c1 * group : n;
+        const size_t bytes = (size_t)(e1 - e0) * 2;
+        for (int r = 0; r < P; ++r) {
+            if (cudaMemcpyAsync(static_cast<uint16_t*>(inputs[r]) + e0,
+                                static_cast<const uint16_t*>(host_inputs[r]) + e0, bytes, cudaMemcpyHostToDevice,
+                                cin) != cudaSuccess)
+                return ECHO_ECUDA;
+        }
+        // a wait binds to the event's latest record, so one event serves every chunk
+        if (cudaEventRecord(ev_in, cin) != cudaSuccess) return ECHO_ECUDA;
+        if (cudaStreamWaitEvent(s, ev_in, 0) != cudaSuccess) return ECHO_ECUDA;
+        if (int rc = echo_allreduce_sim_range(inputs, outputs, st, n, P, bits, group, eta, alpha_long, alpha_short,
+                                              w, c0, c1, stream))
+            return rc;
+        if (host_output) {
+            if (cudaEventRecord(ev_done, s) != cudaSuccess) return ECHO_ECUDA;
+            if (cudaStreamWaitEvent(cout, ev_done, 0) != cudaSuccess) return ECHO_ECUDA;
+            if (cudaMemcpyAsync(static_cast<uint16_t*>(host_output) + e0, static_cast<const uint16_t*>(outputs[0]) + e0,
+                                bytes, cudaMemcpyDeviceToHost, cout) != cudaSuccess)
+                return ECHO_ECUDA;
+        }
+    }
+    // `stream` continues once the last result has reached the host
+    if (host_output) {
+        if (cudaEventRecord(ev_done, cout) != cudaSuccess) return ECHO_ECUDA;
+        if (cudaStreamWaitEvent(s, ev_done, 0) != cudaSuccess) return ECHO_ECUDA;
+    }
+    return ECHO_OK;
+}
+
 int echo_check_watchdog(echo_state* st, uint32_t limit_us, echo_stream_t stream) {
     if (!st || limit_us < 1 || limit_us > 10000000u) return ECHO_EINVAL;
     if (int rc = set_device(st)) return rc;
@@ -356,6 +458,13 @@ int echo_get_status(echo_state* st, echo_stream_t stream, uint32_t* device_flags
 }
 
 int echo_free(echo_state* st) {
+    if (st && st->have_events) {
+        int cur = -1;
+        const bool switched = cudaGetDevice(&cur) == cudaSuccess && cur != st->device &&
+                              cudaSetDevice(st->device) == cudaSuccess;
+        for (cudaEvent_t e : st->ev) cudaEventDestroy(e);
+        if (switched) cudaSetDevice(cur);
+    }
     delete st;
     return ECHO_OK;
 }
@@ -423,6 +532,7 @@ int echo_allreduce_sim_noalloc(const void* const* inputs, void* const* outputs, 
     st.device = dev;
     st.sm_count = sms;
     st.quantizer = ECHO_QUANT_DIRECTED;
+    st.have_events = false;
     echo_dev::Args a;
     if (!make_args(&st, bits, inputs, outputs, eta, alpha_long, alpha_short, w, &a)) return ECHO_EINVAL;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

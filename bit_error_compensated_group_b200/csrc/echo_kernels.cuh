@@ -58,6 +58,10 @@ struct Args {
     float a_long, keep_long, a_short, keep_short;
     float one;   // 1.0f, passed at run time (see add_after_mul2 in echo_pipeline.cuh)
     int write_outputs;   // reduce: also decode into all P outputs (phase 4 in the owner's pass)
+    // the call's group columns: full groups [c0, c1) (c1 <= n / group; the
+    // whole message: 0, n / group) and, when tail != 0, the partial last group
+    long long c0, c1;
+    int tail;
 };
 
 // ------------------------------------------------------------------ helpers

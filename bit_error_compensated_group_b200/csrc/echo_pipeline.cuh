@@ -97,9 +97,10 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 
 // ------------------------------------------------------------ tile walk
 
-// A run is a contiguous range of full groups [j0, j1) of one rank. The tile
-// sequence of a kernel is the concatenation of its runs cut into tiles of at
-// most T groups. The cursor walks it monotonically (tile indices only grow).
+// A run is a contiguous range of full groups [j0, j1) of one rank, clipped to
+// the call's group-column window [c0, c1). The tile sequence of a kernel is
+// the concatenation of its runs cut into tiles of at most T groups. The
+// cursor walks it monotonically (tile indices only grow).
 struct Tile {
     int rank;
     long long j0;
@@ -109,44 +110,45 @@ struct Tile {
 template <int GROUP, int M = 1>
 struct RunWalker {
     static constexpr int T = M * kTileElems / GROUP;   // groups per tile (M sub-tiles)
-    // kind 0: non-owned runs of every rank (quantize); kind 1: owned runs (reduce)
+    // kind 0: non-owned runs of every rank (quantize); kind 1: owned runs (reduce).
+    // G, P and the window are read from the kernel arguments when needed
+    // rather than held in registers.
     int kind;
-    long long G, G_full;
-    int P;
     int run;            // current run index
     long long base;     // first tile index of the current run
     long long run_j0, run_len;
 
-    __device__ __forceinline__ void load_run() {
-        run_j0 = 0;
-        run_len = 0;
-        if (kind == 0) {
-            const int r = run >> 1;
-            const long long lo = (long long)r * G / P, hi = (long long)(r + 1) * G / P;
-            if ((run & 1) == 0) {
-                run_j0 = 0;
-                run_len = min(lo, G_full);
-            } else {
-                run_j0 = hi;
-                run_len = max(0LL, G_full - hi);
-            }
+    // run `run` before clipping: kind 0, rank r = run / 2: [0, lo) for even
+    // runs, [hi, G) for odd; kind 1: [lo, hi) of rank `run`, where [lo, hi)
+    // is that rank's owned segment. Clipped to the call's full-group window
+    // [c0, c1) (a partial last group takes the kernels' scalar path).
+    __device__ __forceinline__ void load_run(const Args& a) {
+        const int r = kind == 0 ? run >> 1 : run;
+        const long long lo = (long long)r * a.G / a.P, hi = (long long)(r + 1) * a.G / a.P;
+        long long b, e;
+        if (kind == 1) {
+            b = lo;
+            e = hi;
+        } else if ((run & 1) == 0) {
+            b = 0;
+            e = lo;
         } else {
-            const long long lo = (long long)run * G / P, hi = (long long)(run + 1) * G / P;
-            run_j0 = lo;
-            run_len = max(0LL, min(hi, G_full) - lo);
+            b = hi;
+            e = a.G;
         }
+        b = max(b, a.c0);
+        e = min(e, a.c1);
+        run_j0 = b;
+        run_len = max(0LL, e - b);
     }
-    __device__ __forceinline__ int runs() const { return kind == 0 ? 2 * P : P; }
+    __device__ __forceinline__ int runs(const Args& a) const { return kind == 0 ? 2 * a.P : a.P; }
     __device__ __forceinline__ int rank_of_run() const { return kind == 0 ? (run >> 1) : run; }
 
-    __device__ __forceinline__ RunWalker(int kind_, long long G_, long long G_full_, int P_)
-        : kind(kind_), G(G_), G_full(G_full_), P(P_), run(0), base(0) {
-        load_run();
-    }
+    __device__ __forceinline__ RunWalker(int kind_, const Args& a) : kind(kind_), run(0), base(0) { load_run(a); }
 
     // Tile k (k never decreases between calls); false when past the end.
-    __device__ __forceinline__ bool locate(long long k, Tile* t) {
-        while (run < runs()) {
+    __device__ __forceinline__ bool locate(long long k, Tile* t, const Args& a) {
+        while (run < runs(a)) {
             const long long nt = (run_len + T - 1) / T;
             if (k < base + nt) {
                 const long long off = (k - base) * T;
@@ -157,7 +159,7 @@ struct RunWalker {
             }
             base += nt;
             ++run;
-            if (run < runs()) load_run();
+            if (run < runs(a)) load_run(a);
         }
         return false;
     }
@@ -204,7 +206,7 @@ __device__ __forceinline__ void produce(const Args& a, const PipeShared& p, RunW
                                         bool with_state) {
     long long issued = 0;
     Tile t;
-    for (long long k = blockIdx.x; walker.locate(k, &t); k += gridDim.x, ++issued) {
+    for (long long k = blockIdx.x; walker.locate(k, &t, a); k += gridDim.x, ++issued) {
         const int s = (int)(issued % kStages);
         const uint32_t use = (uint32_t)(issued / kStages);
         if (issued >= kStages && !mbar_wait(&p.empty[s], (use & 1u) ^ 1u, kWaitLimitNs, p.abort)) {
@@ -650,8 +652,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
     const PipeShared p = pipe_shared(smem);
     pipe_init(p);
     const int warp = threadIdx.x >> 5;
-    const long long G_full = a.n / GROUP;
-    RunWalker<GROUP, M> walker(0, a.G, G_full, a.P);
+    RunWalker<GROUP, M> walker(0, a);
     if (warp == kConsumerWarps) {
         if ((threadIdx.x & 31) == 0) produce<GROUP, M>(a, p, walker, FB);
         return;
@@ -665,7 +666,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
     const int gi = warp * GPW + (FB ? Lane<GROUP>().sub : LNF().sub);
     long long i = 0;
     Tile t;
-    for (long long k = blockIdx.x; walker.locate(k, &t); k += gridDim.x, ++i) {
+    for (long long k = blockIdx.x; walker.locate(k, &t, a); k += gridDim.x, ++i) {
         const int s = (int)(i % kStages);
         if (!mbar_wait(&p.full[s], (uint32_t)(i / kStages) & 1u, kWaitLimitNs, p.abort)) {
             if ((threadIdx.x & 31) == 0) report_timeout(a, p);
@@ -685,7 +686,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
         if ((threadIdx.x & 31) == 0) mbar_arrive(&p.empty[s]);
     }
     // the partial last group (not a multiple of 16 bytes): direct path
-    if (G_full < a.G && blockIdx.x == gridDim.x - 1 && warp == 0) {
+    if (a.tail && blockIdx.x == gridDim.x - 1 && warp == 0) {
         const long long j = a.G - 1;
         for (int r = 0; r < a.P; ++r) {
             const long long lo = (long long)r * a.G / a.P, hi = (long long)(r + 1) * a.G / a.P;
@@ -952,8 +953,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
     const PipeShared p = pipe_shared(smem);
     pipe_init(p);
     const int warp = threadIdx.x >> 5;
-    const long long G_full = a.n / GROUP;
-    RunWalker<GROUP, M> walker(1, a.G, G_full, a.P);
+    RunWalker<GROUP, M> walker(1, a);
     if (warp == kConsumerWarps) {
         if ((threadIdx.x & 31) == 0) produce<GROUP, M>(a, p, walker, FB);
         return;
@@ -965,7 +965,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
     const int gi = warp * GPW + (FB ? Lane<GROUP>().sub : Lane16<GROUP>().sub);
     long long i = 0;
     Tile t;
-    for (long long k = blockIdx.x; walker.locate(k, &t); k += gridDim.x, ++i) {
+    for (long long k = blockIdx.x; walker.locate(k, &t, a); k += gridDim.x, ++i) {
         const int s = (int)(i % kStages);
         if (!mbar_wait(&p.full[s], (uint32_t)(i / kStages) & 1u, kWaitLimitNs, p.abort)) {
             if ((threadIdx.x & 31) == 0) report_timeout(a, p);
@@ -984,7 +984,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
         __syncwarp();
         if ((threadIdx.x & 31) == 0) mbar_arrive(&p.empty[s]);
     }
-    if (G_full < a.G && blockIdx.x == gridDim.x - 1 && warp == 0) {
+    if (a.tail && blockIdx.x == gridDim.x - 1 && warp == 0) {
         const long long j = a.G - 1;
         const int o = (int)((j * a.P + a.P - 1) / a.G);
         reduce_range<GROUP, BITS, QM>(a, o, j, j + 1, 0, 1);
@@ -1041,8 +1041,8 @@ template <int GROUP, int BITS, int QM>
 __global__ void __launch_bounds__(kGatherThreads) k_gather_tma(const Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
     constexpr int L = GROUP / 8, CB = GROUP * BITS / 8, T = kGatherTileElems / GROUP;
-    const long long G_full = a.n / GROUP;
-    const long long ntiles = (G_full + T - 1) / T;
+    const long long c1 = a.c1;   // full groups of the column window [c0, c1)
+    const long long ntiles = c1 > a.c0 ? (c1 - a.c0 + T - 1) / T : 0;
     const int tid = threadIdx.x;
     const int gi = tid / L, t = tid % L;   // group within the tile, lane within the group
     long long i = 0;
@@ -1054,8 +1054,8 @@ __global__ void __launch_bounds__(kGatherThreads) k_gather_tma(const Args a) {
             if (tid == 0) bulk_wait_read<kGatherBufs - 1>();
             __syncthreads();
         }
-        const long long j0 = k * T;
-        const int cnt = (int)min((long long)T, G_full - j0);
+        const long long j0 = a.c0 + k * T;
+        const int cnt = (int)min((long long)T, c1 - j0);
         if (gi < cnt) {
             const long long j = j0 + gi;
             const uint2 w = load_codes8<BITS>(a.g_codes + (size_t)j * CB, t);
@@ -1071,7 +1071,7 @@ __global__ void __launch_bounds__(kGatherThreads) k_gather_tma(const Args a) {
     }
     if (tid == 0) bulk_wait_all();
     // the partial last group (not a multiple of 16 bytes): direct stores
-    if (G_full < a.G && blockIdx.x == gridDim.x - 1 && tid < L) {
+    if (a.tail && blockIdx.x == gridDim.x - 1 && tid < L) {
         const long long j = a.G - 1;
         const uint2 w = load_codes8<BITS>(a.g_codes + (size_t)j * CB, tid);
         const uint4 v = decode8_bf16<BITS, QM>(w, a.g_params[j]);

@@ -68,6 +68,10 @@ def lib() -> ctypes.CDLL:
         L.echo_init_state.restype = I
         L.echo_allreduce_sim.argtypes = [PP, PP, V, I64, I, I, I, F, F, F, F, V]
         L.echo_allreduce_sim.restype = I
+        L.echo_allreduce_sim_range.argtypes = [PP, PP, V, I64, I, I, I, F, F, F, F, I64, I64, V]
+        L.echo_allreduce_sim_range.restype = I
+        L.echo_allreduce_sim_host.argtypes = [PP, V, PP, PP, V, I64, I, I, I, F, F, F, F, I64, V, V, V]
+        L.echo_allreduce_sim_host.restype = I
         L.echo_phase_quantize.argtypes = [PP, V, I, F, F, F, F, V]
         L.echo_phase_quantize.restype = I
         L.echo_phase_reduce.argtypes = [PP, PP, V, I, F, F, F, F, V]
@@ -148,6 +152,38 @@ def echo_allreduce_sim(inputs: Sequence, outputs: Sequence, st, n: int, P: int, 
                        eta: float, alpha_long: float, alpha_short: float, w: float, stream=None) -> None:
     _check(lib().echo_allreduce_sim(_ptr_array(inputs), _ptr_array(outputs), st, n, P, bits, group,
                                     eta, alpha_long, alpha_short, w, _stream(stream)), "echo_allreduce_sim")
+
+
+def echo_allreduce_sim_range(inputs: Sequence, outputs: Sequence, st, n: int, P: int, bits: int, group: int,
+                             eta: float, alpha_long: float, alpha_short: float, w: float, group_begin: int,
+                             group_end: int, stream=None) -> None:
+    _check(lib().echo_allreduce_sim_range(_ptr_array(inputs), _ptr_array(outputs), st, n, P, bits, group,
+                                          eta, alpha_long, alpha_short, w, group_begin, group_end,
+                                          _stream(stream)), "echo_allreduce_sim_range")
+
+
+def _host_ptr(t) -> int:
+    if isinstance(t, int):
+        return t
+    if t.is_cuda or not t.is_contiguous():
+        raise ValueError("host buffers must be contiguous CPU tensors")
+    return t.data_ptr()
+
+
+def echo_allreduce_sim_host(host_inputs: Sequence, host_output, inputs: Sequence, outputs: Sequence, st, n: int,
+                            P: int, bits: int, group: int, eta: float, alpha_long: float, alpha_short: float,
+                            w: float, chunk_groups: int = 0, stream=None, copy_in=None, copy_out=None) -> None:
+    """Host inputs in, host result out, copies overlapped with the kernels
+    (pinned host tensors for the overlap). `copy_in` / `copy_out` default to
+    `stream` (no overlap)."""
+    s = _stream(stream)
+    hin = (ctypes.c_void_p * len(host_inputs))(*[_host_ptr(t) for t in host_inputs])
+    hout = None if host_output is None else _host_ptr(host_output)
+    _check(lib().echo_allreduce_sim_host(hin, hout, _ptr_array(inputs), _ptr_array(outputs), st, n, P, bits, group,
+                                         eta, alpha_long, alpha_short, w, chunk_groups, s,
+                                         s if copy_in is None else _stream(copy_in),
+                                         s if copy_out is None else _stream(copy_out)),
+           "echo_allreduce_sim_host")
 
 
 def echo_phase_quantize(inputs: Sequence, st, bits: int, eta: float, alpha_long: float, alpha_short: float,

@@ -233,6 +233,69 @@ ECHO_API int echo_phase_reduce(const void* const* inputs, void* const* outputs, 
 ECHO_API int echo_phase_gather(void* const* outputs, echo_state* st, int bits, echo_stream_t stream);
 
 /*
+ * echo_allreduce_sim restricted to the group columns [group_begin, group_end)
+ * of the message: for every rank, groups j with group_begin <= j < group_end
+ * (elements [j*group, min(n, (j+1)*group))), with the ownership of the WHOLE
+ * message (owner(j) as documented at echo_layout). A group column -- group j
+ * of every rank, its payload slots and its EMA entries -- is computed
+ * independently of every other column in all five phases (the explainer's
+ * mechanism 1 reduces each segment at its owner, group by group), so calls on
+ * disjoint windows that together cover [0, G) give, bit for bit, the
+ * outputs, payloads, EMAs and flags of one echo_allreduce_sim call, in any
+ * order. Elements outside the window are neither read nor written. This lets
+ * a caller run the all-reduce chunk by chunk while other chunks are still
+ * being produced or copied (see echo_allreduce_sim_host).
+ *   group_begin, group_end  0 <= group_begin <= group_end <= G
+ *                           (G = ceil(n/group)); an empty window enqueues
+ *                           nothing
+ *   all other arguments     as for echo_allreduce_sim
+ * Errors: those of echo_allreduce_sim; ECHO_EINVAL for a window out of range.
+ */
+ECHO_API int echo_allreduce_sim_range(const void* const* inputs, void* const* outputs, echo_state* st,
+                             int64_t n, int P, int bits, int group,
+                             float eta, float alpha_long, float alpha_short, float w,
+                             int64_t group_begin, int64_t group_end, echo_stream_t stream);
+
+/*
+ * One all-reduce call whose P inputs start, and whose result ends, in host
+ * memory: the library copies the inputs in, runs echo_allreduce_sim_range
+ * chunk by chunk and copies the result out, overlapping the host-to-device
+ * copies of later chunks, the kernels of the current chunk and the
+ * device-to-host copy of earlier chunks on three streams. (The pages' own
+ * kernel pipelines quantization with NVLink transfers; on one GPU the
+ * transfers that remain are the host link's.) Results are bit-identical to
+ * copying everything in, one echo_allreduce_sim call, and copying out.
+ *   host_inputs  host array of P host pointers, each to n bf16 values
+ *                (rank r's partial sum). Page-locked (pinned) memory is
+ *                needed for the copies to overlap; pageable memory works but
+ *                serializes them.
+ *   host_output  host pointer to n bf16 values that receives the reduced
+ *                result (identical on every rank; copied from outputs[0]),
+ *                or NULL to leave the result on the device only
+ *   inputs, outputs  the device buffers of echo_allreduce_sim; the inputs
+ *                are overwritten with host_inputs, every output receives the
+ *                result
+ *   chunk_groups group columns per chunk, >= 1; 0 picks ceil(G / 16)
+ *   stream       the kernels run on it; the call is ordered after earlier
+ *                work on `stream`, and later work on `stream` waits until
+ *                the result has reached host_output
+ *   copy_in, copy_out  streams for the host-to-device and device-to-host
+ *                copies (may equal `stream`, which gives up the overlap)
+ *   all other arguments  as for echo_allreduce_sim
+ * Asynchronous: the host buffers must stay valid, and host_output must not
+ * be read, until `stream` has reached this point (synchronize it, or an
+ * event recorded on it after the call). The first call on a handle creates
+ * three CUDA events (no device memory), released by echo_free.
+ * Errors: those of echo_allreduce_sim (nothing enqueued on ECHO_EINVAL);
+ * ECHO_ECUDA when a copy, event or launch fails, in which case part of the
+ * work may already be enqueued.
+ */
+ECHO_API int echo_allreduce_sim_host(const void* const* host_inputs, void* host_output, void* const* inputs,
+                            void* const* outputs, echo_state* st, int64_t n, int P, int bits, int group,
+                            float eta, float alpha_long, float alpha_short, float w, int64_t chunk_groups,
+                            echo_stream_t stream, echo_stream_t copy_in, echo_stream_t copy_out);
+
+/*
  * Synchronize `stream`, read the sticky flag word into *device_flags (may be
  * NULL) and clear it. Returns ECHO_ETIMEOUT when ECHO_FLAG_TIMEOUT was set,
  * else ECHO_ERANGE when ECHO_FLAG_RANGE was set, else ECHO_OK;
@@ -304,7 +367,8 @@ ECHO_API int echo_allreduce_sim_noalloc(const void* const* inputs, void* const* 
                                         int64_t n, int P, int bits, int group, float eta, float alpha_long,
                                         float alpha_short, float w, uint32_t* flags_out, echo_stream_t stream);
 
-/* Release the host handle (never the caller's device buffers). NULL is a no-op. */
+/* Release the host handle and the events echo_allreduce_sim_host created
+ * for it (never the caller's device buffers). NULL is a no-op. */
 ECHO_API int echo_free(echo_state* st);
 
 /* Static string for a status code. */

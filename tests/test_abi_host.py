@@ -90,6 +90,10 @@ def test_init_rejects_bad_pointers_before_cuda(L):
 def test_calls_reject_missing_handle(L):
     arr = (ctypes.c_void_p * 2)(4096, 8192)
     assert L.echo_allreduce_sim(arr, arr, None, 1024, 2, 4, 128, 1.0, 0.05, 0.5, 0.5, None) == E.ECHO_EINVAL
+    assert L.echo_allreduce_sim_range(arr, arr, None, 1024, 2, 4, 128, 1.0, 0.05, 0.5, 0.5, 0, 8,
+                                      None) == E.ECHO_EINVAL
+    assert L.echo_allreduce_sim_host(arr, None, arr, arr, None, 1024, 2, 4, 128, 1.0, 0.05, 0.5, 0.5, 0,
+                                     None, None, None) == E.ECHO_EINVAL
     assert L.echo_phase_quantize(arr, None, 4, 1.0, 0.05, 0.5, 0.5, None) == E.ECHO_EINVAL
     assert L.echo_phase_reduce(arr, arr, None, 4, 1.0, 0.05, 0.5, 0.5, None) == E.ECHO_EINVAL
     assert L.echo_phase_gather(arr, None, 4, None) == E.ECHO_EINVAL
