@@ -95,6 +95,26 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
         : "memory");
 }
 
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 1-D bulk copy shared -> global (no multicast); dst, src, bytes multiples of 16
+__device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_addr(src)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // ------------------------------------------------------------ tile walk
 
 // A run is a contiguous range of full groups [j0, j1) of one rank, clipped to
@@ -499,8 +519,7 @@ __device__ __forceinline__ void store_f8_cs(float* p, const float2 v[4]) {
 // 8 consecutive elements per lane (lane t of the group's L takes elements
 // [8t, 8t + 8)).
 template <int GROUP, int BITS, int QM>
-__device__ __forceinline__ void quantize_tile_group(const Args& a, const uint8_t* st, const Tile& t, int gi,
-                                                    bool act) {
+__device__ __forceinline__ void quantize_tile_group(const Args& a, uint8_t* st, const Tile& t, int gi, bool act) {
     using LN = Lane<GROUP>;
     constexpr int L = LN::L, Q = (1 << BITS) - 1, CB = GROUP * BITS / 8;
     const LN ln;
@@ -508,8 +527,8 @@ __device__ __forceinline__ void quantize_tile_group(const Args& a, const uint8_t
     const long long j = t.j0 + gi;
     const int e0 = 8 * ln.t;
     const uint16_t* xs = reinterpret_cast<const uint16_t*>(st) + gi * GROUP;
-    const float* els = reinterpret_cast<const float*>(st + kTileElems * 2) + gi * GROUP;
-    const float* ess = reinterpret_cast<const float*>(st + kTileElems * 6) + gi * GROUP;
+    float* els = reinterpret_cast<float*>(st + kTileElems * 2) + gi * GROUP;
+    float* ess = reinterpret_cast<float*>(st + kTileElems * 6) + gi * GROUP;
     float2 v[4], el[4], es[4];
     float lmin = __int_as_float(0x7f800000), lmax = -__int_as_float(0x7f800000);
     if (act) {
@@ -541,13 +560,12 @@ __device__ __forceinline__ void quantize_tile_group(const Args& a, const uint8_t
         nl[p] = ema2(el[p], rho, a.keep_long, a.a_long, a);
         ns[p] = ema2(es[p], rho, a.keep_short, a.a_short, a);
     }
-    float* el_g = a.state + (size_t)r * 2 * a.S + j * GROUP + e0;
-    // 16-byte stores here: measured on B200, 32-byte ones made this pass ~2 %
-    // slower (the owner's pass gains from them)
-    store_f4_pair(el_g, nl[0], nl[1]);
-    store_f4_pair(el_g + 4, nl[2], nl[3]);
-    store_f4_pair(el_g + a.S, ns[0], ns[1]);
-    store_f4_pair(el_g + a.S + 4, ns[2], ns[3]);
+    // the updated EMAs go back into the stage, over the values just read; the
+    // warp then sends its rows to global memory with bulk stores
+    *reinterpret_cast<float4*>(els + e0) = make_float4(nl[0].x, nl[0].y, nl[1].x, nl[1].y);
+    *reinterpret_cast<float4*>(els + e0 + 4) = make_float4(nl[2].x, nl[2].y, nl[3].x, nl[3].y);
+    *reinterpret_cast<float4*>(ess + e0) = make_float4(ns[0].x, ns[0].y, ns[1].x, ns[1].y);
+    *reinterpret_cast<float4*>(ess + e0 + 4) = make_float4(ns[2].x, ns[2].y, ns[3].x, ns[3].y);
     if (ln.t == 0) a.a2a_params[(size_t)r * a.G + j] = g.param;
 }
 
@@ -664,17 +682,41 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
     constexpr int PASSES = FB ? 1 : M * kTileElems / (kConsumerWarps * 32 * kQuantizeLaneElemsNF);
     static_assert(FB || PASSES * kConsumerWarps * 32 * kQuantizeLaneElemsNF == M * kTileElems, "tile split");
     const int gi = warp * GPW + (FB ? Lane<GROUP>().sub : LNF().sub);
+    const bool lead = (threadIdx.x & 31) == 0;
     long long i = 0;
     Tile t;
     for (long long k = blockIdx.x; walker.locate(k, &t, a); k += gridDim.x, ++i) {
         const int s = (int)(i % kStages);
         if (!mbar_wait(&p.full[s], (uint32_t)(i / kStages) & 1u, kWaitLimitNs, p.abort)) {
-            if ((threadIdx.x & 31) == 0) report_timeout(a, p);
+            if (lead) {
+                report_timeout(a, p);
+                if (FB) bulk_wait_all();   // this warp's stores still in flight
+            }
             return;
         }
-        const uint8_t* stage = p.stages + (size_t)s * kStageBytes;
+        uint8_t* stage = p.stages + (size_t)s * kStageBytes;
         if (FB) {
             quantize_tile_group<GROUP, BITS, QM>(a, stage, t, gi, gi < t.count);
+            // The warp's groups are GPW consecutive groups of the tile: their
+            // updated EMA rows leave the stage in two bulk stores. The slot is
+            // released once those stores have read it, one tile later.
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lead) {
+                const int g0 = warp * GPW;
+                const int cnt = min(GPW, t.count - g0);
+                if (cnt > 0) {
+                    const uint32_t bytes = (uint32_t)cnt * GROUP * 4;
+                    float* el = a.state + (size_t)t.rank * 2 * a.S + (t.j0 + g0) * GROUP;
+                    bulk_store(el, stage + kTileElems * 2 + g0 * GROUP * 4, bytes);
+                    bulk_store(el + a.S, stage + kTileElems * 6 + g0 * GROUP * 4, bytes);
+                }
+                bulk_commit();
+                bulk_wait_read<1>();
+                if (i > 0) mbar_arrive(&p.empty[(i - 1) % kStages]);
+            }
+            __syncwarp();
+            continue;
         } else {
 #pragma unroll 1
             for (int m = 0; m < PASSES; ++m) {
@@ -683,7 +725,12 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
             }
         }
         __syncwarp();
-        if ((threadIdx.x & 31) == 0) mbar_arrive(&p.empty[s]);
+        if (lead) mbar_arrive(&p.empty[s]);
+    }
+    if (FB && lead) {
+        bulk_wait_read<0>();
+        if (i > 0) mbar_arrive(&p.empty[(i - 1) % kStages]);
+        bulk_wait_all();
     }
     // the partial last group (not a multiple of 16 bytes): direct path
     if (a.tail && blockIdx.x == gridDim.x - 1 && warp == 0) {
@@ -1003,25 +1050,6 @@ constexpr int kGatherTileElems = kGatherThreads * 8;                 // 2048 ele
 constexpr int kGatherBufs = 4;
 constexpr int kGatherSmem = kGatherBufs * kGatherTileElems * 2;     // 16 KB
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// 1-D bulk copy shared -> global (no multicast); dst, src, bytes multiples of 16
-__device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_addr(src)),
-                 "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-
-template <int N>
-__device__ __forceinline__ void bulk_wait_read() {
-    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
-
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // eight contiguous decoded elements of a group as bf16 (codes word w: 4-bit in
 // w.x, 8-bit in w.x and w.y)
