@@ -578,6 +578,71 @@ def run_ablation(args):
           flush=True)
 
 
+def run_workloads(args):
+    """Every workload's call timed on the GPU (inputs resident, state carried
+    from call to call) and the oracle's call timed on the host, single thread.
+    Chains are timed per site at each bit width they use; the 1 GB message's
+    oracle figure is the main line's sampled `cpu_baseline`."""
+    import numpy as np
+    import torch
+    import oracle as O
+    import workloads as W
+    import bit_error_compensated_group_b200 as E
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    peak, peak_kind = _peak_hbm()
+    out = {}
+    for w in W.ALL:
+        P, n, group = w.P, w.n, w.group
+        widths = sorted({w.bits_at(t) for t in range(w.sites)})
+        ar = E.EchoAllReduce(n, P, group, max(widths), feedback=True, device=dev)
+        inputs = [W.rank_input(w, r, 0, dev) for r in range(P)]
+        outputs = [torch.empty_like(t) for t in inputs]
+        fb = (w.eta, w.alpha_long, w.alpha_short, w.w)
+        entry = {"P": P, "n": n, "sites": w.sites, "int8_sites": w.int8_sites, "per_call": {}}
+        steps = max(3, args.steps)
+        for bits in widths:
+            def call():
+                E.echo_allreduce_sim(inputs, outputs, ar.handle, n, P, bits, group, *fb, stream=stream)
+            for _ in range(max(3, args.warmup)):
+                call()
+            torch.cuda.synchronize(dev)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(steps):
+                call()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            ms = a.elapsed_time(b) / steps
+            ab = algorithmic_bytes(P, n, group, bits)["total"]
+            rc, flags = ar.status()
+            entry["per_call"][f"int{bits}"] = {
+                "gpu_ms": ms, "gbs_bf16_input": P * n * 2 / (ms * 1e-3) / 1e9,
+                "roofline_frac": ab / (ms * 1e-3) / 1e9 / peak, "algorithmic_bytes": ab, "status": rc,
+                "l2_resident": ab < 126e6, "steps": steps}
+        ar.close()
+        del ar, inputs, outputs
+        torch.cuda.empty_cache()
+        if w.sites > 1:
+            entry["gpu_ms_per_chain"] = sum(entry["per_call"][f"int{w.bits_at(t)}"]["gpu_ms"] for t in range(w.sites))
+        if w is not W.HEADLINE and not args.no_cpu_baseline:
+            G = -(-n // group)
+            x = np.zeros((P, G * group), np.uint16)
+            x[:, :n] = W.bf16_bits(W.inputs(w, 0, "cpu"))
+            for bits in widths:
+                el = np.zeros((P, G * group), np.float32)
+                es = np.zeros((P, G * group), np.float32)
+                t0 = time.perf_counter()
+                O.echo_allreduce(x, n_total=n, group=group, bits=bits, e_long=el, e_short=es, eta=w.eta,
+                                 alpha_long=w.alpha_long, alpha_short=w.alpha_short, w=w.w)
+                dt = time.perf_counter() - t0
+                entry["per_call"][f"int{bits}"]["oracle_ms"] = dt * 1e3
+                entry["per_call"][f"int{bits}"]["oracle_cores"] = 1
+        out[w.name] = entry
+    print(json.dumps({"workloads": out, "peak_gbs": peak, "peak_kind": peak_kind, "data": "synthetic"}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -593,6 +658,8 @@ def main():
                     help="off: time the call without EMA state as the main step (profiling)")
     ap.add_argument("--ablation", action="store_true",
                     help="print the accuracy ablations on the synthetic chains instead of timing")
+    ap.add_argument("--workloads", action="store_true",
+                    help="print every workload's GPU and oracle time per call instead of the main line")
     ap.add_argument("--tokens", type=int, default=None,
                     help="tokens per rank (default 131072, the 1 GB message); smaller values are for profiling")
     args = ap.parse_args()
@@ -603,6 +670,8 @@ def main():
         run_reference(args)
     elif args.ablation:
         run_ablation(args)
+    elif args.workloads:
+        run_workloads(args)
     else:
         run_gpu(args)
 
