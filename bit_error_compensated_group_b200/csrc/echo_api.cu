@@ -83,12 +83,11 @@ int grid_for(K kernel, const echo_state* st, int threads = echo_dev::kThreads, i
 
 // Pipelined kernels: opt in to their dynamic shared memory once.
 template <typename K>
-int pipe_grid(K kernel, const echo_state* st) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, echo_dev::kPipeSmem) !=
-        cudaSuccess) {
+int pipe_grid(K kernel, const echo_state* st, int smem) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
         return 0;
     }
-    return grid_for(kernel, st, echo_dev::kPipeThreads, echo_dev::kPipeSmem);
+    return grid_for(kernel, st, echo_dev::kPipeThreads, smem);
 }
 
 enum class Stage { Quantize, Reduce, Gather };
@@ -108,11 +107,11 @@ int64_t tile_bound(Stage stage, const echo_dev::Args& a, int tile_groups) {
 // start only the CTAs that have work.
 template <typename K>
 int launch_pipe(K kernel, int* grid, int64_t max_tiles, const echo_dev::Args& a, const echo_state* st,
-                cudaStream_t s) {
-    if (*grid == 0) *grid = pipe_grid(kernel, st);
+                cudaStream_t s, int smem) {
+    if (*grid == 0) *grid = pipe_grid(kernel, st, smem);
     if (*grid == 0) return ECHO_ECUDA;
     const int g = (int)(max_tiles < (int64_t)*grid ? max_tiles : (int64_t)*grid);
-    kernel<<<g, echo_dev::kPipeThreads, echo_dev::kPipeSmem, s>>>(a);
+    kernel<<<g, echo_dev::kPipeThreads, smem, s>>>(a);
     return ECHO_OK;
 }
 
@@ -129,19 +128,23 @@ int launch_stage(Stage stage, const echo_dev::Args& a, const echo_state* st, cud
         case Stage::Quantize:
             if (a.state) {
                 static int grid = 0;
-                rc = launch_pipe(echo_dev::k_quantize_tma<GROUP, BITS, true, QM>, &grid, tiles, a, st, s);
+                rc = launch_pipe(echo_dev::k_quantize_tma<GROUP, BITS, true, QM>, &grid, tiles, a, st, s,
+                                 echo_dev::pipe_smem(echo_dev::kStagesQuantizeFB));
             } else {
                 static int grid = 0;
-                rc = launch_pipe(echo_dev::k_quantize_tma<GROUP, BITS, false, QM>, &grid, tiles, a, st, s);
+                rc = launch_pipe(echo_dev::k_quantize_tma<GROUP, BITS, false, QM>, &grid, tiles, a, st, s,
+                                 echo_dev::pipe_smem(echo_dev::kStagesQuantizeNF));
             }
             break;
         case Stage::Reduce:
             if (a.state) {
                 static int grid = 0;
-                rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, true, QM>, &grid, tiles, a, st, s);
+                rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, true, QM>, &grid, tiles, a, st, s,
+                                 echo_dev::pipe_smem(echo_dev::kStagesReduceFB));
             } else {
                 static int grid = 0;
-                rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, false, QM>, &grid, tiles, a, st, s);
+                rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, false, QM>, &grid, tiles, a, st, s,
+                                 echo_dev::pipe_smem(echo_dev::kStagesReduceNF));
             }
             break;
         case Stage::Gather: {

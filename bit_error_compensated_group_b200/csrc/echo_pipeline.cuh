@@ -23,11 +23,19 @@
 namespace echo_dev {
 
 constexpr int kConsumerWarps = 8;
-constexpr int kStages = 4;
 constexpr int kPipeThreads = (kConsumerWarps + 1) * 32;
 constexpr int kTileElems = kConsumerWarps * 32 * 8;           // 2048 elements per tile
 constexpr int kStageBytes = kTileElems * (2 + 4 + 4);          // bf16 x + two fp32 EMAs
-constexpr int kPipeSmem = kStages * kStageBytes + 2 * kStages * 8 + 16;
+// ring stages per pipelined kernel (with and without feedback), measured on
+// B200: fewer tiles in flight per CTA stream faster here. The quantize pass
+// with feedback keeps each slot one tile longer (until the bulk stores of the
+// EMAs have read it).
+constexpr int kStagesQuantizeFB = 3;
+constexpr int kStagesReduceFB = 4;
+constexpr int kStagesQuantizeNF = 4;
+constexpr int kStagesReduceNF = 4;
+// dynamic shared memory of a pipelined kernel with NS ring stages
+__host__ __device__ constexpr int pipe_smem(int NS) { return NS * kStageBytes + 2 * NS * 8 + 16; }
 constexpr unsigned long long kWaitLimitNs = 1000ull * 1000ull * 1000ull;   // 1 s
 
 // ------------------------------------------------------------ PTX wrappers
@@ -192,18 +200,20 @@ struct PipeShared {
     uint8_t* stages;
 };
 
+template <int NS>
 __device__ __forceinline__ PipeShared pipe_shared(uint8_t* smem) {
     PipeShared p;
     p.stages = smem;
-    p.full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
-    p.empty = p.full + kStages;
-    p.abort = reinterpret_cast<volatile int*>(p.empty + kStages);
+    p.full = reinterpret_cast<uint64_t*>(smem + NS * kStageBytes);
+    p.empty = p.full + NS;
+    p.abort = reinterpret_cast<volatile int*>(p.empty + NS);
     return p;
 }
 
+template <int NS>
 __device__ __forceinline__ void pipe_init(const PipeShared& p) {
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < NS; ++s) {
             mbar_init(&p.full[s], 1);
             mbar_init(&p.empty[s], kConsumerWarps);
         }
@@ -221,15 +231,15 @@ __device__ __forceinline__ void report_timeout(const Args& a, const PipeShared& 
 // Producer lane: stream tiles of `walker` into the stage ring. `with_state`
 // adds the two EMA tiles of the tile's rank (then M == 1); without state a
 // stage holds M = 5 sub-tiles of bf16 inputs, the same 20 KB.
-template <int GROUP, int M>
+template <int GROUP, int M, int NS>
 __device__ __forceinline__ void produce(const Args& a, const PipeShared& p, RunWalker<GROUP, M>& walker,
                                         bool with_state) {
     long long issued = 0;
     Tile t;
     for (long long k = blockIdx.x; walker.locate(k, &t, a); k += gridDim.x, ++issued) {
-        const int s = (int)(issued % kStages);
-        const uint32_t use = (uint32_t)(issued / kStages);
-        if (issued >= kStages && !mbar_wait(&p.empty[s], (use & 1u) ^ 1u, kWaitLimitNs, p.abort)) {
+        const int s = (int)(issued % NS);
+        const uint32_t use = (uint32_t)(issued / NS);
+        if (issued >= NS && !mbar_wait(&p.empty[s], (use & 1u) ^ 1u, kWaitLimitNs, p.abort)) {
             report_timeout(a, p);
             break;
         }
@@ -245,12 +255,12 @@ __device__ __forceinline__ void produce(const Args& a, const PipeShared& p, RunW
             bulk_load(st + kTileElems * 6, el + a.S + e0, sbytes, &p.full[s]);
         }
     }
-    // drain: the last (up to kStages) tiles' copies must land before the CTA
+    // drain: the last (up to NS) tiles' copies must land before the CTA
     // may retire, whatever happened to the consumers
-    const long long first = issued > kStages ? issued - kStages : 0;
+    const long long first = issued > NS ? issued - NS : 0;
     for (long long i = first; i < issued; ++i) {
-        const int s = (int)(i % kStages);
-        if (!mbar_wait(&p.full[s], (uint32_t)(i / kStages) & 1u, kWaitLimitNs, nullptr)) {
+        const int s = (int)(i % NS);
+        if (!mbar_wait(&p.full[s], (uint32_t)(i / NS) & 1u, kWaitLimitNs, nullptr)) {
             atomicOr(a.flags, (unsigned)ECHO_FLAG_TIMEOUT);
         }
     }
@@ -667,12 +677,13 @@ template <int GROUP, int BITS, bool FB, int QM>
 __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
     constexpr int M = FB ? 1 : kQuantizeSubtilesNF;
-    const PipeShared p = pipe_shared(smem);
-    pipe_init(p);
+    constexpr int NS = FB ? kStagesQuantizeFB : kStagesQuantizeNF;
+    const PipeShared p = pipe_shared<NS>(smem);
+    pipe_init<NS>(p);
     const int warp = threadIdx.x >> 5;
     RunWalker<GROUP, M> walker(0, a);
     if (warp == kConsumerWarps) {
-        if ((threadIdx.x & 31) == 0) produce<GROUP, M>(a, p, walker, FB);
+        if ((threadIdx.x & 31) == 0) produce<GROUP, M, NS>(a, p, walker, FB);
         return;
     }
     // with feedback: 8 elements per lane, one pass per tile; without: 32 per
@@ -686,8 +697,8 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
     long long i = 0;
     Tile t;
     for (long long k = blockIdx.x; walker.locate(k, &t, a); k += gridDim.x, ++i) {
-        const int s = (int)(i % kStages);
-        if (!mbar_wait(&p.full[s], (uint32_t)(i / kStages) & 1u, kWaitLimitNs, p.abort)) {
+        const int s = (int)(i % NS);
+        if (!mbar_wait(&p.full[s], (uint32_t)(i / NS) & 1u, kWaitLimitNs, p.abort)) {
             if (lead) {
                 report_timeout(a, p);
                 if (FB) bulk_wait_all();   // this warp's stores still in flight
@@ -713,7 +724,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
                 }
                 bulk_commit();
                 bulk_wait_read<1>();
-                if (i > 0) mbar_arrive(&p.empty[(i - 1) % kStages]);
+                if (i > 0) mbar_arrive(&p.empty[(i - 1) % NS]);
             }
             __syncwarp();
             continue;
@@ -729,7 +740,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
     }
     if (FB && lead) {
         bulk_wait_read<0>();
-        if (i > 0) mbar_arrive(&p.empty[(i - 1) % kStages]);
+        if (i > 0) mbar_arrive(&p.empty[(i - 1) % NS]);
         bulk_wait_all();
     }
     // the partial last group (not a multiple of 16 bytes): direct path
@@ -997,12 +1008,13 @@ template <int GROUP, int BITS, bool FB, int QM>
 __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
     constexpr int M = FB ? 1 : kReduceSubtilesNF;
-    const PipeShared p = pipe_shared(smem);
-    pipe_init(p);
+    constexpr int NS = FB ? kStagesReduceFB : kStagesReduceNF;
+    const PipeShared p = pipe_shared<NS>(smem);
+    pipe_init<NS>(p);
     const int warp = threadIdx.x >> 5;
     RunWalker<GROUP, M> walker(1, a);
     if (warp == kConsumerWarps) {
-        if ((threadIdx.x & 31) == 0) produce<GROUP, M>(a, p, walker, FB);
+        if ((threadIdx.x & 31) == 0) produce<GROUP, M, NS>(a, p, walker, FB);
         return;
     }
     // with feedback: 8 elements per lane, one pass per tile; without: 16 per
@@ -1013,8 +1025,8 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
     long long i = 0;
     Tile t;
     for (long long k = blockIdx.x; walker.locate(k, &t, a); k += gridDim.x, ++i) {
-        const int s = (int)(i % kStages);
-        if (!mbar_wait(&p.full[s], (uint32_t)(i / kStages) & 1u, kWaitLimitNs, p.abort)) {
+        const int s = (int)(i % NS);
+        if (!mbar_wait(&p.full[s], (uint32_t)(i / NS) & 1u, kWaitLimitNs, p.abort)) {
             if ((threadIdx.x & 31) == 0) report_timeout(a, p);
             return;
         }
