@@ -105,18 +105,33 @@ int64_t tile_bound(Stage stage, const echo_dev::Args& a, int tile_groups) {
 
 // A persistent launch never needs more CTAs than tiles: small messages then
 // start only the CTAs that have work.
+// `pdl`: launch as a programmatic dependent of the kernel before it on the
+// stream (the owners' pass right after this call's quantize pass).
 template <typename K>
 int launch_pipe(K kernel, int* grid, int64_t max_tiles, const echo_dev::Args& a, const echo_state* st,
-                cudaStream_t s, int smem) {
+                cudaStream_t s, int smem, bool pdl = false) {
     if (*grid == 0) *grid = pipe_grid(kernel, st, smem);
     if (*grid == 0) return ECHO_ECUDA;
     const int g = (int)(max_tiles < (int64_t)*grid ? max_tiles : (int64_t)*grid);
-    kernel<<<g, echo_dev::kPipeThreads, smem, s>>>(a);
-    return ECHO_OK;
+    if (!pdl) {
+        kernel<<<g, echo_dev::kPipeThreads, smem, s>>>(a);
+        return ECHO_OK;
+    }
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(g);
+    cfg.blockDim = dim3(echo_dev::kPipeThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, a) == cudaSuccess ? ECHO_OK : ECHO_ECUDA;
 }
 
 template <int GROUP, int BITS, int QM>
-int launch_stage(Stage stage, const echo_dev::Args& a, const echo_state* st, cudaStream_t s) {
+int launch_stage(Stage stage, const echo_dev::Args& a, const echo_state* st, cudaStream_t s, bool pdl) {
     int rc = ECHO_OK;
     // tiles of 2048 elements with feedback; without, 4 x 2048 (quantize) and
     // 5 x 2048 (reduce) -- the sub-tile counts of the kernels' RunWalkers
@@ -140,11 +155,11 @@ int launch_stage(Stage stage, const echo_dev::Args& a, const echo_state* st, cud
             if (a.state) {
                 static int grid = 0;
                 rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, true, QM>, &grid, tiles, a, st, s,
-                                 echo_dev::pipe_smem(echo_dev::kStagesReduceFB));
+                                 echo_dev::pipe_smem(echo_dev::kStagesReduceFB), pdl);
             } else {
                 static int grid = 0;
                 rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, false, QM>, &grid, tiles, a, st, s,
-                                 echo_dev::pipe_smem(echo_dev::kStagesReduceNF));
+                                 echo_dev::pipe_smem(echo_dev::kStagesReduceNF), pdl);
             }
             break;
         case Stage::Gather: {
@@ -160,27 +175,29 @@ int launch_stage(Stage stage, const echo_dev::Args& a, const echo_state* st, cud
 }
 
 template <int GROUP>
-int launch_bits(Stage stage, int bits, const echo_dev::Args& a, const echo_state* st, cudaStream_t s) {
+int launch_bits(Stage stage, int bits, const echo_dev::Args& a, const echo_state* st, cudaStream_t s, bool pdl) {
     switch (st->quantizer) {
         case ECHO_QUANT_DIRECTED:
-            return bits == 4 ? launch_stage<GROUP, 4, echo_dev::kQuantDirected>(stage, a, st, s)
-                             : launch_stage<GROUP, 8, echo_dev::kQuantDirected>(stage, a, st, s);
+            return bits == 4 ? launch_stage<GROUP, 4, echo_dev::kQuantDirected>(stage, a, st, s, pdl)
+                             : launch_stage<GROUP, 8, echo_dev::kQuantDirected>(stage, a, st, s, pdl);
         case ECHO_QUANT_NEAREST:
-            return bits == 4 ? launch_stage<GROUP, 4, echo_dev::kQuantNearest>(stage, a, st, s)
-                             : launch_stage<GROUP, 8, echo_dev::kQuantNearest>(stage, a, st, s);
+            return bits == 4 ? launch_stage<GROUP, 4, echo_dev::kQuantNearest>(stage, a, st, s, pdl)
+                             : launch_stage<GROUP, 8, echo_dev::kQuantNearest>(stage, a, st, s, pdl);
         case ECHO_QUANT_INT_ZERO:
-            return bits == 4 ? launch_stage<GROUP, 4, echo_dev::kQuantIntZero>(stage, a, st, s)
-                             : launch_stage<GROUP, 8, echo_dev::kQuantIntZero>(stage, a, st, s);
+            return bits == 4 ? launch_stage<GROUP, 4, echo_dev::kQuantIntZero>(stage, a, st, s, pdl)
+                             : launch_stage<GROUP, 8, echo_dev::kQuantIntZero>(stage, a, st, s, pdl);
     }
     return ECHO_EINVAL;
 }
 
-int launch(Stage stage, int bits, const echo_dev::Args& a, const echo_state* st, cudaStream_t s) {
+// `pdl` (owners' pass only): this launch directly follows the same call's
+// quantize launch on the stream and may overlap its tail.
+int launch(Stage stage, int bits, const echo_dev::Args& a, const echo_state* st, cudaStream_t s, bool pdl = false) {
     switch (st->group) {
-        case 32: return launch_bits<32>(stage, bits, a, st, s);
-        case 64: return launch_bits<64>(stage, bits, a, st, s);
-        case 128: return launch_bits<128>(stage, bits, a, st, s);
-        case 256: return launch_bits<256>(stage, bits, a, st, s);
+        case 32: return launch_bits<32>(stage, bits, a, st, s, pdl);
+        case 64: return launch_bits<64>(stage, bits, a, st, s, pdl);
+        case 128: return launch_bits<128>(stage, bits, a, st, s, pdl);
+        case 256: return launch_bits<256>(stage, bits, a, st, s, pdl);
     }
     return ECHO_EINVAL;
 }
@@ -350,7 +367,7 @@ int echo_allreduce_sim(const void* const* inputs, void* const* outputs, echo_sta
     if (P >= 2) {
         if (int rc = launch(Stage::Quantize, bits, a, st, s)) return rc;
     }
-    return launch(Stage::Reduce, bits, a, st, s);
+    return launch(Stage::Reduce, bits, a, st, s, P >= 2);
 }
 
 int echo_allreduce_sim_range(const void* const* inputs, void* const* outputs, echo_state* st, int64_t n, int P,
@@ -371,7 +388,7 @@ int echo_allreduce_sim_range(const void* const* inputs, void* const* outputs, ec
     if (P >= 2) {
         if (int rc = launch(Stage::Quantize, bits, a, st, s)) return rc;
     }
-    return launch(Stage::Reduce, bits, a, st, s);
+    return launch(Stage::Reduce, bits, a, st, s, P >= 2);
 }
 
 int echo_allreduce_sim_host(const void* const* host_inputs, void* host_output, void* const* inputs,

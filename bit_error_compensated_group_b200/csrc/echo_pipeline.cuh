@@ -48,6 +48,17 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
 }
 
+// Programmatic dependent launch. The quantize pass lets the owners' pass
+// launch as soon as every quantize CTA has started; the owners' consumers wait
+// for the quantize grid to complete (and its writes to be visible) before they
+// read the all-to-all payload. Without a programmatic dependency the wait
+// returns at once.
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void mbar_fence_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
@@ -679,6 +690,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
     constexpr int M = FB ? 1 : kQuantizeSubtilesNF;
     constexpr int NS = FB ? kStagesQuantizeFB : kStagesQuantizeNF;
     const PipeShared p = pipe_shared<NS>(smem);
+    griddep_launch_dependents();
     pipe_init<NS>(p);
     const int warp = threadIdx.x >> 5;
     RunWalker<GROUP, M> walker(0, a);
@@ -1014,9 +1026,14 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
     const int warp = threadIdx.x >> 5;
     RunWalker<GROUP, M> walker(1, a);
     if (warp == kConsumerWarps) {
+        // the owned groups' x and EMAs: the quantize pass writes neither, so
+        // the producer may stage them while that pass is still running
         if ((threadIdx.x & 31) == 0) produce<GROUP, M, NS>(a, p, walker, FB);
         return;
     }
+    // the payload, the flag word and the outputs: only once the quantize pass
+    // is complete (an output may be the same buffer as an input it reads)
+    griddep_wait();
     // with feedback: 8 elements per lane, one pass per tile; without: 16 per
     // lane, two passes over the 4-sub-tile stage
     constexpr int GPW = FB ? Lane<GROUP>::GPW : Lane16<GROUP>::GPW;
