@@ -162,3 +162,74 @@ def test_host_call(P, n, group, bits, chunk):
             compare(gpu, orc, el, es, n, G, P, p, True, f"host call {c}")
     finally:
         gpu.close()
+
+
+@pytest.mark.parametrize("windowed", [False, True])
+def test_in_place_large(windowed):
+    """Outputs that are the inputs, on a message whose quantize pass spans
+    many tiles per CTA: the owners' pass (a programmatic dependent of the
+    quantize pass) must not write an output before the quantize pass has read
+    it. Two calls with carried state; every element checked."""
+    P, n, group = 8, (1 << 22) + 77, 128
+    p = Params()
+    G = -(-n // group)
+    ld = G * group
+    x = random_inputs(P, n, 4242)
+    gpu = GpuEcho(P, n, group, 4, True)
+    el = np.zeros((P, ld), np.float32)
+    es = np.zeros((P, ld), np.float32)
+    try:
+        xb = padded(u16(x), ld)
+        for c in range(2):
+            gpu.set_inputs(x if c == 0 else E_out)
+            if windowed:
+                for b, e in windows(G, [G // 3 + 1], "forward"):
+                    E.echo_allreduce_sim_range(gpu.inputs, gpu.inputs, gpu.ar.handle, n, P, 4, group, p.eta,
+                                               p.alpha_long, p.alpha_short, p.w, b, e)
+            else:
+                E.echo_allreduce_sim(gpu.inputs, gpu.inputs, gpu.ar.handle, n, P, 4, group, p.eta, p.alpha_long,
+                                     p.alpha_short, p.w)
+            orc = O.echo_allreduce(xb, n_total=n, group=group, bits=4, e_long=el, e_short=es)
+            got = np.stack([u16(t) for t in gpu.inputs])
+            assert np.array_equal(got, orc.y[:, :n]), f"call {c}"
+            gl, gs = gpu.state()
+            assert np.array_equal(gl, el[:, :n]) and np.array_equal(gs, es[:, :n]), f"state call {c}"
+            # the next call reduces this call's result again (every rank holds it)
+            E_out = torch.from_numpy(orc.y[:, :n].astype(np.uint16).view(np.int16)).view(torch.bfloat16)
+            xb = padded(orc.y[:, :n].copy(), ld)
+    finally:
+        gpu.close()
+
+
+@pytest.mark.parametrize("to_host,streams", [(False, "separate"), (True, "same"), (True, "pageable")])
+def test_host_call_forms(to_host, streams):
+    """The host-buffer call without a host result (the result stays on the
+    device), with every copy on the caller's stream, and from pageable host
+    memory (the copies then serialize): the same bits in every form."""
+    P, n, group = 4, 70001, 64
+    p = Params(group=group)
+    G = -(-n // group)
+    ld = G * group
+    gpu = GpuEcho(P, n, group, 4, True)
+    pin = streams != "pageable"
+    host_in = [torch.empty(n, dtype=torch.bfloat16, pin_memory=pin) for _ in range(P)]
+    host_out = torch.empty(n, dtype=torch.bfloat16, pin_memory=pin) if to_host else None
+    s = torch.cuda.current_stream()
+    cin, cout = (torch.cuda.Stream(), torch.cuda.Stream()) if streams == "separate" else (s, s)
+    el = np.zeros((P, ld), np.float32)
+    es = np.zeros((P, ld), np.float32)
+    try:
+        for c in range(2):
+            x = random_inputs(P, n, 77 * c + 5)
+            for r in range(P):
+                host_in[r].copy_(x[r])
+            E.echo_allreduce_sim_host(host_in, host_out, gpu.inputs, gpu.outputs, gpu.ar.handle, n, P, 4, group,
+                                      p.eta, p.alpha_long, p.alpha_short, p.w, 9, stream=s, copy_in=cin,
+                                      copy_out=cout)
+            s.synchronize()
+            orc = O.echo_allreduce(padded(u16(x), ld), n_total=n, group=group, bits=4, e_long=el, e_short=es)
+            if to_host:
+                assert np.array_equal(u16(host_out), orc.y[0, :n])
+            compare(gpu, orc, el, es, n, G, P, p, True, f"{streams} call {c}")
+    finally:
+        gpu.close()
