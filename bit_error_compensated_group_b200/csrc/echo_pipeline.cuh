@@ -786,15 +786,10 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
     float2 xo[4], acc[4];
 #pragma unroll
     for (int p = 0; p < 4; ++p) xo[p] = acc[p] = make_float2(0.0f, 0.0f);
-    if (act) {
-        load_x8c_smem(xs + e0, xo);
-        float2 el[4], es[4];
-        load_f8_smem(els, e0, e0 + 4, el);
-        load_f8_smem(ess, e0, e0 + 4, es);
-#pragma unroll
-        for (int p = 0; p < 4; ++p) xo[p] = inject2(xo[p], el[p], es[p], a);
-    }
-    // binary32 sum in rank order 0..P-1: own x' unquantized, others decoded
+    // binary32 sum in rank order 0..P-1: own x' unquantized, others decoded.
+    // The payload loads of a batch of RB ranks are issued together; the first
+    // batch's go out before the staged x and EMAs are read, so that their
+    // latency overlaps the feedback injection.
     for (int r0 = 0; r0 < a.P; r0 += RB) {
         uint32_t cw[RB][CW];
         uint32_t pw[RB];
@@ -816,6 +811,14 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
                 }
                 pw[k] = a.a2a_params[slot];
             }
+        }
+        if (r0 == 0 && act) {
+            load_x8c_smem(xs + e0, xo);
+            float2 el[4], es[4];
+            load_f8_smem(els, e0, e0 + 4, el);
+            load_f8_smem(ess, e0, e0 + 4, es);
+#pragma unroll
+            for (int p = 0; p < 4; ++p) xo[p] = inject2(xo[p], el[p], es[p], a);
         }
 #pragma unroll
         for (int k = 0; k < RB; ++k) {
