@@ -34,6 +34,9 @@ struct echo_state {
 namespace {
 
 constexpr uint64_t kAlign = 256;
+// Launch configurations are cached per device (a process may drive several
+// GPUs; the shared-memory opt-in of a kernel is made on each device).
+constexpr int kMaxDevices = 64;
 constexpr int64_t kMaxN = int64_t(1) << 40;
 
 uint64_t align_up(uint64_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
@@ -108,11 +111,12 @@ int64_t tile_bound(Stage stage, const echo_dev::Args& a, int tile_groups) {
 // `pdl`: launch as a programmatic dependent of the kernel before it on the
 // stream (the owners' pass right after this call's quantize pass).
 template <typename K>
-int launch_pipe(K kernel, int* grid, int64_t max_tiles, const echo_dev::Args& a, const echo_state* st,
+int launch_pipe(K kernel, int* grids, int64_t max_tiles, const echo_dev::Args& a, const echo_state* st,
                 cudaStream_t s, int smem, bool pdl = false) {
-    if (*grid == 0) *grid = pipe_grid(kernel, st, smem);
-    if (*grid == 0) return ECHO_ECUDA;
-    const int g = (int)(max_tiles < (int64_t)*grid ? max_tiles : (int64_t)*grid);
+    int& grid = grids[st->device];
+    if (grid == 0) grid = pipe_grid(kernel, st, smem);
+    if (grid == 0) return ECHO_ECUDA;
+    const int g = (int)(max_tiles < (int64_t)grid ? max_tiles : (int64_t)grid);
     if (!pdl) {
         kernel<<<g, echo_dev::kPipeThreads, smem, s>>>(a);
         return ECHO_OK;
@@ -142,31 +146,32 @@ int launch_stage(Stage stage, const echo_dev::Args& a, const echo_state* st, cud
     switch (stage) {
         case Stage::Quantize:
             if (a.state) {
-                static int grid = 0;
-                rc = launch_pipe(echo_dev::k_quantize_tma<GROUP, BITS, true, QM>, &grid, tiles, a, st, s,
+                static int grid[kMaxDevices];
+                rc = launch_pipe(echo_dev::k_quantize_tma<GROUP, BITS, true, QM>, grid, tiles, a, st, s,
                                  echo_dev::pipe_smem(echo_dev::kStagesQuantizeFB));
             } else {
-                static int grid = 0;
-                rc = launch_pipe(echo_dev::k_quantize_tma<GROUP, BITS, false, QM>, &grid, tiles, a, st, s,
+                static int grid[kMaxDevices];
+                rc = launch_pipe(echo_dev::k_quantize_tma<GROUP, BITS, false, QM>, grid, tiles, a, st, s,
                                  echo_dev::pipe_smem(echo_dev::kStagesQuantizeNF));
             }
             break;
         case Stage::Reduce:
             if (a.state) {
-                static int grid = 0;
-                rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, true, QM>, &grid, tiles, a, st, s,
+                static int grid[kMaxDevices];
+                rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, true, QM>, grid, tiles, a, st, s,
                                  echo_dev::pipe_smem(echo_dev::kStagesReduceFB), pdl);
             } else {
-                static int grid = 0;
-                rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, false, QM>, &grid, tiles, a, st, s,
+                static int grid[kMaxDevices];
+                rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, false, QM>, grid, tiles, a, st, s,
                                  echo_dev::pipe_smem(echo_dev::kStagesReduceNF), pdl);
             }
             break;
         case Stage::Gather: {
             auto k = echo_dev::k_gather_tma<GROUP, BITS, QM>;
-            static int grid = 0;
-            if (grid == 0) grid = grid_for(k, st, echo_dev::kGatherThreads, echo_dev::kGatherSmem);
-            k<<<grid, echo_dev::kGatherThreads, echo_dev::kGatherSmem, s>>>(a);
+            static int grid[kMaxDevices];
+            int& g = grid[st->device];
+            if (g == 0) g = grid_for(k, st, echo_dev::kGatherThreads, echo_dev::kGatherSmem);
+            k<<<g, echo_dev::kGatherThreads, echo_dev::kGatherSmem, s>>>(a);
             break;
         }
     }
@@ -289,7 +294,7 @@ int echo_init_state(echo_state** out, int64_t n, int P, int group, int max_bits,
     if (!workspace_dev || !aligned(workspace_dev, kAlign)) return ECHO_EINVAL;
     if (state_dev && !aligned(state_dev, 16)) return ECHO_EINVAL;
     int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return ECHO_ECUDA;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ECHO_ECUDA;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return ECHO_ECUDA;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (state_dev && cudaMemsetAsync(state_dev, 0, L.state_bytes, s) != cudaSuccess) return ECHO_ECUDA;
