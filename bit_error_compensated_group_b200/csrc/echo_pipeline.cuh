@@ -6,7 +6,7 @@
 // loads issued from registers, bytes in flight per SM are capped by the
 // register file; here one producer lane per CTA streams whole tiles
 // (T groups x (bf16 x, e_long, e_short)) into a ring of shared-memory stages
-// with cp.async.bulk (the TMA engine, 1-D, no tensor map, no multicast), and
+// with cp.async.bulk (the TMA engine, 1-D, no tensor map, this CTA only), and
 // the consumer warps compute from shared memory and write results straight
 // back to HBM. Several 20 KB tiles per CTA are in flight at any time.
 //
@@ -118,7 +118,7 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// 1-D bulk copy shared -> global (no multicast); dst, src, bytes multiples of 16
+// 1-D bulk copy shared -> global (this CTA's buffer); dst, src, bytes multiples of 16
 __device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes) {
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_addr(src)),
                  "r"(bytes)
