@@ -187,7 +187,12 @@ ECHO_API int echo_set_quantizer(echo_state* st, int quantizer);
  *   eta        feedback gain, finite
  *   alpha_long, alpha_short   EMA rates in [0, 1]
  *   w          weight of the short EMA in the compensation, in [0, 1]
- *   stream     CUDA stream; the call is asynchronous on it
+ *   stream     CUDA stream; the call is asynchronous on it. It is two
+ *              kernels (the non-owners' quantize pass, then the owners'
+ *              pass); the second is a programmatic dependent launch of the
+ *              first, so it may start while the first drains, but it reads
+ *              nothing the first writes before that kernel has completed.
+ *              Towards other work on the stream the call is ordered as usual.
  * Arithmetic (binary32, round-to-nearest, no contraction into fused
  * multiply-add): c = eta*(w*e_short + (1-w)*e_long), x' = float(x) + c
  * (x' = float(x) without state); per group mn = min + 0, mx = max + 0,
