@@ -187,7 +187,7 @@ ECHO_API int echo_set_quantizer(echo_state* st, int quantizer);
  *   eta        feedback gain, finite
  *   alpha_long, alpha_short   EMA rates in [0, 1]
  *   w          weight of the short EMA in the compensation, in [0, 1]
- *   stream     CUDA stream; the call is asynchronous on it. It is two
+ *   stream     CUDA stream; the call is asynchronous on it. For P >= 2 it is two
  *              kernels (the non-owners' quantize pass, then the owners'
  *              pass); the second is a programmatic dependent launch of the
  *              first, so it may start while the first drains, but it reads
