@@ -22,6 +22,7 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = [
     "-O3", "-lineinfo", "-std=c++17",
     "-fmad=false",                 # every float op below is an explicit _rn intrinsic anyway
+    "-split-compile", "0",         # optimize the kernel instantiations on all host cores
     "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
     "-shared", "-cudart", "static",
 ]

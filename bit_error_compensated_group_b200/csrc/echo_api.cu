@@ -29,6 +29,8 @@ struct echo_state {
     // the two copy streams, created on first use, destroyed by echo_free
     cudaEvent_t ev[3];
     bool have_events;
+    int rank;              // -1: the single-GPU simulation; else this rank of a multi-GPU call
+    echo_rank_layout rl;   // rank handles: the layout for max_bits
 };
 
 namespace {
@@ -145,7 +147,15 @@ int launch_stage(Stage stage, const echo_dev::Args& a, const echo_state* st, cud
     const int64_t tiles = tile_bound(stage, a, subtiles * echo_dev::kTileElems / GROUP);
     switch (stage) {
         case Stage::Quantize:
-            if (a.state) {
+            if (st->rank >= 0 && a.state) {
+                static int grid[kMaxDevices];
+                rc = launch_pipe(echo_dev::k_quantize_tma<GROUP, BITS, true, QM, true>, grid, tiles, a, st, s,
+                                 echo_dev::pipe_smem(echo_dev::kStagesQuantizeFB));
+            } else if (st->rank >= 0) {
+                static int grid[kMaxDevices];
+                rc = launch_pipe(echo_dev::k_quantize_tma<GROUP, BITS, false, QM, true>, grid, tiles, a, st, s,
+                                 echo_dev::pipe_smem(echo_dev::kStagesQuantizeNF));
+            } else if (a.state) {
                 static int grid[kMaxDevices];
                 rc = launch_pipe(echo_dev::k_quantize_tma<GROUP, BITS, true, QM>, grid, tiles, a, st, s,
                                  echo_dev::pipe_smem(echo_dev::kStagesQuantizeFB));
@@ -156,7 +166,17 @@ int launch_stage(Stage stage, const echo_dev::Args& a, const echo_state* st, cud
             }
             break;
         case Stage::Reduce:
-            if (a.state) {
+            // one rank of a multi-GPU call reads its received rows: the
+            // instantiation with the general slot addressing
+            if (st->rank >= 0 && a.state) {
+                static int grid[kMaxDevices];
+                rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, true, QM, true>, grid, tiles, a, st, s,
+                                 echo_dev::pipe_smem(echo_dev::kStagesReduceFB), pdl);
+            } else if (st->rank >= 0) {
+                static int grid[kMaxDevices];
+                rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, false, QM, true>, grid, tiles, a, st, s,
+                                 echo_dev::pipe_smem(echo_dev::kStagesReduceNF), pdl);
+            } else if (a.state) {
                 static int grid[kMaxDevices];
                 rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, true, QM>, grid, tiles, a, st, s,
                                  echo_dev::pipe_smem(echo_dev::kStagesReduceFB), pdl);
@@ -167,6 +187,14 @@ int launch_stage(Stage stage, const echo_dev::Args& a, const echo_state* st, cud
             }
             break;
         case Stage::Gather: {
+            if (st->rank >= 0) {   // one rank's output: the register-path decoder
+                auto k = echo_dev::k_decode_rank<GROUP, BITS, QM>;
+                static int grid[kMaxDevices];
+                int& g = grid[st->device];
+                if (g == 0) g = grid_for(k, st, echo_dev::kDecodeThreads, 0);
+                k<<<g, echo_dev::kDecodeThreads, 0, s>>>(a);
+                break;
+            }
             auto k = echo_dev::k_gather_tma<GROUP, BITS, QM>;
             static int grid[kMaxDevices];
             int& g = grid[st->device];
@@ -245,6 +273,12 @@ bool make_args(const echo_state* st, int bits, const void* const* inputs, void* 
     a->n = st->n;
     a->G = st->G;
     set_window(a, st, 0, st->G);
+    // every rank, in the simulation's layouts
+    a->rank_lo = 0;
+    a->rank_hi = st->P;
+    a->a2a_stride = st->G;
+    a->out_lo = 0;
+    a->out_hi = st->P;
     a->S = st->S;
     a->P = st->P;
     a->eta = eta;
@@ -257,6 +291,115 @@ bool make_args(const echo_state* st, int bits, const void* const* inputs, void* 
     a->one = 1.0f;
     return true;
 }
+
+// Layout of one rank's workspace in a multi-GPU call (see echo_rank_layout).
+bool rank_layout(int64_t n, int P, int rank, int group, int max_bits, int bits, echo_rank_layout* L) {
+    if (!valid_sizes(n, P, group) || !valid_bits(max_bits) || !valid_bits(bits) || bits > max_bits) return false;
+    if (rank < 0 || rank >= P) return false;
+    const int64_t G = (n + group - 1) / group;
+    const uint64_t cb = (uint64_t)group * (uint64_t)bits / 8, cb_max = (uint64_t)group * (uint64_t)max_bits / 8;
+    int64_t seg_max = 0;
+    for (int s = 0; s < P; ++s) {
+        const int64_t len = (int64_t)(s + 1) * G / P - (int64_t)s * G / P;
+        if (len > seg_max) seg_max = len;
+    }
+    L->groups = G;
+    L->seg_begin = (int64_t)rank * G / P;
+    L->seg_groups = (int64_t)(rank + 1) * G / P - L->seg_begin;
+    L->seg_max = seg_max;
+    L->code_bytes = cb;
+    const uint64_t Pu = (uint64_t)P, Gu = (uint64_t)G, seg = (uint64_t)L->seg_groups, sm = (uint64_t)seg_max;
+    uint64_t off = 0;
+    L->flags_offset = off;
+    off += kAlign;
+    L->send_codes_offset = off;
+    off = align_up(off + Gu * cb_max);
+    L->send_params_offset = off;
+    off = align_up(off + Gu * 4);
+    L->recv_codes_offset = off;
+    off = align_up(off + Pu * seg * cb_max);
+    L->recv_params_offset = off;
+    off = align_up(off + Pu * seg * 4);
+    L->gsend_codes_offset = off;
+    off = align_up(off + sm * cb_max);
+    L->gsend_params_offset = off;
+    off = align_up(off + sm * 4);
+    L->grecv_codes_offset = off;
+    off = align_up(off + Pu * sm * cb_max);
+    L->grecv_params_offset = off;
+    off = align_up(off + Pu * sm * 4);
+    L->workspace_bytes = off;
+    L->state_bytes = 2 * Gu * (uint64_t)group * sizeof(float);
+    return true;
+}
+
+// Kernel arguments of one rank's phase. `x` / `out`: this rank's input and
+// output (either may be null where the phase does not use it).
+enum class RankPhase { Quantize, Reduce, Decode };
+
+bool make_rank_args(const echo_state* st, int bits, RankPhase phase, const void* x, void* out, float eta, float aL,
+                    float aS, float w, echo_dev::Args* a) {
+    std::memset(a, 0, sizeof(*a));
+    echo_rank_layout L;
+    if (!rank_layout(st->n, st->P, st->rank, st->group, st->max_bits, bits, &L)) return false;
+    const int r = st->rank;
+    if (x) {
+        if (!aligned(x, 16)) return false;
+        a->in[r] = static_cast<const uint16_t*>(x);
+    }
+    if (out) {
+        if (!aligned(out, 16)) return false;
+        a->out[r] = static_cast<uint16_t*>(out);
+    }
+    uint8_t* ws = st->workspace;
+    a->state = st->state;
+    a->state_rank_base = r;
+    a->flags = reinterpret_cast<uint32_t*>(ws + L.flags_offset);
+    a->n = st->n;
+    a->G = st->G;
+    a->S = st->S;
+    a->P = st->P;
+    set_window(a, st, 0, st->G);
+    a->rank_lo = r;
+    a->rank_hi = r + 1;
+    a->out_lo = r;
+    a->out_hi = r + 1;
+    switch (phase) {
+        case RankPhase::Quantize:   // this rank's row of slots [r][j], all j
+            a->a2a_codes = ws + L.send_codes_offset;
+            a->a2a_params = reinterpret_cast<uint32_t*>(ws + L.send_params_offset);
+            a->a2a_rank_base = r;
+            a->a2a_stride = st->G;
+            break;
+        case RankPhase::Reduce:     // slots [r'][j] of this rank's segment, received from every r'
+            a->a2a_codes = ws + L.recv_codes_offset;
+            a->a2a_params = reinterpret_cast<uint32_t*>(ws + L.recv_params_offset);
+            a->a2a_stride = L.seg_groups;
+            a->a2a_col_base = L.seg_begin;
+            a->g_codes = ws + L.gsend_codes_offset;
+            a->g_params = reinterpret_cast<uint32_t*>(ws + L.gsend_params_offset);
+            a->g_col_base = L.seg_begin;
+            a->write_outputs = st->P == 1;   // a single rank's output comes from this pass
+            break;
+        case RankPhase::Decode:     // every owner's segment, gathered and padded to seg_max
+            a->g_codes = ws + L.grecv_codes_offset;
+            a->g_params = reinterpret_cast<uint32_t*>(ws + L.grecv_params_offset);
+            a->g_seg_stride = L.seg_max;
+            break;
+    }
+    a->eta = eta;
+    a->w = w;
+    a->one_minus_w = 1.0f - w;
+    a->a_long = aL;
+    a->keep_long = 1.0f - aL;
+    a->a_short = aS;
+    a->keep_short = 1.0f - aS;
+    a->one = 1.0f;
+    return true;
+}
+
+bool sim_handle(const echo_state* st) { return st && st->rank < 0; }
+bool rank_handle(const echo_state* st) { return st && st->rank >= 0; }
 
 int set_device(const echo_state* st) {
     int cur = -1;
@@ -314,6 +457,7 @@ int echo_init_state(echo_state** out, int64_t n, int P, int group, int max_bits,
     st->sm_count = sms;
     st->quantizer = ECHO_QUANT_DIRECTED;
     st->have_events = false;
+    st->rank = -1;
     *out = st;
     return ECHO_OK;
 }
@@ -328,7 +472,7 @@ int echo_set_quantizer(echo_state* st, int quantizer) {
 
 int echo_phase_quantize(const void* const* inputs, echo_state* st, int bits, float eta, float alpha_long,
                         float alpha_short, float w, echo_stream_t stream) {
-    if (!st || !inputs || !valid_bits(bits) || bits > st->max_bits) return ECHO_EINVAL;
+    if (!sim_handle(st) || !inputs || !valid_bits(bits) || bits > st->max_bits) return ECHO_EINVAL;
     if (!valid_feedback(eta, alpha_long, alpha_short, w)) return ECHO_EINVAL;
     echo_dev::Args a;
     if (!make_args(st, bits, inputs, nullptr, eta, alpha_long, alpha_short, w, &a)) return ECHO_EINVAL;
@@ -339,7 +483,7 @@ int echo_phase_quantize(const void* const* inputs, echo_state* st, int bits, flo
 
 int echo_phase_reduce(const void* const* inputs, void* const* outputs, echo_state* st, int bits, float eta,
                       float alpha_long, float alpha_short, float w, echo_stream_t stream) {
-    if (!st || !inputs || !valid_bits(bits) || bits > st->max_bits) return ECHO_EINVAL;
+    if (!sim_handle(st) || !inputs || !valid_bits(bits) || bits > st->max_bits) return ECHO_EINVAL;
     if (!valid_feedback(eta, alpha_long, alpha_short, w)) return ECHO_EINVAL;
     if (st->P == 1 && !outputs) return ECHO_EINVAL;
     echo_dev::Args a;
@@ -350,7 +494,7 @@ int echo_phase_reduce(const void* const* inputs, void* const* outputs, echo_stat
 }
 
 int echo_phase_gather(void* const* outputs, echo_state* st, int bits, echo_stream_t stream) {
-    if (!st || !outputs || !valid_bits(bits) || bits > st->max_bits) return ECHO_EINVAL;
+    if (!sim_handle(st) || !outputs || !valid_bits(bits) || bits > st->max_bits) return ECHO_EINVAL;
     echo_dev::Args a;
     if (!make_args(st, bits, nullptr, outputs, 0.0f, 0.0f, 0.0f, 0.0f, &a)) return ECHO_EINVAL;
     if (int rc = set_device(st)) return rc;
@@ -360,7 +504,7 @@ int echo_phase_gather(void* const* outputs, echo_state* st, int bits, echo_strea
 
 int echo_allreduce_sim(const void* const* inputs, void* const* outputs, echo_state* st, int64_t n, int P, int bits,
                        int group, float eta, float alpha_long, float alpha_short, float w, echo_stream_t stream) {
-    if (!st || !inputs || !outputs) return ECHO_EINVAL;
+    if (!sim_handle(st) || !inputs || !outputs) return ECHO_EINVAL;
     if (n != st->n || P != st->P || group != st->group) return ECHO_EINVAL;
     if (!valid_bits(bits) || bits > st->max_bits) return ECHO_EINVAL;
     if (!valid_feedback(eta, alpha_long, alpha_short, w)) return ECHO_EINVAL;
@@ -378,7 +522,7 @@ int echo_allreduce_sim(const void* const* inputs, void* const* outputs, echo_sta
 int echo_allreduce_sim_range(const void* const* inputs, void* const* outputs, echo_state* st, int64_t n, int P,
                              int bits, int group, float eta, float alpha_long, float alpha_short, float w,
                              int64_t group_begin, int64_t group_end, echo_stream_t stream) {
-    if (!st || !inputs || !outputs) return ECHO_EINVAL;
+    if (!sim_handle(st) || !inputs || !outputs) return ECHO_EINVAL;
     if (n != st->n || P != st->P || group != st->group) return ECHO_EINVAL;
     if (!valid_bits(bits) || bits > st->max_bits) return ECHO_EINVAL;
     if (!valid_feedback(eta, alpha_long, alpha_short, w)) return ECHO_EINVAL;
@@ -400,7 +544,7 @@ int echo_allreduce_sim_host(const void* const* host_inputs, void* host_output, v
                             void* const* outputs, echo_state* st, int64_t n, int P, int bits, int group, float eta,
                             float alpha_long, float alpha_short, float w, int64_t chunk_groups,
                             echo_stream_t stream, echo_stream_t copy_in, echo_stream_t copy_out) {
-    if (!st || !host_inputs || !inputs || !outputs) return ECHO_EINVAL;
+    if (!sim_handle(st) || !host_inputs || !inputs || !outputs) return ECHO_EINVAL;
     if (n != st->n || P != st->P || group != st->group) return ECHO_EINVAL;
     if (!valid_bits(bits) || bits > st->max_bits) return ECHO_EINVAL;
     if (!valid_feedback(eta, alpha_long, alpha_short, w)) return ECHO_EINVAL;
@@ -459,6 +603,82 @@ int echo_allreduce_sim_host(const void* const* host_inputs, void* host_output, v
         if (cudaStreamWaitEvent(s, ev_done, 0) != cudaSuccess) return ECHO_ECUDA;
     }
     return ECHO_OK;
+}
+
+int echo_query_rank_layout(int64_t n, int P, int rank, int group, int max_bits, int bits, echo_rank_layout* out) {
+    if (!out) return ECHO_EINVAL;
+    echo_rank_layout L;
+    if (!rank_layout(n, P, rank, group, max_bits, bits, &L)) return ECHO_EINVAL;
+    *out = L;
+    return ECHO_OK;
+}
+
+int echo_init_rank(echo_state** out, int64_t n, int P, int rank, int group, int max_bits, void* state_dev,
+                   void* workspace_dev, echo_stream_t stream) {
+    echo_rank_layout L;
+    if (!out || !rank_layout(n, P, rank, group, max_bits, max_bits, &L)) return ECHO_EINVAL;
+    if (!workspace_dev || !aligned(workspace_dev, kAlign)) return ECHO_EINVAL;
+    if (state_dev && !aligned(state_dev, 16)) return ECHO_EINVAL;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ECHO_ECUDA;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return ECHO_ECUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (state_dev && cudaMemsetAsync(state_dev, 0, L.state_bytes, s) != cudaSuccess) return ECHO_ECUDA;
+    // the flag word, and the payload buffers: padding the exchange never
+    // writes is then defined
+    if (cudaMemsetAsync(workspace_dev, 0, L.workspace_bytes, s) != cudaSuccess) return ECHO_ECUDA;
+    echo_state* st = new (std::nothrow) echo_state;
+    if (!st) return ECHO_EINVAL;
+    st->n = n;
+    st->P = P;
+    st->group = group;
+    st->max_bits = max_bits;
+    st->G = L.groups;
+    st->S = L.groups * group;
+    st->state = static_cast<float*>(state_dev);
+    st->workspace = static_cast<uint8_t*>(workspace_dev);
+    st->device = dev;
+    st->sm_count = sms;
+    st->quantizer = ECHO_QUANT_DIRECTED;
+    st->have_events = false;
+    st->rank = rank;
+    st->rl = L;
+    *out = st;
+    return ECHO_OK;
+}
+
+int echo_rank_quantize(const void* x, echo_state* st, int bits, float eta, float alpha_long, float alpha_short,
+                       float w, echo_stream_t stream) {
+    if (!rank_handle(st) || !x || !valid_bits(bits) || bits > st->max_bits) return ECHO_EINVAL;
+    if (!valid_feedback(eta, alpha_long, alpha_short, w)) return ECHO_EINVAL;
+    echo_dev::Args a;
+    if (!make_rank_args(st, bits, RankPhase::Quantize, x, nullptr, eta, alpha_long, alpha_short, w, &a))
+        return ECHO_EINVAL;
+    if (int rc = set_device(st)) return rc;
+    if (st->P < 2) return ECHO_OK;
+    return launch(Stage::Quantize, bits, a, st, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int echo_rank_reduce(const void* x, void* out, echo_state* st, int bits, float eta, float alpha_long,
+                     float alpha_short, float w, echo_stream_t stream) {
+    if (!rank_handle(st) || !x || !valid_bits(bits) || bits > st->max_bits) return ECHO_EINVAL;
+    if (st->P == 1 && !out) return ECHO_EINVAL;
+    if (!valid_feedback(eta, alpha_long, alpha_short, w)) return ECHO_EINVAL;
+    echo_dev::Args a;
+    if (!make_rank_args(st, bits, RankPhase::Reduce, x, st->P == 1 ? out : nullptr, eta, alpha_long, alpha_short,
+                        w, &a))
+        return ECHO_EINVAL;
+    if (int rc = set_device(st)) return rc;
+    return launch(Stage::Reduce, bits, a, st, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int echo_rank_decode(void* out, echo_state* st, int bits, echo_stream_t stream) {
+    if (!rank_handle(st) || !out || !valid_bits(bits) || bits > st->max_bits) return ECHO_EINVAL;
+    echo_dev::Args a;
+    if (!make_rank_args(st, bits, RankPhase::Decode, nullptr, out, 0.0f, 0.0f, 0.0f, 0.0f, &a)) return ECHO_EINVAL;
+    if (int rc = set_device(st)) return rc;
+    if (st->P < 2) return ECHO_OK;
+    return launch(Stage::Gather, bits, a, st, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int echo_check_watchdog(echo_state* st, uint32_t limit_us, echo_stream_t stream) {
@@ -558,6 +778,7 @@ int echo_allreduce_sim_noalloc(const void* const* inputs, void* const* outputs, 
     st.sm_count = sms;
     st.quantizer = ECHO_QUANT_DIRECTED;
     st.have_events = false;
+    st.rank = -1;
     echo_dev::Args a;
     if (!make_args(&st, bits, inputs, outputs, eta, alpha_long, alpha_short, w, &a)) return ECHO_EINVAL;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

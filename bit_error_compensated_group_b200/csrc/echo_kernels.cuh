@@ -62,7 +62,53 @@ struct Args {
     // whole message: 0, n / group) and, when tail != 0, the partial last group
     long long c0, c1;
     int tail;
+    // Which ranks a launch serves and how their buffers are addressed. The
+    // single-GPU simulation serves ranks [0, P) with the layouts above
+    // (rank_lo 0, rank_hi P, a2a_stride G, every base 0, g_seg_stride 0).
+    // One rank of a multi-GPU call (rank_lo = r, rank_hi = r + 1) holds
+    // only its own rows: its EMA state (state_rank_base = r), its all-to-all
+    // send row or the P received rows of its segment, its gather send
+    // buffer, and the P gathered segments padded to g_seg_stride groups.
+    int rank_lo, rank_hi;           // quantize: these ranks' runs; reduce: these owners' runs
+    int state_rank_base;            // state row of rank r: r - state_rank_base
+    int a2a_rank_base;              // all-to-all slot (r, j): row r - a2a_rank_base,
+    long long a2a_stride;           //   of a2a_stride groups, column j - a2a_col_base
+    long long a2a_col_base;
+    long long g_col_base;           // gather payload written at j - g_col_base
+    long long g_seg_stride;         // > 0: gathered payload read as [owner][g_seg_stride]
+    int out_lo, out_hi;             // gather decode: outputs of ranks [out_lo, out_hi)
 };
+
+__device__ __forceinline__ size_t a2a_slot(const Args& a, int r, long long j) {
+    return (size_t)(r - a.a2a_rank_base) * (size_t)a.a2a_stride + (size_t)(j - a.a2a_col_base);
+}
+
+// The pipelined kernels' simulation instantiations (RK = false) keep the
+// plain [P][G] slot and [P][2][S] state addressing; one rank of a
+// multi-GPU call (RK = true) uses the general form above.
+template <bool RK>
+__device__ __forceinline__ size_t a2a_slot_t(const Args& a, int r, long long j) {
+    return RK ? a2a_slot(a, r, j) : (size_t)r * (size_t)a.G + (size_t)j;
+}
+
+__device__ __forceinline__ float* state_row(const Args& a, int r) {
+    return a.state + (size_t)(r - a.state_rank_base) * 2 * (size_t)a.S;
+}
+
+template <bool RK>
+__device__ __forceinline__ float* state_row_t(const Args& a, int r) {
+    return RK ? state_row(a, r) : a.state + (size_t)r * 2 * (size_t)a.S;
+}
+
+// where the gather payload of group j is read: group j itself, or, for a
+// gathered buffer of P owner segments padded to g_seg_stride groups, its
+// place in its owner's segment (owner(j) = (j P + P - 1) / G, the segment
+// starting at floor(owner G / P))
+__device__ __forceinline__ size_t g_read_slot(const Args& a, long long j) {
+    if (a.g_seg_stride == 0) return (size_t)j;
+    const long long o = (j * a.P + a.P - 1) / a.G;
+    return (size_t)(o * a.g_seg_stride + j - o * a.G / a.P);
+}
 
 // ------------------------------------------------------------------ helpers
 
@@ -274,7 +320,7 @@ __device__ __forceinline__ void quantize_range(const Args& a, int r, long long j
     constexpr int L = LN::L, GPW = LN::GPW, Q = (1 << BITS) - 1, CB = GROUP * BITS / 8;
     const LN ln;
     const uint16_t* x = a.in[r];
-    float* el_base = a.state ? a.state + (size_t)r * 2 * a.S : nullptr;
+    float* el_base = a.state ? state_row(a, r) : nullptr;
     float* es_base = a.state ? el_base + a.S : nullptr;
     for (long long j0 = j_begin + warp * GPW; j0 < j_end; j0 += nwarps * GPW) {
         const long long j = j0 + ln.sub;
@@ -311,7 +357,7 @@ __device__ __forceinline__ void quantize_range(const Args& a, int r, long long j
         raise_flags(a, bad);
         const Grid g = make_grid<L, Q, QM>(lmin, lmax);
         if (act) {
-            uint8_t* codes = a.a2a_codes + ((size_t)r * a.G + j) * CB;
+            uint8_t* codes = a.a2a_codes + a2a_slot(a, r, j) * CB;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const long long e = j * GROUP + 4 * ln.chunk(h);
@@ -333,7 +379,7 @@ __device__ __forceinline__ void quantize_range(const Args& a, int r, long long j
                     store_f4(es_base, e, a.n, full, &es[4 * h]);
                 }
             }
-            if (ln.t == 0) a.a2a_params[(size_t)r * a.G + j] = g.param;
+            if (ln.t == 0) a.a2a_params[a2a_slot(a, r, j)] = g.param;
         }
     }
 }
@@ -347,7 +393,7 @@ __device__ __forceinline__ void reduce_range(const Args& a, int o, long long j_b
     constexpr int RB = 8;   // ranks whose payload loads are issued together
     const LN ln;
     const uint16_t* x = a.in[o];
-    float* el_base = a.state ? a.state + (size_t)o * 2 * a.S : nullptr;
+    float* el_base = a.state ? state_row(a, o) : nullptr;
     float* es_base = a.state ? el_base + a.S : nullptr;
     for (long long j0 = j_begin + warp * GPW; j0 < j_end; j0 += nwarps * GPW) {
         const long long j = j0 + ln.sub;
@@ -381,7 +427,7 @@ __device__ __forceinline__ void reduce_range(const Args& a, int o, long long j_b
                 cw[k][0] = cw[k][1] = 0u;
                 pw[k] = 0u;
                 if (act && r < a.P && r != o) {
-                    const size_t slot = (size_t)r * a.G + j;
+                    const size_t slot = a2a_slot(a, r, j);
                     const uint8_t* codes = a.a2a_codes + slot * CB;
                     cw[k][0] = load_chunk_codes<BITS>(codes, ln.chunk(0));
                     cw[k][1] = load_chunk_codes<BITS>(codes, ln.chunk(1));
@@ -424,7 +470,7 @@ __device__ __forceinline__ void reduce_range(const Args& a, int o, long long j_b
         if (a.P >= 2) {
             const Grid g = make_grid<L, Q, QM>(lmin, lmax);
             if (act) {
-                uint8_t* codes = a.g_codes + (size_t)j * CB;
+                uint8_t* codes = a.g_codes + (size_t)(j - a.g_col_base) * CB;
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const long long e = j * GROUP + 4 * ln.chunk(h);
@@ -440,7 +486,7 @@ __device__ __forceinline__ void reduce_range(const Args& a, int o, long long j_b
                         for (int r = 0; r < a.P; ++r) store_y4(a.out[r], e, a.n, full, &yb[4 * h]);
                     }
                 }
-                if (ln.t == 0) a.g_params[j] = g.param;
+                if (ln.t == 0) a.g_params[j - a.g_col_base] = g.param;
             }
         } else if (act) {
             // a single rank sends nothing: its output is its own x'

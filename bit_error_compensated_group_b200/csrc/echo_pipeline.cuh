@@ -149,7 +149,8 @@ struct Tile {
 template <int GROUP, int M = 1>
 struct RunWalker {
     static constexpr int T = M * kTileElems / GROUP;   // groups per tile (M sub-tiles)
-    // kind 0: non-owned runs of every rank (quantize); kind 1: owned runs (reduce).
+    // kind 0: non-owned runs of the ranks [rank_lo, rank_hi) (quantize); kind
+    // 1: the owned runs of those ranks (reduce).
     // G, P and the window are read from the kernel arguments when needed
     // rather than held in registers.
     int kind;
@@ -180,10 +181,13 @@ struct RunWalker {
         run_j0 = b;
         run_len = max(0LL, e - b);
     }
-    __device__ __forceinline__ int runs(const Args& a) const { return kind == 0 ? 2 * a.P : a.P; }
+    __device__ __forceinline__ int runs(const Args& a) const { return kind == 0 ? 2 * a.rank_hi : a.rank_hi; }
     __device__ __forceinline__ int rank_of_run() const { return kind == 0 ? (run >> 1) : run; }
 
-    __device__ __forceinline__ RunWalker(int kind_, const Args& a) : kind(kind_), run(0), base(0) { load_run(a); }
+    __device__ __forceinline__ RunWalker(int kind_, const Args& a)
+        : kind(kind_), run(kind_ == 0 ? 2 * a.rank_lo : a.rank_lo), base(0) {
+        if (run < runs(a)) load_run(a);
+    }
 
     // Tile k (k never decreases between calls); false when past the end.
     __device__ __forceinline__ bool locate(long long k, Tile* t, const Args& a) {
@@ -242,7 +246,7 @@ __device__ __forceinline__ void report_timeout(const Args& a, const PipeShared& 
 // Producer lane: stream tiles of `walker` into the stage ring. `with_state`
 // adds the two EMA tiles of the tile's rank (then M == 1); without state a
 // stage holds M = 5 sub-tiles of bf16 inputs, the same 20 KB.
-template <int GROUP, int M, int NS>
+template <int GROUP, int M, int NS, bool RK>
 __device__ __forceinline__ void produce(const Args& a, const PipeShared& p, RunWalker<GROUP, M>& walker,
                                         bool with_state) {
     long long issued = 0;
@@ -261,7 +265,7 @@ __device__ __forceinline__ void produce(const Args& a, const PipeShared& p, RunW
         mbar_arrive_expect_tx(&p.full[s], xbytes + (with_state ? 2 * sbytes : 0));
         bulk_load(st, a.in[t.rank] + e0, xbytes, &p.full[s]);
         if (with_state) {
-            const float* el = a.state + (size_t)t.rank * 2 * a.S;
+            const float* el = state_row_t<RK>(a, t.rank);
             bulk_load(st + kTileElems * 2, el + e0, sbytes, &p.full[s]);
             bulk_load(st + kTileElems * 6, el + a.S + e0, sbytes, &p.full[s]);
         }
@@ -539,7 +543,7 @@ __device__ __forceinline__ void store_f8_cs(float* p, const float2 v[4]) {
 // One non-owned group of a tile with feedback (x, e_long, e_short staged):
 // 8 consecutive elements per lane (lane t of the group's L takes elements
 // [8t, 8t + 8)).
-template <int GROUP, int BITS, int QM>
+template <int GROUP, int BITS, int QM, bool RK>
 __device__ __forceinline__ void quantize_tile_group(const Args& a, uint8_t* st, const Tile& t, int gi, bool act) {
     using LN = Lane<GROUP>;
     constexpr int L = LN::L, Q = (1 << BITS) - 1, CB = GROUP * BITS / 8;
@@ -569,7 +573,7 @@ __device__ __forceinline__ void quantize_tile_group(const Args& a, uint8_t* st, 
     float2 e[4];
 #pragma unroll
     for (int p = 0; p < 4; ++p) e[p] = encode2<QM, Q>(v[p], g, a);
-    uint8_t* codes = a.a2a_codes + ((size_t)r * a.G + j) * CB;
+    uint8_t* codes = a.a2a_codes + a2a_slot_t<RK>(a, r, j) * CB;
     const uint2 pk = pack_codes8<BITS>(e);
     if (BITS == 4) *reinterpret_cast<uint32_t*>(codes + 4 * ln.t) = pk.x;
     else *reinterpret_cast<uint2*>(codes + 8 * ln.t) = pk;
@@ -587,7 +591,7 @@ __device__ __forceinline__ void quantize_tile_group(const Args& a, uint8_t* st, 
     *reinterpret_cast<float4*>(els + e0 + 4) = make_float4(nl[2].x, nl[2].y, nl[3].x, nl[3].y);
     *reinterpret_cast<float4*>(ess + e0) = make_float4(ns[0].x, ns[0].y, ns[1].x, ns[1].y);
     *reinterpret_cast<float4*>(ess + e0 + 4) = make_float4(ns[2].x, ns[2].y, ns[3].x, ns[3].y);
-    if (ln.t == 0) a.a2a_params[(size_t)r * a.G + j] = g.param;
+    if (ln.t == 0) a.a2a_params[a2a_slot_t<RK>(a, r, j)] = g.param;
 }
 
 // Without feedback the quantizer reads bf16 values only, and the per-group
@@ -634,7 +638,7 @@ __device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
 
 __device__ __forceinline__ float2 bf16_pair(uint32_t u) { return make_float2(bf16_lo(u), bf16_hi(u)); }
 
-template <int GROUP, int BITS, int QM>
+template <int GROUP, int BITS, int QM, bool RK>
 __device__ __forceinline__ void quantize_tile_group_nf(const Args& a, const uint8_t* st, const Tile& t, int gi,
                                                        bool act) {
     using LN = LaneE<GROUP, kQuantizeLaneElemsNF>;
@@ -668,7 +672,7 @@ __device__ __forceinline__ void quantize_tile_group_nf(const Args& a, const uint
     raise_flags(a, act && g.bad);
     if (!act) return;
     const long long j = t.j0 + gi;
-    uint8_t* codes = a.a2a_codes + ((size_t)t.rank * a.G + j) * CB;
+    uint8_t* codes = a.a2a_codes + a2a_slot_t<RK>(a, t.rank, j) * CB;
 #pragma unroll
     for (int h = 0; h < H; ++h) {
         float2 e[4];
@@ -681,10 +685,10 @@ __device__ __forceinline__ void quantize_tile_group_nf(const Args& a, const uint
         if (BITS == 4) *reinterpret_cast<uint32_t*>(codes + 4 * c) = pk.x;
         else *reinterpret_cast<uint2*>(codes + 8 * c) = pk;
     }
-    if (ln.t == 0) a.a2a_params[(size_t)t.rank * a.G + j] = g.param;
+    if (ln.t == 0) a.a2a_params[a2a_slot_t<RK>(a, t.rank, j)] = g.param;
 }
 
-template <int GROUP, int BITS, bool FB, int QM>
+template <int GROUP, int BITS, bool FB, int QM, bool RK = false>
 __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
     constexpr int M = FB ? 1 : kQuantizeSubtilesNF;
@@ -695,7 +699,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
     const int warp = threadIdx.x >> 5;
     RunWalker<GROUP, M> walker(0, a);
     if (warp == kConsumerWarps) {
-        if ((threadIdx.x & 31) == 0) produce<GROUP, M, NS>(a, p, walker, FB);
+        if ((threadIdx.x & 31) == 0) produce<GROUP, M, NS, RK>(a, p, walker, FB);
         return;
     }
     // with feedback: 8 elements per lane, one pass per tile; without: 32 per
@@ -719,7 +723,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
         }
         uint8_t* stage = p.stages + (size_t)s * kStageBytes;
         if (FB) {
-            quantize_tile_group<GROUP, BITS, QM>(a, stage, t, gi, gi < t.count);
+            quantize_tile_group<GROUP, BITS, QM, RK>(a, stage, t, gi, gi < t.count);
             // The warp's groups are GPW consecutive groups of the tile: their
             // updated EMA rows leave the stage in two bulk stores. The slot is
             // released once those stores have read it, one tile later.
@@ -730,7 +734,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
                 const int cnt = min(GPW, t.count - g0);
                 if (cnt > 0) {
                     const uint32_t bytes = (uint32_t)cnt * GROUP * 4;
-                    float* el = a.state + (size_t)t.rank * 2 * a.S + (t.j0 + g0) * GROUP;
+                    float* el = state_row_t<RK>(a, t.rank) + (t.j0 + g0) * GROUP;
                     bulk_store(el, stage + kTileElems * 2 + g0 * GROUP * 4, bytes);
                     bulk_store(el + a.S, stage + kTileElems * 6 + g0 * GROUP * 4, bytes);
                 }
@@ -744,7 +748,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
 #pragma unroll 1
             for (int m = 0; m < PASSES; ++m) {
                 const int g = gi + m * kConsumerWarps * GPW;
-                quantize_tile_group_nf<GROUP, BITS, QM>(a, stage, t, g, g < t.count);
+                quantize_tile_group_nf<GROUP, BITS, QM, RK>(a, stage, t, g, g < t.count);
             }
         }
         __syncwarp();
@@ -758,7 +762,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
     // the partial last group (not a multiple of 16 bytes): direct path
     if (a.tail && blockIdx.x == gridDim.x - 1 && warp == 0) {
         const long long j = a.G - 1;
-        for (int r = 0; r < a.P; ++r) {
+        for (int r = a.rank_lo; r < a.rank_hi; ++r) {
             const long long lo = (long long)r * a.G / a.P, hi = (long long)(r + 1) * a.G / a.P;
             if (j < lo || j >= hi) quantize_range<GROUP, BITS, QM>(a, r, j, j + 1, 0, 1);
         }
@@ -769,7 +773,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
 
 // One owned group of a tile with feedback (x, e_long, e_short staged): 8
 // consecutive elements per lane, like the quantize pass.
-template <int GROUP, int BITS, int QM>
+template <int GROUP, int BITS, int QM, bool RK>
 __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* st, const Tile& t, int gi,
                                                   bool act) {
     using LN = Lane<GROUP>;
@@ -800,7 +804,7 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
             for (int c = 0; c < CW; ++c) cw[k][c] = 0u;
             pw[k] = 0u;
             if (act && r < a.P && r != o) {
-                const size_t slot = (size_t)r * a.G + j;
+                const size_t slot = a2a_slot_t<RK>(a, r, j);
                 const uint8_t* codes = a.a2a_codes + slot * CB;
                 if (BITS == 4) {
                     cw[k][0] = *reinterpret_cast<const uint32_t*>(codes + 4 * ln.t);
@@ -860,11 +864,11 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
             e[p] = encode2<QM, Q>(acc[p], g, a);
             yb[p] = bf16x2_rn(fma2_rn(add2_rn(e[p], splat(-kMagic)), g.s, g.z));
         }
-        uint8_t* codes = a.g_codes + (size_t)j * CB;
+        uint8_t* codes = a.g_codes + (size_t)(j - a.g_col_base) * CB;
         const uint2 pk = pack_codes8<BITS>(e);
         if (BITS == 4) *reinterpret_cast<uint32_t*>(codes + 4 * ln.t) = pk.x;
         else *reinterpret_cast<uint2*>(codes + 8 * ln.t) = pk;
-        if (ln.t == 0) a.g_params[j] = g.param;
+        if (ln.t == 0) a.g_params[j - a.g_col_base] = g.param;
         if (a.write_outputs) {
             // phase 4 in the owner's pass: every rank's output gets the decoded
             // requantized sum -- the same bits a decode of the gathered payload gives
@@ -890,7 +894,7 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
         nl[p] = ema2(el[p], rho, a.keep_long, a.a_long, a);
         ns[p] = ema2(es[p], rho, a.keep_short, a.a_short, a);
     }
-    float* el_g = a.state + (size_t)o * 2 * a.S + j * GROUP + e0;
+    float* el_g = state_row_t<RK>(a, o) + j * GROUP + e0;
     store_f8_cs(el_g, nl);
     store_f8_cs(el_g + a.S, ns);
 }
@@ -898,7 +902,7 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
 // The owner's pass without feedback, 16 elements per lane (chunks t and
 // t + L16 of 8 elements): twice the elements per payload load batch and per
 // group-level step of the 8-element path, and 16-byte output stores.
-template <int GROUP, int BITS, int QM>
+template <int GROUP, int BITS, int QM, bool RK>
 __device__ __forceinline__ void reduce_tile_group_nf(const Args& a, const uint8_t* st, const Tile& t, int gi,
                                                      bool act) {
     using LN = Lane16<GROUP>;
@@ -928,7 +932,7 @@ __device__ __forceinline__ void reduce_tile_group_nf(const Args& a, const uint8_
 #pragma unroll
             for (int c = 0; c < 2 * CW; ++c) cw[k][c] = 0u;
             if (act && r < a.P && r != o) {
-                const size_t slot = (size_t)r * a.G + j;
+                const size_t slot = a2a_slot_t<RK>(a, r, j);
                 const uint8_t* codes = a.a2a_codes + slot * CB;
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
@@ -985,7 +989,7 @@ __device__ __forceinline__ void reduce_tile_group_nf(const Args& a, const uint8_
         const GridP g = make_grid_p<L, Q, QM>(lmin, lmax);
         raise_flags(a, act && g.bad);
         if (!act) return;
-        uint8_t* codes = a.g_codes + (size_t)j * CB;
+        uint8_t* codes = a.g_codes + (size_t)(j - a.g_col_base) * CB;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             float2 e[4];
@@ -997,7 +1001,7 @@ __device__ __forceinline__ void reduce_tile_group_nf(const Args& a, const uint8_
 #pragma unroll
             for (int p = 0; p < 4; ++p) yw[4 * h + p] = bf16x2_rn(fma2_rn(add2_rn(e[p], splat(-kMagic)), g.s, g.z));
         }
-        if (ln.t == 0) a.g_params[j] = g.param;
+        if (ln.t == 0) a.g_params[j - a.g_col_base] = g.param;
         if (a.write_outputs) {
             // phase 4 in the owner's pass: every rank's output gets the decoded
             // requantized sum -- the same bits a decode of the gathered payload gives
@@ -1019,7 +1023,7 @@ __device__ __forceinline__ void reduce_tile_group_nf(const Args& a, const uint8_
     }
 }
 
-template <int GROUP, int BITS, bool FB, int QM>
+template <int GROUP, int BITS, bool FB, int QM, bool RK = false>
 __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
     constexpr int M = FB ? 1 : kReduceSubtilesNF;
@@ -1031,7 +1035,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
     if (warp == kConsumerWarps) {
         // the owned groups' x and EMAs: the quantize pass writes neither, so
         // the producer may stage them while that pass is still running
-        if ((threadIdx.x & 31) == 0) produce<GROUP, M, NS>(a, p, walker, FB);
+        if ((threadIdx.x & 31) == 0) produce<GROUP, M, NS, RK>(a, p, walker, FB);
         return;
     }
     // the payload, the flag word and the outputs: only once the quantize pass
@@ -1052,12 +1056,12 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
         }
         const uint8_t* stage = p.stages + (size_t)s * kStageBytes;
         if (FB) {
-            reduce_tile_group<GROUP, BITS, QM>(a, stage, t, gi, gi < t.count);
+            reduce_tile_group<GROUP, BITS, QM, RK>(a, stage, t, gi, gi < t.count);
         } else {
 #pragma unroll 1
             for (int m = 0; m < PASSES; ++m) {
                 const int g = gi + m * kConsumerWarps * GPW;
-                reduce_tile_group_nf<GROUP, BITS, QM>(a, stage, t, g, g < t.count);
+                reduce_tile_group_nf<GROUP, BITS, QM, RK>(a, stage, t, g, g < t.count);
             }
         }
         __syncwarp();
@@ -1066,7 +1070,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
     if (a.tail && blockIdx.x == gridDim.x - 1 && warp == 0) {
         const long long j = a.G - 1;
         const int o = (int)((j * a.P + a.P - 1) / a.G);
-        reduce_range<GROUP, BITS, QM>(a, o, j, j + 1, 0, 1);
+        if (o >= a.rank_lo && o < a.rank_hi) reduce_range<GROUP, BITS, QM>(a, o, j, j + 1, 0, 1);
     }
 }
 
@@ -1118,14 +1122,15 @@ __global__ void __launch_bounds__(kGatherThreads) k_gather_tma(const Args a) {
         const int cnt = (int)min((long long)T, c1 - j0);
         if (gi < cnt) {
             const long long j = j0 + gi;
-            const uint2 w = load_codes8<BITS>(a.g_codes + (size_t)j * CB, t);
-            *reinterpret_cast<uint4*>(buf + gi * GROUP + 8 * t) = decode8_bf16<BITS, QM>(w, a.g_params[j]);
+            const size_t gs = g_read_slot(a, j);
+            const uint2 w = load_codes8<BITS>(a.g_codes + gs * CB, t);
+            *reinterpret_cast<uint4*>(buf + gi * GROUP + 8 * t) = decode8_bf16<BITS, QM>(w, a.g_params[gs]);
         }
         fence_proxy_async_smem();
         __syncthreads();
         if (tid == 0) {
             const uint32_t bytes = (uint32_t)cnt * GROUP * 2;
-            for (int r = 0; r < a.P; ++r) bulk_store(a.out[r] + j0 * GROUP, buf, bytes);
+            for (int r = a.out_lo; r < a.out_hi; ++r) bulk_store(a.out[r] + j0 * GROUP, buf, bytes);
             bulk_commit();
         }
     }
@@ -1133,11 +1138,75 @@ __global__ void __launch_bounds__(kGatherThreads) k_gather_tma(const Args a) {
     // the partial last group (not a multiple of 16 bytes): direct stores
     if (a.tail && blockIdx.x == gridDim.x - 1 && tid < L) {
         const long long j = a.G - 1;
-        const uint2 w = load_codes8<BITS>(a.g_codes + (size_t)j * CB, tid);
-        const uint4 v = decode8_bf16<BITS, QM>(w, a.g_params[j]);
+        const size_t gs = g_read_slot(a, j);
+        const uint2 w = load_codes8<BITS>(a.g_codes + gs * CB, tid);
+        const uint4 v = decode8_bf16<BITS, QM>(w, a.g_params[gs]);
         const uint32_t yb[4] = {v.x, v.y, v.z, v.w};
         const long long e = j * GROUP + 8 * tid;
-        for (int r = 0; r < a.P; ++r) {
+        for (int r = a.out_lo; r < a.out_hi; ++r) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                if (e + k < a.n) a.out[r][e + k] = (uint16_t)(yb[k >> 1] >> (16 * (k & 1)));
+        }
+    }
+}
+
+// Phase 4 on one rank of a multi-GPU call: every group of the gathered
+// payload (P owner segments, each padded to g_seg_stride groups) decoded into
+// this rank's output. With a single output there is no tile to share between
+// stores, so each thread decodes 8-element chunks straight from registers:
+// the loads of U chunks (code word and parameter word each) are issued
+// together, then each chunk leaves in one 16-byte streaming store. Chunk c
+// covers elements [8c, 8c + 8) of group c / (GROUP/8). A CTA walks tiles of
+// U * blockDim consecutive chunks, so a thread's chunks only move forward:
+// the owner of a group is found by advancing an index over the segment
+// starts kept in shared memory (no division per chunk).
+constexpr int kDecodeThreads = 256;
+constexpr int kDecodeUnroll = 8;
+
+template <int GROUP, int BITS, int QM>
+__global__ void __launch_bounds__(kDecodeThreads) k_decode_rank(const Args a) {
+    constexpr int L = GROUP / 8, CB = GROUP * BITS / 8, U = kDecodeUnroll;
+    __shared__ long long seg_start[ECHO_MAX_RANKS + 1];
+    for (int s = threadIdx.x; s <= a.P; s += blockDim.x) seg_start[s] = (long long)s * a.G / a.P;
+    __syncthreads();
+    const long long c_begin = a.c0 * L, c_end = a.c1 * L;   // the window's full groups
+    const long long tile_chunks = (long long)U * blockDim.x;
+    int o = 0;
+    for (long long base = c_begin + blockIdx.x * tile_chunks; base < c_end; base += gridDim.x * tile_chunks) {
+        uint2 w[U];
+        uint32_t pw[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const long long c = base + u * blockDim.x + threadIdx.x;
+            w[u] = make_uint2(0u, 0u);
+            pw[u] = 0u;
+            if (c < c_end) {
+                const long long j = c / L;
+                while (j >= seg_start[o + 1]) ++o;
+                const size_t gs = (size_t)((long long)o * a.g_seg_stride + j - seg_start[o]);
+                w[u] = load_codes8<BITS>(a.g_codes + gs * CB, (int)(c % L));
+                pw[u] = a.g_params[gs];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const long long c = base + u * blockDim.x + threadIdx.x;
+            if (c < c_end) {
+                const uint4 y = decode8_bf16<BITS, QM>(w[u], pw[u]);
+                for (int r = a.out_lo; r < a.out_hi; ++r) __stcs(reinterpret_cast<uint4*>(a.out[r] + 8 * c), y);
+            }
+        }
+    }
+    // the partial last group (not a multiple of 16 bytes): guarded stores
+    if (a.tail && blockIdx.x == gridDim.x - 1 && threadIdx.x < L) {
+        const long long j = a.G - 1;
+        const size_t gs = g_read_slot(a, j);
+        const uint2 w = load_codes8<BITS>(a.g_codes + gs * CB, threadIdx.x);
+        const uint4 v = decode8_bf16<BITS, QM>(w, a.g_params[gs]);
+        const uint32_t yb[4] = {v.x, v.y, v.z, v.w};
+        const long long e = j * GROUP + 8 * threadIdx.x;
+        for (int r = a.out_lo; r < a.out_hi; ++r) {
 #pragma unroll
             for (int k = 0; k < 8; ++k)
                 if (e + k < a.n) a.out[r][e + k] = (uint16_t)(yb[k >> 1] >> (16 * (k & 1)));

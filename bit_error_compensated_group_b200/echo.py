@@ -48,6 +48,27 @@ class EchoLayout(ctypes.Structure):
     ]
 
 
+class EchoRankLayout(ctypes.Structure):
+    _fields_ = [
+        ("groups", ctypes.c_int64),
+        ("seg_begin", ctypes.c_int64),
+        ("seg_groups", ctypes.c_int64),
+        ("seg_max", ctypes.c_int64),
+        ("code_bytes", ctypes.c_uint64),
+        ("flags_offset", ctypes.c_uint64),
+        ("send_codes_offset", ctypes.c_uint64),
+        ("send_params_offset", ctypes.c_uint64),
+        ("recv_codes_offset", ctypes.c_uint64),
+        ("recv_params_offset", ctypes.c_uint64),
+        ("gsend_codes_offset", ctypes.c_uint64),
+        ("gsend_params_offset", ctypes.c_uint64),
+        ("grecv_codes_offset", ctypes.c_uint64),
+        ("grecv_params_offset", ctypes.c_uint64),
+        ("workspace_bytes", ctypes.c_uint64),
+        ("state_bytes", ctypes.c_uint64),
+    ]
+
+
 def lib() -> ctypes.CDLL:
     """Load the CUDA library; raises if it was not built."""
     global _lib
@@ -84,6 +105,16 @@ def lib() -> ctypes.CDLL:
         L.echo_get_status.restype = I
         L.echo_set_quantizer.argtypes = [V, I]
         L.echo_set_quantizer.restype = I
+        L.echo_query_rank_layout.argtypes = [I64, I, I, I, I, I, ctypes.POINTER(EchoRankLayout)]
+        L.echo_query_rank_layout.restype = I
+        L.echo_init_rank.argtypes = [ctypes.POINTER(V), I64, I, I, I, I, V, V, V]
+        L.echo_init_rank.restype = I
+        L.echo_rank_quantize.argtypes = [V, V, I, F, F, F, F, V]
+        L.echo_rank_quantize.restype = I
+        L.echo_rank_reduce.argtypes = [V, V, V, I, F, F, F, F, V]
+        L.echo_rank_reduce.restype = I
+        L.echo_rank_decode.argtypes = [V, V, I, V]
+        L.echo_rank_decode.restype = I
         L.echo_free.argtypes = [V]
         L.echo_free.restype = I
         L.echo_status_string.argtypes = [I]
@@ -284,6 +315,154 @@ class EchoAllReduce:
         g_c = ws[L.gather_codes_offset:L.gather_codes_offset + G * cb].view(G, cb)
         g_p = ws[L.gather_params_offset:L.gather_params_offset + G * 4].view(torch.int32)
         return a2a_c, a2a_p, g_c, g_p
+
+    def status(self, stream=None):
+        return echo_get_status(self.handle, stream)
+
+    def close(self) -> None:
+        if self.handle is not None:
+            echo_free(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+# ----------------------------------------------------------------- one rank of a multi-GPU call
+
+def echo_query_rank_layout(n: int, P: int, rank: int, group: int, max_bits: int, bits: int) -> EchoRankLayout:
+    out = EchoRankLayout()
+    _check(lib().echo_query_rank_layout(n, P, rank, group, max_bits, bits, ctypes.byref(out)),
+           "echo_query_rank_layout")
+    return out
+
+
+def echo_init_rank(n: int, P: int, rank: int, group: int, max_bits: int, state, workspace,
+                   stream=None) -> ctypes.c_void_p:
+    h = ctypes.c_void_p()
+    _check(lib().echo_init_rank(ctypes.byref(h), n, P, rank, group, max_bits, _ptr(state), _ptr(workspace),
+                                _stream(stream)), "echo_init_rank")
+    return h
+
+
+def echo_rank_quantize(x, st, bits: int, eta: float, alpha_long: float, alpha_short: float, w: float,
+                       stream=None) -> None:
+    _check(lib().echo_rank_quantize(_ptr(x), st, bits, eta, alpha_long, alpha_short, w, _stream(stream)),
+           "echo_rank_quantize")
+
+
+def echo_rank_reduce(x, out, st, bits: int, eta: float, alpha_long: float, alpha_short: float, w: float,
+                     stream=None) -> None:
+    _check(lib().echo_rank_reduce(_ptr(x), _ptr(out), st, bits, eta, alpha_long, alpha_short, w, _stream(stream)),
+           "echo_rank_reduce")
+
+
+def echo_rank_decode(out, st, bits: int, stream=None) -> None:
+    _check(lib().echo_rank_decode(_ptr(out), st, bits, _stream(stream)), "echo_rank_decode")
+
+
+class ExchangePlan:
+    """Views of one rank's workspace for the two exchanges of a multi-GPU
+    call and their split sizes, in the argument order of
+    torch.distributed.all_to_all_single / all_gather_into_tensor. Built from
+    the library's layouts alone, so it serves a workspace on any device."""
+
+    def __init__(self, workspace: torch.Tensor, n: int, P: int, rank: int, group: int, max_bits: int, bits: int):
+        L = echo_query_rank_layout(n, P, rank, group, max_bits, bits)
+        segs = [int(echo_query_rank_layout(n, P, s, group, max_bits, bits).seg_groups) for s in range(P)]
+        G, seg, sm, cb = int(L.groups), int(L.seg_groups), int(L.seg_max), int(L.code_bytes)
+        ws = workspace
+
+        def u8(off, nbytes):
+            return ws[int(off):int(off) + nbytes]
+
+        def i32(off, count):
+            return ws[int(off):int(off) + 4 * count].view(torch.int32)
+
+        self.layout = L
+        self.send_codes = u8(L.send_codes_offset, G * cb)
+        self.send_params = i32(L.send_params_offset, G)
+        self.recv_codes = u8(L.recv_codes_offset, P * seg * cb)
+        self.recv_params = i32(L.recv_params_offset, P * seg)
+        self.codes_in_splits = [g * cb for g in segs]      # to owner s: its segment of this rank's row
+        self.codes_out_splits = [seg * cb] * P             # from every rank: this owner's segment
+        self.params_in_splits = list(segs)
+        self.params_out_splits = [seg] * P
+        self.gsend_codes = u8(L.gsend_codes_offset, sm * cb)
+        self.gsend_params = i32(L.gsend_params_offset, sm)
+        self.grecv_codes = u8(L.grecv_codes_offset, P * sm * cb)
+        self.grecv_params = i32(L.grecv_params_offset, P * sm)
+
+
+def exchange_all_to_all(plan: ExchangePlan, group=None) -> None:
+    """The all-to-all of the packed payload (codes and parameters)."""
+    import torch.distributed as dist
+    dist.all_to_all_single(plan.recv_codes, plan.send_codes, plan.codes_out_splits, plan.codes_in_splits,
+                           group=group)
+    dist.all_to_all_single(plan.recv_params, plan.send_params, plan.params_out_splits, plan.params_in_splits,
+                           group=group)
+
+
+def exchange_all_gather(plan: ExchangePlan, group=None) -> None:
+    """The all-gather of the owners' requantized segments."""
+    import torch.distributed as dist
+    dist.all_gather_into_tensor(plan.grecv_codes, plan.gsend_codes, group=group)
+    dist.all_gather_into_tensor(plan.grecv_params, plan.gsend_params, group=group)
+
+
+class EchoRank:
+    """One rank of a multi-GPU Echo all-reduce (one process per GPU): owns,
+    through torch, this rank's EMA state and workspace, and the library
+    handle. `allreduce` runs the five steps with torch.distributed
+    collectives between the kernels (NCCL for CUDA tensors)."""
+
+    def __init__(self, n: int, P: int, rank: int, group: int = 128, max_bits: int = 4, feedback: bool = True,
+                 device=None, stream=None, quantizer: int = ECHO_QUANT_DIRECTED):
+        device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        self.n, self.P, self.rank, self.group, self.max_bits = n, P, rank, group, max_bits
+        L = echo_query_rank_layout(n, P, rank, group, max_bits, max_bits)
+        self.workspace = torch.empty(int(L.workspace_bytes), dtype=torch.uint8, device=device)
+        self.state = torch.empty(int(L.state_bytes) // 4, dtype=torch.float32, device=device) if feedback else None
+        self.handle = echo_init_rank(n, P, rank, group, max_bits, self.state, self.workspace, stream)
+        if quantizer != ECHO_QUANT_DIRECTED:
+            echo_set_quantizer(self.handle, quantizer)
+        self._plans = {}
+
+    def plan(self, bits: int) -> ExchangePlan:
+        if bits not in self._plans:
+            self._plans[bits] = ExchangePlan(self.workspace, self.n, self.P, self.rank, self.group, self.max_bits,
+                                             bits)
+        return self._plans[bits]
+
+    def quantize(self, x, bits=4, eta=1.0, alpha_long=0.05, alpha_short=0.5, w=0.5, stream=None) -> None:
+        echo_rank_quantize(x, self.handle, bits, eta, alpha_long, alpha_short, w, stream)
+
+    def reduce(self, x, out, bits=4, eta=1.0, alpha_long=0.05, alpha_short=0.5, w=0.5, stream=None) -> None:
+        echo_rank_reduce(x, out, self.handle, bits, eta, alpha_long, alpha_short, w, stream)
+
+    def decode(self, out, bits=4, stream=None) -> None:
+        echo_rank_decode(out, self.handle, bits, stream)
+
+    def allreduce(self, x, out, bits=4, eta=1.0, alpha_long=0.05, alpha_short=0.5, w=0.5, group=None) -> None:
+        """Steps 1-5 on torch's current stream, with the process group's
+        collectives in between (every rank of the group calls this)."""
+        fb = (eta, alpha_long, alpha_short, w)
+        self.quantize(x, bits, *fb)
+        if self.P > 1:
+            exchange_all_to_all(self.plan(bits), group)
+        self.reduce(x, out, bits, *fb)
+        if self.P > 1:
+            exchange_all_gather(self.plan(bits), group)
+            self.decode(out, bits)
+
+    def ema_views(self):
+        """(e_long [n], e_short [n]) of this rank."""
+        S = -(-self.n // self.group) * self.group
+        st = self.state.view(2, S)
+        return st[0, :self.n], st[1, :self.n]
 
     def status(self, stream=None):
         return echo_get_status(self.handle, stream)

@@ -372,6 +372,101 @@ ECHO_API int echo_allreduce_sim_noalloc(const void* const* inputs, void* const* 
                                         int64_t n, int P, int bits, int group, float eta, float alpha_long,
                                         float alpha_short, float w, uint32_t* flags_out, echo_stream_t stream);
 
+/*
+ * ------------------------------------------------------------------------
+ * One rank of a multi-GPU call: one process (or one handle) per GPU, P ranks.
+ *
+ * The same restructured all-reduce ([EXP] mechanism 1) with the transport
+ * between the phases done by the caller's collectives (NCCL through
+ * torch.distributed, say) instead of shared device memory:
+ *   1. echo_rank_quantize   phases 1, 2, 5 for this rank's non-owned groups:
+ *                           fills its all-to-all send row
+ *   2. all-to-all           (caller) send row -> every owner's receive rows
+ *   3. echo_rank_reduce     phases 1, 3, 5 for this rank's own segment: sums
+ *                           its x' and the P-1 received payloads in rank order,
+ *                           requantizes into its all-gather send buffer
+ *   4. all-gather           (caller) every rank's send buffer -> receive rows
+ *   5. echo_rank_decode     phase 4: decodes every gathered segment into this
+ *                           rank's output
+ * The arithmetic is that of echo_allreduce_sim: P ranks running this
+ * sequence produce, bit for bit, the simulation's outputs, payloads and EMA
+ * state (rank r holding rows r of the simulation's [P][2][S] state).
+ *
+ * Workspace of one rank (byte offsets; code regions sized for max_bits, laid
+ * out with code_bytes = group * bits / 8 of the call):
+ *   send codes   [G][code_bytes], send params [G] (uint32 {s, z} words):
+ *                this rank's payload for group j at j; the part for owner s
+ *                is groups [seg_begin(s), seg_begin(s) + seg_groups(s)),
+ *                i.e. seg_groups(s) * code_bytes bytes at
+ *                seg_begin(s) * code_bytes (params: seg_groups(s) words at
+ *                seg_begin(s)). The part for this rank itself is written and
+ *                never read.
+ *   recv codes   [P][seg_groups][code_bytes], recv params [P][seg_groups]:
+ *                what rank r sent to this owner, at r * seg_groups groups.
+ *                An all-to-all with these splits (send counts seg_groups(s),
+ *                receive counts seg_groups of this rank from every rank) fills
+ *                it; torch.distributed.all_to_all_single does.
+ *   gsend codes  [seg_max][code_bytes], gsend params [seg_max]: this owner's
+ *                requantized segment (the first seg_groups entries).
+ *   grecv codes  [P][seg_max][code_bytes], grecv params [P][seg_max]: every
+ *                owner's gsend, in rank order: an all-gather of gsend.
+ * segment s = groups [floor(s G / P), floor((s + 1) G / P)); seg_max = the
+ * largest segment.
+ */
+typedef struct echo_rank_layout {
+    int64_t groups;               /* G = ceil(n / group) */
+    int64_t seg_begin;            /* first group this rank owns */
+    int64_t seg_groups;           /* groups this rank owns (may be 0 when G < P) */
+    int64_t seg_max;              /* largest segment of any rank */
+    uint64_t code_bytes;          /* group * bits / 8 */
+    uint64_t flags_offset;
+    uint64_t send_codes_offset;
+    uint64_t send_params_offset;
+    uint64_t recv_codes_offset;
+    uint64_t recv_params_offset;
+    uint64_t gsend_codes_offset;
+    uint64_t gsend_params_offset;
+    uint64_t grecv_codes_offset;
+    uint64_t grecv_params_offset;
+    uint64_t workspace_bytes;     /* for max_bits */
+    uint64_t state_bytes;         /* this rank's two EMAs: float32 [2][S] */
+} echo_rank_layout;
+
+/* Fill *out for rank `rank` (0 <= rank < P) and a call with `bits`.
+ * Host-only. ECHO_EINVAL on bad sizes. */
+ECHO_API int echo_query_rank_layout(int64_t n, int P, int rank, int group, int max_bits, int bits,
+                                    echo_rank_layout* out);
+
+/*
+ * Handle of one rank. Arguments as for echo_init_state, with
+ *   rank       this rank, 0 <= rank < P
+ *   state_dev  NULL (no feedback) or device memory of
+ *              echo_query_rank_layout(...).state_bytes, 16-byte aligned:
+ *              this rank's long EMA then short EMA (S floats each)
+ *   workspace_dev  device memory of workspace_bytes, 256-byte aligned
+ * The state and the whole workspace are zeroed on `stream`. The handle
+ * serves only the echo_rank_* calls (and echo_set_quantizer,
+ * echo_get_status, echo_check_watchdog, echo_free); the simulation's calls
+ * return ECHO_EINVAL for it.
+ */
+ECHO_API int echo_init_rank(echo_state** out, int64_t n, int P, int rank, int group, int max_bits,
+                            void* state_dev, void* workspace_dev, echo_stream_t stream);
+
+/* Step 1 on this rank: x = its n bf16 inputs (device, 16-byte aligned).
+ * Nothing to do when P == 1. Errors as for echo_allreduce_sim. */
+ECHO_API int echo_rank_quantize(const void* x, echo_state* st, int bits, float eta, float alpha_long,
+                                float alpha_short, float w, echo_stream_t stream);
+
+/* Step 3 on this rank, after the all-to-all has filled its receive rows: x =
+ * the same inputs as step 1. When P == 1 it also writes the result into
+ * `out` (n bf16, required then); otherwise `out` is ignored (may be NULL). */
+ECHO_API int echo_rank_reduce(const void* x, void* out, echo_state* st, int bits, float eta, float alpha_long,
+                              float alpha_short, float w, echo_stream_t stream);
+
+/* Step 5 on this rank, after the all-gather has filled its gathered rows:
+ * writes the reduced result (n bf16) into `out`. Nothing to do when P == 1. */
+ECHO_API int echo_rank_decode(void* out, echo_state* st, int bits, echo_stream_t stream);
+
 /* Release the host handle and the events echo_allreduce_sim_host created
  * for it (never the caller's device buffers). NULL is a no-op. */
 ECHO_API int echo_free(echo_state* st);

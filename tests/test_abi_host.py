@@ -118,3 +118,45 @@ def test_no_gpu_fails_loudly(L):
     with pytest.raises(E.EchoError) as ei:
         E.echo_init_state(1024, 2, 128, 4, None, 4096, stream=0)
     assert ei.value.status == E.ECHO_ECUDA
+
+
+@pytest.mark.parametrize("n,P,g,mb,bits", [(1000, 3, 64, 8, 4), (1 << 29, 8, 128, 4, 4), (3 * 128, 4, 128, 4, 4),
+                                           (777, 5, 32, 8, 8), (1, 2, 32, 4, 4)])
+def test_rank_layout(L, n, P, g, mb, bits):
+    """One rank's layout of a multi-GPU call: the segments tile [0, G) in rank
+    order, seg_max is the largest, and the workspace regions are 256-byte
+    aligned, disjoint and as large as the exchange needs."""
+    G = _G(n, g)
+    cb, cbm = g * bits // 8, g * mb // 8
+    lays = [E.echo_query_rank_layout(n, P, r, g, mb, bits) for r in range(P)]
+    begin = 0
+    for r, lay in enumerate(lays):
+        assert lay.groups == G and lay.code_bytes == cb
+        assert lay.seg_begin == begin == r * G // P
+        assert lay.seg_groups == (r + 1) * G // P - r * G // P
+        begin += lay.seg_groups
+        assert lay.seg_max == max(l.seg_groups for l in lays)
+        assert lay.state_bytes == 2 * G * g * 4
+        seg, sm = lay.seg_groups, lay.seg_max
+        regions = [(lay.flags_offset, 4), (lay.send_codes_offset, G * cbm), (lay.send_params_offset, G * 4),
+                   (lay.recv_codes_offset, P * seg * cbm), (lay.recv_params_offset, P * seg * 4),
+                   (lay.gsend_codes_offset, sm * cbm), (lay.gsend_params_offset, sm * 4),
+                   (lay.grecv_codes_offset, P * sm * cbm), (lay.grecv_params_offset, P * sm * 4)]
+        for (o1, s1), (o2, _) in zip(regions, regions[1:]):
+            assert o1 % 256 == 0 and o1 + s1 <= o2
+        assert regions[-1][0] + regions[-1][1] <= lay.workspace_bytes
+    assert begin == G
+
+
+def test_rank_calls_reject_bad_arguments(L):
+    lay = E.EchoRankLayout()
+    assert L.echo_query_rank_layout(1000, 3, 3, 64, 4, 4, ctypes.byref(lay)) == E.ECHO_EINVAL   # rank >= P
+    assert L.echo_query_rank_layout(1000, 3, -1, 64, 4, 4, ctypes.byref(lay)) == E.ECHO_EINVAL
+    assert L.echo_query_rank_layout(1000, 3, 0, 64, 4, 8, ctypes.byref(lay)) == E.ECHO_EINVAL   # bits > max_bits
+    h = ctypes.c_void_p()
+    assert L.echo_init_rank(ctypes.byref(h), 1000, 3, 5, 64, 4, None, 4096, None) == E.ECHO_EINVAL
+    assert L.echo_init_rank(ctypes.byref(h), 1000, 3, 1, 64, 4, None, 4096 + 8, None) == E.ECHO_EINVAL
+    assert L.echo_rank_quantize(4096, None, 4, 1.0, 0.05, 0.5, 0.5, None) == E.ECHO_EINVAL
+    assert L.echo_rank_reduce(4096, 4096, None, 4, 1.0, 0.05, 0.5, 0.5, None) == E.ECHO_EINVAL
+    assert L.echo_rank_decode(4096, None, 4, None) == E.ECHO_EINVAL
+    assert h.value is None

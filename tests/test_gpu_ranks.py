@@ -1,0 +1,138 @@
+"""One rank per handle (the multi-GPU call's kernels) against the oracle, on
+one GPU.
+
+P EchoRank objects stand for the P GPUs. The two exchanges are emulated
+in-process with stream-ordered copies that follow the same ExchangePlan
+views and split sizes that torch.distributed receives on real GPUs
+(all_to_all_single: chunk `dst` of the sender's input goes to chunk `src` of
+the receiver's output; all_gather_into_tensor: rank order). Kernels run one
+after another on one stream; none waits on another. Checked bit for bit
+against the oracle's whole call: every rank's output, its EMA rows, its
+all-to-all send row (non-owned groups) and every owner's requantized
+segment, over two calls with carried state.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import bit_error_compensated_group_b200 as E
+from parity import Params, padded, random_inputs, seeded_state, u16
+
+pytestmark = pytest.mark.gpu
+
+
+def emulate_all_to_all(plans):
+    for dst, pd in enumerate(plans):
+        for src, ps in enumerate(plans):
+            for send, recv, ins, outs in ((ps.send_codes, pd.recv_codes, ps.codes_in_splits, pd.codes_out_splits),
+                                          (ps.send_params, pd.recv_params, ps.params_in_splits,
+                                           pd.params_out_splits)):
+                ln = ins[dst]
+                assert ln == outs[src]
+                a, b = sum(ins[:dst]), sum(outs[:src])
+                recv[b:b + ln].copy_(send[a:a + ln])
+
+
+def emulate_all_gather(plans):
+    for pd in plans:
+        for s, ps in enumerate(plans):
+            for send, recv in ((ps.gsend_codes, pd.grecv_codes), (ps.gsend_params, pd.grecv_params)):
+                k = send.numel()
+                recv[s * k:(s + 1) * k].copy_(send)
+
+
+CASES = [
+    # P, n, group, bits, feedback, quantizer
+    (2, 4096, 128, 4, True, O.Q_DIRECTED),
+    (3, 1000, 64, 8, True, O.Q_DIRECTED),
+    (8, 8192 * 3 + 77, 128, 4, True, O.Q_DIRECTED),    # partial last group
+    (8, 8192 * 3 + 77, 128, 4, False, O.Q_DIRECTED),
+    (4, 3 * 128, 128, 4, True, O.Q_DIRECTED),          # G < P: a rank owns nothing
+    (1, 5000, 128, 4, True, O.Q_DIRECTED),             # one rank: nothing exchanged
+    (5, 148 * 8 * 256 + 37, 256, 8, True, O.Q_DIRECTED),
+    (8, 50000, 32, 4, True, O.Q_NEAREST),
+    (6, 70001, 64, 4, True, O.Q_INT_ZERO),
+]
+
+
+@pytest.mark.parametrize("P,n,group,bits,feedback,quantizer", CASES)
+def test_ranks_match_the_oracle(P, n, group, bits, feedback, quantizer):
+    p = Params(bits=bits, group=group, w=0.3, alpha_long=0.1, alpha_short=0.6, quantizer=quantizer)
+    fb = (p.eta, p.alpha_long, p.alpha_short, p.w)
+    G = -(-n // group)
+    ld = G * group
+    ranks = [E.EchoRank(n, P, r, group, max(bits, 4), feedback, quantizer=quantizer) for r in range(P)]
+    try:
+        x = random_inputs(P, n, 17 * P + n, 2.0)
+        xs = [x[r].cuda() for r in range(P)]
+        outs = [torch.empty_like(t) for t in xs]
+        el = es = None
+        if feedback:
+            el0, es0 = seeded_state(P, n, n + 5 * P)
+            for r in range(P):
+                L, S = ranks[r].ema_views()
+                L.copy_(torch.from_numpy(el0[r]))
+                S.copy_(torch.from_numpy(es0[r]))
+            el, es = padded(el0, ld), padded(es0, ld)
+        plans = [rk.plan(bits) for rk in ranks]
+        xb = padded(u16(x), ld)
+        for call in range(2):
+            for r in range(P):
+                ranks[r].quantize(xs[r], bits, *fb)
+            emulate_all_to_all(plans)
+            for r in range(P):
+                ranks[r].reduce(xs[r], outs[r], bits, *fb)
+            emulate_all_gather(plans)
+            for r in range(P):
+                ranks[r].decode(outs[r], bits)
+            orc = O.echo_allreduce(xb, n_total=n, group=group, bits=bits, e_long=el, e_short=es, eta=p.eta,
+                                   alpha_long=p.alpha_long, alpha_short=p.alpha_short, w=p.w, quantizer=quantizer)
+            flags = 0
+            for rk in ranks:
+                flags |= rk.status()[1]
+            assert flags == orc.flags
+            for r in range(P):
+                assert np.array_equal(u16(outs[r]), orc.y[r, :n]), f"call {call}: output of rank {r}"
+                if feedback:
+                    L, S = ranks[r].ema_views()
+                    assert np.array_equal(L.cpu().numpy(), el[r, :n]), f"call {call}: e_long of rank {r}"
+                    assert np.array_equal(S.cpu().numpy(), es[r, :n]), f"call {call}: e_short of rank {r}"
+            cb = group * bits // 8
+            for r in range(P):
+                pl = plans[r]
+                send_c = pl.send_codes.cpu().numpy().reshape(G, cb)
+                send_p = pl.send_params.cpu().numpy().view(np.uint16).reshape(G, 2)
+                owned = [O.owner(j, G, P) == r for j in range(G)]
+                for j in range(G):
+                    if not owned[j]:
+                        assert np.array_equal(send_c[j], orc.a2a_codes[r, j]), f"a2a codes r={r} j={j}"
+                        assert np.array_equal(send_p[j], orc.a2a_params[r, j]), f"a2a params r={r} j={j}"
+                if P >= 2:
+                    b0, seg = int(pl.layout.seg_begin), int(pl.layout.seg_groups)
+                    g_c = pl.gsend_codes.cpu().numpy()[:seg * cb].reshape(seg, cb)
+                    g_p = pl.gsend_params.cpu().numpy()[:seg].view(np.uint16).reshape(seg, 2)
+                    assert np.array_equal(g_c, orc.gather_codes[b0:b0 + seg]), f"gather codes of owner {r}"
+                    assert np.array_equal(g_p, orc.gather_params[b0:b0 + seg]), f"gather params of owner {r}"
+            # the next call reduces the result again
+            xs = [o.clone() for o in outs]
+            xb = padded(orc.y[:, :n].copy(), ld)
+    finally:
+        for rk in ranks:
+            rk.close()
+
+
+def test_rank_and_simulation_handles_do_not_mix():
+    rk = E.EchoRank(4096, 2, 0)
+    ar = E.EchoAllReduce(4096, 2)
+    try:
+        x = torch.zeros(4096, dtype=torch.bfloat16, device="cuda")
+        with pytest.raises(E.EchoError) as ei:
+            E.echo_allreduce_sim([x, x], [x, x], rk.handle, 4096, 2, 4, 128, 1.0, 0.05, 0.5, 0.5)
+        assert ei.value.status == E.ECHO_EINVAL
+        with pytest.raises(E.EchoError) as ei:
+            E.echo_rank_quantize(x, ar.handle, 4, 1.0, 0.05, 0.5, 0.5)
+        assert ei.value.status == E.ECHO_EINVAL
+    finally:
+        rk.close()
+        ar.close()

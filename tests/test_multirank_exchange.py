@@ -1,0 +1,97 @@
+"""The exchanges of a multi-GPU call on CPU ranks (gloo): the all-to-all and
+all-gather that EchoRank.allreduce runs between its kernels, over the
+workspace views and split sizes of ExchangePlan (the library's rank
+layout). Every byte a rank sends is tagged with (sender, group, byte), so
+the test checks that each owner receives exactly the payload of its segment
+from every rank, in rank order, and every rank every owner's requantized
+segment. No kernel runs here; the kernels' side of the same layout is
+checked against the oracle on the GPU (tests/test_gpu_ranks.py)."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _tag_codes(r, j, cb):
+    """Codes byte b of group j sent by rank r."""
+    return (torch.arange(cb, dtype=torch.int64) * 7 + 31 * j + 101 * r) % 251
+
+
+def _tag_param(r, j):
+    return 1_000_000 * (r + 1) + j
+
+
+def _worker(rank, world, port, n, group, bits, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bit_error_compensated_group_b200 as E
+    from datetime import timedelta
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        P = world
+        L = E.echo_query_rank_layout(n, P, rank, group, 8, bits)
+        ws = torch.zeros(int(L.workspace_bytes), dtype=torch.uint8)
+        plan = E.ExchangePlan(ws, n, P, rank, group, 8, bits)
+        G, cb = int(L.groups), int(L.code_bytes)
+        lay = [E.echo_query_rank_layout(n, P, s, group, 8, bits) for s in range(P)]
+        # this rank's send row: every group j
+        for j in range(G):
+            plan.send_codes[j * cb:(j + 1) * cb] = _tag_codes(rank, j, cb).to(torch.uint8)
+            plan.send_params[j] = _tag_param(rank, j)
+        seg, b0, sm = int(L.seg_groups), int(L.seg_begin), int(L.seg_max)
+        for k in range(seg):
+            plan.gsend_codes[k * cb:(k + 1) * cb] = _tag_codes(rank, b0 + k, cb).to(torch.uint8) ^ 0x55
+            plan.gsend_params[k] = -_tag_param(rank, b0 + k)
+        E.exchange_all_to_all(plan)
+        E.exchange_all_gather(plan)
+        bad = []
+        for r in range(P):
+            for k in range(seg):
+                j = b0 + k
+                got = plan.recv_codes[(r * seg + k) * cb:(r * seg + k + 1) * cb].to(torch.int64)
+                if not torch.equal(got, _tag_codes(r, j, cb)):
+                    bad.append(("a2a codes", r, j))
+                if int(plan.recv_params[r * seg + k]) != _tag_param(r, j):
+                    bad.append(("a2a params", r, j))
+        for s in range(P):
+            sb, ss = int(lay[s].seg_begin), int(lay[s].seg_groups)
+            for k in range(ss):
+                got = plan.grecv_codes[(s * sm + k) * cb:(s * sm + k + 1) * cb].to(torch.int64)
+                if not torch.equal(got, _tag_codes(s, sb + k, cb) ^ 0x55):
+                    bad.append(("gather codes", s, sb + k))
+                if int(plan.grecv_params[s * sm + k]) != -_tag_param(s, sb + k):
+                    bad.append(("gather params", s, sb + k))
+        q.put((rank, bad[:5], seg))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,n,group,bits", [
+    (3, 1000, 64, 4),        # G = 16: segments of 5, 5 and 6 groups
+    (2, 777, 32, 8),         # partial last group
+    (4, 3 * 128, 128, 4),    # G = 3 < P: one rank owns nothing
+])
+def test_exchange_delivers_each_segment(world, n, group, bits):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, n, group, bits, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+        assert p.exitcode == 0
+    got = sorted(q.get(timeout=5) for _ in range(world))
+    assert [g[0] for g in got] == list(range(world))
+    for rank, bad, seg in got:
+        assert bad == [], (rank, bad)
