@@ -654,6 +654,82 @@ def run_workloads(args):
     print(json.dumps({"workloads": out, "peak_gbs": peak, "peak_kind": peak_kind, "data": "synthetic"}), flush=True)
 
 
+def run_ranks(args):
+    """One rank's kernels of a real multi-GPU call (rank 0 of P = 8 on the
+    1 GB message), on one GPU: the P ranks' handles are set up on this GPU and
+    one call is run with the exchanges done in-process (so the payloads are
+    real), then rank 0's quantize / reduce / decode are timed. The exchanges
+    themselves are not timed (they need P GPUs); their bytes are printed."""
+    import torch
+    import workloads as W
+    import bit_error_compensated_group_b200 as E
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = _workload()
+    P, n, group, bits = w.P, w.n, w.group, w.bits
+    fb = (w.eta, w.alpha_long, w.alpha_short, w.w)
+    peak, peak_kind = _peak_hbm()
+    G = -(-n // group)
+    pb = group * bits // 8 + 4
+    out = {}
+    for feedback in (True, False):
+        ranks = [E.EchoRank(n, P, r, group, bits, feedback, device=dev) for r in range(P)]
+        xs = [W.rank_input(w, r, 0, dev) for r in range(P)]
+        ys = [torch.empty_like(t) for t in xs]
+        plans = [rk.plan(bits) for rk in ranks]
+        for r in range(P):
+            ranks[r].quantize(xs[r], bits, *fb)
+        E.exchange_in_process(plans, "all_to_all")
+        for r in range(P):
+            ranks[r].reduce(xs[r], ys[r], bits, *fb)
+        E.exchange_in_process(plans, "all_gather")
+        for r in range(P):
+            ranks[r].decode(ys[r], bits)
+        torch.cuda.synchronize(dev)
+        r0 = ranks[0]
+        s = torch.cuda.current_stream(dev)
+        steps = max(3, args.steps)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+        for i in range(args.warmup + steps):
+            e = evs[i - args.warmup] if i >= args.warmup else None
+            if e:
+                e[0].record(s)
+            r0.quantize(xs[0], bits, *fb)
+            if e:
+                e[1].record(s)
+            r0.reduce(xs[0], ys[0], bits, *fb)
+            if e:
+                e[2].record(s)
+            r0.decode(ys[0], bits)
+            if e:
+                e[3].record(s)
+        torch.cuda.synchronize(dev)
+        ms = [sum(e[k].elapsed_time(e[k + 1]) for e in evs) / steps for k in range(3)]
+        seg = int(plans[0].layout.seg_groups)
+        st = 16 if feedback else 0
+        nbytes = [(G - seg) * (2 * group + st * group + pb),                        # x, EMAs, send row
+                  seg * (2 * group + st * group + (P - 1) * pb + pb),               # x, EMAs, received rows, gather send
+                  G * (pb + 2 * group)]                                            # gathered rows, output
+        rc, flags = r0.status()
+        out["feedback" if feedback else "no_feedback"] = {
+            "phases_ms": {"quantize": ms[0], "reduce": ms[1], "decode": ms[2]}, "ms": sum(ms),
+            "algorithmic_bytes": {"quantize": nbytes[0], "reduce": nbytes[1], "decode": nbytes[2]},
+            "roofline_frac": {k: b / (t * 1e-3) / 1e9 / peak for k, b, t in zip(("quantize", "reduce", "decode"),
+                                                                               nbytes, ms)},
+            "status": rc, "flags": flags}
+        for rk in ranks:
+            rk.close()
+        del ranks, xs, ys, plans
+        torch.cuda.empty_cache()
+    lay0 = E.echo_query_rank_layout(n, P, 0, group, bits, bits)
+    seg0, segm = int(lay0.seg_groups), int(lay0.seg_max)
+    print(json.dumps({"ranks": out, "config": {"workload": w.name, "P": P, "n": n, "group": group, "bits": bits,
+                                               "rank": 0},
+                      "exchange_bytes_per_rank": {"all_to_all_out": (G - seg0) * pb, "all_to_all_in": (P - 1) * seg0 * pb,
+                                                  "all_gather_in": (P - 1) * segm * pb},
+                      "peak_gbs": peak, "peak_kind": peak_kind, "data": "synthetic"}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -669,6 +745,8 @@ def main():
                     help="off: time the call without EMA state as the main step (profiling)")
     ap.add_argument("--ablation", action="store_true",
                     help="print the accuracy ablations on the synthetic chains instead of timing")
+    ap.add_argument("--ranks", action="store_true",
+                    help="print one rank's kernel times of a multi-GPU call (rank 0 of P = 8, 1 GB) instead")
     ap.add_argument("--workloads", action="store_true",
                     help="print every workload's GPU and oracle time per call instead of the main line")
     ap.add_argument("--tokens", type=int, default=None,
@@ -683,6 +761,8 @@ def main():
         run_ablation(args)
     elif args.workloads:
         run_workloads(args)
+    elif args.ranks:
+        run_ranks(args)
     else:
         run_gpu(args)
 

@@ -477,3 +477,31 @@ class EchoRank:
             self.close()
         except Exception:
             pass
+
+
+def exchange_in_process(plans: Sequence[ExchangePlan], step: str) -> None:
+    """Both exchanges for P ranks held by one process on one device (tests and
+    one-GPU benchmarks of the rank kernels): stream-ordered copies with the
+    semantics of all_to_all_single (`step` "all_to_all": chunk `dst` of the
+    sender's input into chunk `src` of the receiver's output) and of
+    all_gather_into_tensor (`step` "all_gather": rank order), over the same
+    views and split sizes the collectives receive."""
+    if step == "all_to_all":
+        for dst, pd in enumerate(plans):
+            for src, ps in enumerate(plans):
+                for send, recv, ins, outs in ((ps.send_codes, pd.recv_codes, ps.codes_in_splits, pd.codes_out_splits),
+                                              (ps.send_params, pd.recv_params, ps.params_in_splits,
+                                               pd.params_out_splits)):
+                    ln = ins[dst]
+                    if ln != outs[src]:
+                        raise ValueError("exchange plans of different messages")
+                    a, b = sum(ins[:dst]), sum(outs[:src])
+                    recv[b:b + ln].copy_(send[a:a + ln])
+    elif step == "all_gather":
+        for pd in plans:
+            for s, ps in enumerate(plans):
+                for send, recv in ((ps.gsend_codes, pd.grecv_codes), (ps.gsend_params, pd.grecv_params)):
+                    k = send.numel()
+                    recv[s * k:(s + 1) * k].copy_(send)
+    else:
+        raise ValueError(step)

@@ -23,23 +23,11 @@ pytestmark = pytest.mark.gpu
 
 
 def emulate_all_to_all(plans):
-    for dst, pd in enumerate(plans):
-        for src, ps in enumerate(plans):
-            for send, recv, ins, outs in ((ps.send_codes, pd.recv_codes, ps.codes_in_splits, pd.codes_out_splits),
-                                          (ps.send_params, pd.recv_params, ps.params_in_splits,
-                                           pd.params_out_splits)):
-                ln = ins[dst]
-                assert ln == outs[src]
-                a, b = sum(ins[:dst]), sum(outs[:src])
-                recv[b:b + ln].copy_(send[a:a + ln])
+    E.exchange_in_process(plans, "all_to_all")
 
 
 def emulate_all_gather(plans):
-    for pd in plans:
-        for s, ps in enumerate(plans):
-            for send, recv in ((ps.gsend_codes, pd.grecv_codes), (ps.gsend_params, pd.grecv_params)):
-                k = send.numel()
-                recv[s * k:(s + 1) * k].copy_(send)
+    E.exchange_in_process(plans, "all_gather")
 
 
 CASES = [
