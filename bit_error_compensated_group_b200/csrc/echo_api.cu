@@ -30,7 +30,6 @@ struct echo_state {
     cudaEvent_t ev[3];
     bool have_events;
     int rank;              // -1: the single-GPU simulation; else this rank of a multi-GPU call
-    echo_rank_layout rl;   // rank handles: the layout for max_bits
 };
 
 namespace {
@@ -97,8 +96,6 @@ int pipe_grid(K kernel, const echo_state* st, int smem) {
 
 enum class Stage { Quantize, Reduce, Gather };
 
-// One pipelined launch; `grid` caches the grid (and the shared-memory opt-in)
-// of this kernel instantiation.
 // An upper bound on the tiles a pipelined launch walks: the runs (2 per rank
 // for quantize, 1 per owner for reduce) cut into tiles of `tile_groups`.
 int64_t tile_bound(Stage stage, const echo_dev::Args& a, int tile_groups) {
@@ -108,10 +105,12 @@ int64_t tile_bound(Stage stage, const echo_dev::Args& a, int tile_groups) {
     return groups / tile_groups + runs + 1;
 }
 
-// A persistent launch never needs more CTAs than tiles: small messages then
-// start only the CTAs that have work.
-// `pdl`: launch as a programmatic dependent of the kernel before it on the
-// stream (the owners' pass right after this call's quantize pass).
+// One pipelined launch; `grids` caches, per device, the grid (and the
+// shared-memory opt-in) of this kernel instantiation. A persistent launch
+// never needs more CTAs than tiles: small messages then start only the CTAs
+// that have work. `pdl`: launch as a programmatic dependent of the kernel
+// before it on the stream (the owners' pass right after this call's quantize
+// pass).
 template <typename K>
 int launch_pipe(K kernel, int* grids, int64_t max_tiles, const echo_dev::Args& a, const echo_state* st,
                 cudaStream_t s, int smem, bool pdl = false) {
@@ -139,8 +138,8 @@ int launch_pipe(K kernel, int* grids, int64_t max_tiles, const echo_dev::Args& a
 template <int GROUP, int BITS, int QM>
 int launch_stage(Stage stage, const echo_dev::Args& a, const echo_state* st, cudaStream_t s, bool pdl) {
     int rc = ECHO_OK;
-    // tiles of 2048 elements with feedback; without, 4 x 2048 (quantize) and
-    // 5 x 2048 (reduce) -- the sub-tile counts of the kernels' RunWalkers
+    // tiles of kTileElems elements with feedback; without, the sub-tile
+    // counts of the kernels' RunWalkers (kQuantizeSubtilesNF, kReduceSubtilesNF)
     const int subtiles = a.state ? 1
                          : stage == Stage::Quantize ? echo_dev::kQuantizeSubtilesNF
                                                     : echo_dev::kReduceSubtilesNF;
@@ -642,7 +641,6 @@ int echo_init_rank(echo_state** out, int64_t n, int P, int rank, int group, int 
     st->quantizer = ECHO_QUANT_DIRECTED;
     st->have_events = false;
     st->rank = rank;
-    st->rl = L;
     *out = st;
     return ECHO_OK;
 }
