@@ -438,12 +438,24 @@ def run_gpu(args):
     # inputs copied in and the reduced result copied out, chunk by chunk on
     # two copy streams overlapping the kernels (echo_allreduce_sim_host)
     e2e = None
+    host_in = host_out = None
     if not args.no_e2e:
+        # every rank pins P + 1 message buffers; the leg runs only if all could
+        # (a collective decision, so that every rank takes the same steps)
+        why = None
+        try:
+            host_in = [torch.empty(n, dtype=torch.bfloat16, pin_memory=True) for _ in range(P)]
+            host_out = torch.empty(n, dtype=torch.bfloat16, pin_memory=True)
+        except (RuntimeError, MemoryError) as exc:
+            host_in = host_out = None
+            why = f"pinned host buffers: {exc}".splitlines()[0][:200]
+        if max_over_ranks(0.0 if why is None else 1.0, world, dev) > 0.0:
+            e2e = {"unavailable": why or "another rank could not pin its host buffers"}
+            host_in = host_out = None
+    if host_in is not None:
         e2e_steps = max(1, min(args.steps, 4))
-        host_in = [torch.empty(n, dtype=torch.bfloat16, pin_memory=True) for _ in range(P)]
         for r in range(P):
             host_in[r].copy_(inputs[r])
-        host_out = torch.empty(n, dtype=torch.bfloat16, pin_memory=True)
         cin, cout = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
         def e2e_step():
