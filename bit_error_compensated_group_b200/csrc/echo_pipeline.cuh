@@ -1180,19 +1180,28 @@ __global__ void __launch_bounds__(kGatherThreads) k_gather_tma(const Args a) {
 // Phase 4 on one rank of a multi-GPU call: every group of the gathered
 // payload (P owner segments, each padded to g_seg_stride groups) decoded into
 // this rank's output. With a single output there is no tile to share between
-// stores, so each thread decodes 8-element chunks straight from registers:
-// the loads of U chunks (code word and parameter word each) are issued
-// together, then each chunk leaves in one 16-byte streaming store. Chunk c
-// covers elements [8c, 8c + 8) of group c / (GROUP/8). A CTA walks tiles of
-// U * blockDim consecutive chunks, so a thread's chunks only move forward:
-// the owner of a group is found by advancing an index over the segment
-// starts kept in shared memory (no division per chunk).
+// stores, so each thread decodes E-element chunks straight from registers:
+// the loads of U chunks (code words and parameter word each) are issued
+// together, then each chunk leaves in one streaming store (32 bytes at
+// E = 16 when the output is 32-byte aligned, else 16-byte stores). Chunk c
+// covers elements [E c, E c + E) of group c / (GROUP / E). A CTA walks tiles
+// of U * blockDim consecutive chunks, so a thread's chunks only move
+// forward: the owner of a group is found by advancing an index over the
+// segment starts kept in shared memory (no division per chunk).
 constexpr int kDecodeThreads = 256;
 constexpr int kDecodeUnroll = 8;
+constexpr int kDecodeElems = 16;
+
+__device__ __forceinline__ void store_v8_cs(void* p, uint4 lo, uint4 hi) {
+    asm volatile("st.global.cs.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(lo.x), "r"(lo.y),
+                 "r"(lo.z), "r"(lo.w), "r"(hi.x), "r"(hi.y), "r"(hi.z), "r"(hi.w)
+                 : "memory");
+}
 
 template <int GROUP, int BITS, int QM>
 __global__ void __launch_bounds__(kDecodeThreads) k_decode_rank(const Args a) {
-    constexpr int L = GROUP / 8, CB = GROUP * BITS / 8, U = kDecodeUnroll;
+    constexpr int E = kDecodeElems, H = E / 8, L = GROUP / E, CB = GROUP * BITS / 8, U = kDecodeUnroll;
+    static_assert(E == 8 || E == 16, "chunk of 8 or 16 elements");
     __shared__ long long seg_start[ECHO_MAX_RANKS + 1];
     for (int s = threadIdx.x; s <= a.P; s += blockDim.x) seg_start[s] = (long long)s * a.G / a.P;
     __syncthreads();
@@ -1200,18 +1209,21 @@ __global__ void __launch_bounds__(kDecodeThreads) k_decode_rank(const Args a) {
     const long long tile_chunks = (long long)U * blockDim.x;
     int o = 0;
     for (long long base = c_begin + blockIdx.x * tile_chunks; base < c_end; base += gridDim.x * tile_chunks) {
-        uint2 w[U];
+        uint2 w[U][H];
         uint32_t pw[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const long long c = base + u * blockDim.x + threadIdx.x;
-            w[u] = make_uint2(0u, 0u);
+#pragma unroll
+            for (int h = 0; h < H; ++h) w[u][h] = make_uint2(0u, 0u);
             pw[u] = 0u;
             if (c < c_end) {
                 const long long j = c / L;
                 while (j >= seg_start[o + 1]) ++o;
                 const size_t gs = (size_t)((long long)o * a.g_seg_stride + j - seg_start[o]);
-                w[u] = load_codes8<BITS>(a.g_codes + gs * CB, (int)(c % L));
+                const uint8_t* codes = a.g_codes + gs * CB;
+#pragma unroll
+                for (int h = 0; h < H; ++h) w[u][h] = load_codes8<BITS>(codes, (int)(c % L) * H + h);
                 pw[u] = a.g_params[gs];
             }
         }
@@ -1219,13 +1231,23 @@ __global__ void __launch_bounds__(kDecodeThreads) k_decode_rank(const Args a) {
         for (int u = 0; u < U; ++u) {
             const long long c = base + u * blockDim.x + threadIdx.x;
             if (c < c_end) {
-                const uint4 y = decode8_bf16<BITS, QM>(w[u], pw[u]);
-                for (int r = a.out_lo; r < a.out_hi; ++r) __stcs(reinterpret_cast<uint4*>(a.out[r] + 8 * c), y);
+                uint4 y[H];
+#pragma unroll
+                for (int h = 0; h < H; ++h) y[h] = decode8_bf16<BITS, QM>(w[u][h], pw[u]);
+                for (int r = a.out_lo; r < a.out_hi; ++r) {
+                    uint16_t* dst = a.out[r] + (long long)E * c;
+                    if (E == 16 && (reinterpret_cast<uintptr_t>(a.out[r]) & 31) == 0) {
+                        store_v8_cs(dst, y[0], y[H - 1]);
+                    } else {
+#pragma unroll
+                        for (int h = 0; h < H; ++h) __stcs(reinterpret_cast<uint4*>(dst + 8 * h), y[h]);
+                    }
+                }
             }
         }
     }
     // the partial last group (not a multiple of 16 bytes): guarded stores
-    if (a.tail && blockIdx.x == gridDim.x - 1 && threadIdx.x < L) {
+    if (a.tail && blockIdx.x == gridDim.x - 1 && threadIdx.x < GROUP / 8) {
         const long long j = a.G - 1;
         const size_t gs = g_read_slot(a, j);
         const uint2 w = load_codes8<BITS>(a.g_codes + gs * CB, threadIdx.x);
