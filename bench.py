@@ -742,6 +742,68 @@ def run_ranks(args):
                       "peak_gbs": peak, "peak_kind": peak_kind, "data": "synthetic"}), flush=True)
 
 
+def run_dist(args):
+    """The real multi-GPU call against NCCL's bf16 all-reduce (the pages'
+    comparison): under torchrun, P = world size, one rank per GPU, each with
+    its own 1 GB bf16 message (the same workload as the main line; rank r's
+    input is the workload's rank r). Times, on each rank's stream and as the
+    max over ranks, EchoRank.allreduce with and without feedback and
+    torch.distributed.all_reduce (SUM) of the same bf16 tensor."""
+    import torch
+    import torch.distributed as dist
+    import workloads as W
+    import bit_error_compensated_group_b200 as E
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from datetime import timedelta
+    if not dist.is_initialized():
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    w = _workload()
+    n, group, bits = w.n, w.group, w.bits
+    fb = (w.eta, w.alpha_long, w.alpha_short, w.w)
+    x = W.rank_input(w, rank % w.P, 0, dev)
+    y = torch.empty_like(x)
+    s = torch.cuda.current_stream(dev)
+    steps = max(3, args.steps)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s)
+        for _ in range(steps):
+            fn()
+        b.record(s)
+        torch.cuda.synchronize(dev)
+        dist.barrier()
+        return max_over_ranks(a.elapsed_time(b) / steps, world, dev)
+
+    out = {}
+    for feedback in (True, False):
+        er = E.EchoRank(n, world, rank, group, bits, feedback, device=dev)
+        out["echo_feedback" if feedback else "echo_no_feedback"] = timed(lambda: er.allreduce(x, y, bits, *fb))
+        rc, flags = er.status()
+        er.close()
+        del er
+        torch.cuda.empty_cache()
+    z = x.clone()
+    out["nccl_bf16_all_reduce"] = timed(lambda: dist.all_reduce(z))
+    if rank == 0:
+        line = {"dist": {k: {"ms_per_call": v, "gbs_bf16_per_rank": n * 2 / (v * 1e-3) / 1e9} for k, v in out.items()},
+                "speedup_vs_nccl_bf16": {k: out["nccl_bf16_all_reduce"] / out[k] for k in ("echo_feedback",
+                                                                                         "echo_no_feedback")},
+                "n_gpus": world, "P": world, "steps": steps, "warmup": args.warmup,
+                "config": {"workload": w.name, "n": n, "group": group, "bits": bits}, "data": "synthetic"}
+        print(json.dumps(line), flush=True)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -757,6 +819,8 @@ def main():
                     help="off: time the call without EMA state as the main step (profiling)")
     ap.add_argument("--ablation", action="store_true",
                     help="print the accuracy ablations on the synthetic chains instead of timing")
+    ap.add_argument("--dist", action="store_true",
+                    help="under torchrun: the multi-GPU call (P = world size) against NCCL's bf16 all-reduce")
     ap.add_argument("--ranks", action="store_true",
                     help="print one rank's kernel times of a multi-GPU call (rank 0 of P = 8, 1 GB) instead")
     ap.add_argument("--workloads", action="store_true",
@@ -775,6 +839,8 @@ def main():
         run_workloads(args)
     elif args.ranks:
         run_ranks(args)
+    elif args.dist:
+        run_dist(args)
     else:
         run_gpu(args)
 
