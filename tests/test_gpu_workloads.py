@@ -153,17 +153,19 @@ def test_chain_48_sites_p4_early_int8():
     run_chain(w, True)
 
 
-@pytest.mark.parametrize("feedback", [True, False])
-def test_headline_1gb_sampled_columns(feedback):
+@pytest.mark.parametrize("feedback,bits", [(True, 4), (False, 4), (True, 8)])
+def test_headline_1gb_sampled_columns(feedback, bits):
     """P = 8, 1 GB per rank, two calls (state carried when there is one), in
-    the exact launch sequence the benchmark times (quantize, then the owners'
-    reduce writing the outputs)."""
+    the launch sequences the benchmark times: first one echo_allreduce_sim
+    call (its headline steps: the owners' pass a programmatic dependent of
+    the quantize pass), then the two phase entry points (its per-kernel
+    pass). The early-site 8-bit mode on the same message too."""
     w = W.HEADLINE
     P, n = w.P, w.n
     free, _ = torch.cuda.mem_get_info()
-    if free < 60e9:
-        pytest.skip("needs ~55 GB of free device memory")
-    ar = E.EchoAllReduce(n, P, w.group, 4, feedback)
+    if free < 65e9:
+        pytest.skip("needs ~60 GB of free device memory")
+    ar = E.EchoAllReduce(n, P, w.group, bits, feedback)
     S = Sampled(w, 256, feedback)
     try:
         inputs = [W.rank_input(w, r, 0, "cuda") for r in range(P)]
@@ -175,12 +177,15 @@ def test_headline_1gb_sampled_columns(feedback):
             x_orc[j0][:, :c.stop - c.start] = _gpu_inputs_u16(inputs, c)
         fb = (w.eta, w.alpha_long, w.alpha_short, w.w)
         for call in range(2):
-            E.echo_phase_quantize(inputs, ar.handle, 4, *fb)
-            E.echo_phase_reduce(inputs, outputs, ar.handle, 4, *fb)
-            orcs = _oracle_step(S, x_orc, 4)
+            if call == 0:
+                E.echo_allreduce_sim(inputs, outputs, ar.handle, n, P, bits, w.group, *fb)
+            else:
+                E.echo_phase_quantize(inputs, ar.handle, bits, *fb)
+                E.echo_phase_reduce(inputs, outputs, ar.handle, bits, *fb)
+            orcs = _oracle_step(S, x_orc, bits)
             rc, flags = ar.status()
             assert rc == E.ECHO_OK
-            _compare_sampled(ar, outputs, S, orcs, 4, call)
+            _compare_sampled(ar, outputs, S, orcs, bits, call)
         # properties over the whole message: every rank holds the same result
         for r in range(1, P):
             assert torch.equal(outputs[r].view(torch.int16), outputs[0].view(torch.int16))
