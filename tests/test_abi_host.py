@@ -160,3 +160,38 @@ def test_rank_calls_reject_bad_arguments(L):
     assert L.echo_rank_reduce(4096, 4096, None, 4, 1.0, 0.05, 0.5, 0.5, None) == E.ECHO_EINVAL
     assert L.echo_rank_decode(4096, None, 4, None) == E.ECHO_EINVAL
     assert h.value is None
+
+
+def test_header_is_c_and_links(L, tmp_path):
+    """include/echo.h compiles as pedantic C99 and a C program linked against
+    the library gets the same host-only answers as the binding."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include "echo.h"
+int main(void) {
+    echo_layout L;
+    echo_rank_layout R;
+    if (echo_query_layout(1000, 3, 64, 8, 4, &L) != ECHO_OK) return 2;
+    if (echo_query_rank_layout(1000, 3, 1, 64, 8, 4, &R) != ECHO_OK) return 3;
+    printf("%zu %llu %lld %lld %llu\n", echo_state_bytes(1000, 3, 64),
+           (unsigned long long)L.workspace_bytes, (long long)R.seg_begin, (long long)R.seg_groups,
+           (unsigned long long)R.workspace_bytes);
+    return echo_query_rank_layout(1000, 3, 3, 64, 8, 4, &R) == ECHO_EINVAL ? 0 : 4;
+}
+''')
+    exe = tmp_path / "abi"
+    lib = _build.LIB
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), lib, "-o", str(exe)], check=True)
+    env = dict(os.environ, LD_LIBRARY_PATH=os.path.dirname(lib))
+    out = subprocess.run([str(exe)], capture_output=True, text=True, env=env, check=True).stdout.split()
+    lay = E.echo_query_layout(1000, 3, 64, 8, 4)
+    rl = E.echo_query_rank_layout(1000, 3, 1, 64, 8, 4)
+    assert [int(v) for v in out] == [E.echo_state_bytes(1000, 3, 64), lay.workspace_bytes, rl.seg_begin,
+                                     rl.seg_groups, rl.workspace_bytes]
