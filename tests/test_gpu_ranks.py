@@ -41,6 +41,8 @@ CASES = [
     (5, 148 * 8 * 256 + 37, 256, 8, True, O.Q_DIRECTED),
     (8, 50000, 32, 4, True, O.Q_NEAREST),
     (6, 70001, 64, 4, True, O.Q_INT_ZERO),
+    (16, 50000, 128, 4, True, O.Q_DIRECTED),
+    (64, 3 * 64 * 128 + 17, 128, 4, True, O.Q_DIRECTED),   # largest P
 ]
 
 
