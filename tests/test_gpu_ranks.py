@@ -126,3 +126,35 @@ def test_rank_and_simulation_handles_do_not_mix():
     finally:
         rk.close()
         ar.close()
+
+
+@pytest.mark.parametrize("bad", [1e6, float("nan")])
+@pytest.mark.parametrize("rank", [0, 1])
+def test_rank_range_flag(bad, rank):
+    """A value outside the fp16 parameter range (or a NaN) on one rank sets
+    ECHO_FLAG_RANGE on the handle whose kernel met it -- the non-owner's
+    quantize pass or the owner's sum -- and echo_get_status clears it."""
+    P, n = 2, 4096
+    x = random_inputs(P, n, 10)
+    x[rank, 100] = bad            # group 0: owned by rank 0
+    ranks = [E.EchoRank(n, P, r, 128, 4, True) for r in range(P)]
+    try:
+        xs = [x[r].cuda() for r in range(P)]
+        outs = [torch.empty_like(t) for t in xs]
+        plans = [rk.plan(4) for rk in ranks]
+        for r in range(P):
+            ranks[r].quantize(xs[r], 4)
+        emulate_all_to_all(plans)
+        for r in range(P):
+            ranks[r].reduce(xs[r], outs[r], 4)
+        emulate_all_gather(plans)
+        for r in range(P):
+            ranks[r].decode(outs[r], 4)
+        flags = [rk.status()[1] for rk in ranks]
+        assert flags[0] & E.ECHO_FLAG_RANGE          # the owner's sum holds the bad value
+        if rank == 1:
+            assert flags[1] & E.ECHO_FLAG_RANGE      # and rank 1 quantized it
+        assert [rk.status()[1] for rk in ranks] == [0, 0]   # cleared
+    finally:
+        for rk in ranks:
+            rk.close()
