@@ -225,6 +225,7 @@ def cpu_sample_rate(cols, seed=123):
     w = _workload()
     P, group = w.P, w.group
     G = -(-w.n // group)
+    cols = min(cols, w.n // group)                # full groups only (a smaller message when profiling)
     j0 = (G // 2) - cols // 2                     # straddles an owner boundary at P = 8
     m = cols * group
     x = np.empty((P, m), np.uint16)
@@ -526,7 +527,7 @@ def run_gpu(args):
         if world == 1 and not args.no_cpu_baseline:
             gbs, dt, er = cpu_sample_rate(CPU_BASELINE_COLS)
             line["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                                    "sample": f"{CPU_BASELINE_COLS} group columns x P={P} "
+                                    "sample": f"{er // (P * group)} group columns x P={P} "
                                               f"({er} element-ranks, {dt:.1f} s, single thread)"}
         print(json.dumps(line), flush=True)
     ar.close()

@@ -1,0 +1,54 @@
+"""The benchmark's JSON line: the keys its consumers read.
+
+CPU: the reference arm (the oracle timed on the host) prints one line with
+the metric, the unit, its cpu_baseline and an e2e entry of zero copies.
+GPU: the main arm on a small message of the same shape family prints one line
+with the roofline, the clocks, the end-to-end leg, the CPU baseline and the
+launch count.
+"""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _last_json(out: str) -> dict:
+    lines = [l for l in out.splitlines() if l.startswith("{")]
+    assert lines, out[-2000:]
+    return json.loads(lines[-1])
+
+
+def test_reference_arm_line():
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1")
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "0"],
+                         cwd=ROOT, env=env, capture_output=True, text=True, timeout=600, check=True).stdout
+    line = _last_json(out)
+    assert line["impl"] == "reference"
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["value"] > 0 and line["cpu_baseline"]["value"] == line["value"]
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert line["config"]["workload"] == "p8_1GB_student_t"
+
+
+@pytest.mark.gpu
+def test_main_arm_line():
+    out = subprocess.run([sys.executable, "bench.py", "--tokens", "2048", "--steps", "3", "--warmup", "3",
+                          "--no-variants"], cwd=ROOT, capture_output=True, text=True, timeout=900, check=True).stdout
+    line = _last_json(out)
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "roofline_call", "clocks", "e2e",
+                "gpu_launches", "cpu_baseline", "status", "flags"):
+        assert key in line, key
+    assert line["status"] == 0 and line["flags"] == 0
+    assert line["value"] > 0 and line["gpu_launches"] == 6
+    r = line["roofline"]
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and 0 < r["frac"] == pytest.approx(r["achieved"] / r["peak"])
+    assert line["e2e"]["value"] > 0 and line["e2e"]["h2d_bytes_per_step"] == 8 * 2048 * 4096 * 2
+    assert line["cpu_baseline"]["kind"] == "oracle"
