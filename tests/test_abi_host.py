@@ -195,3 +195,15 @@ int main(void) {
     rl = E.echo_query_rank_layout(1000, 3, 1, 64, 8, 4)
     assert [int(v) for v in out] == [E.echo_state_bytes(1000, 3, 64), lay.workspace_bytes, rl.seg_begin,
                                      rl.seg_groups, rl.workspace_bytes]
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    """Without the CUDA library the binding raises at the first call; there is
+    no fallback path."""
+    import bit_error_compensated_group_b200.echo as EE
+    monkeypatch.setattr(EE, "_lib", None)
+    monkeypatch.setattr(EE, "LIB_PATH", "/nonexistent/libecho_b200.so")
+    with pytest.raises(RuntimeError, match="missing"):
+        EE.echo_state_bytes(1024, 2, 128)
+    with pytest.raises(RuntimeError, match="missing"):
+        EE.EchoAllReduce(1024, 2, device="cpu")
