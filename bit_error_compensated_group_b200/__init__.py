@@ -9,7 +9,7 @@ from .echo import (  # noqa: F401
     ECHO_EINVAL, ECHO_ECUDA, ECHO_ERANGE, ECHO_ETIMEOUT, ECHO_FLAG_RANGE, ECHO_FLAG_TIMEOUT, ECHO_MAX_RANKS, ECHO_OK,
     ECHO_QUANT_DIRECTED, ECHO_QUANT_INT_ZERO, ECHO_QUANT_NEAREST,
     EchoAllReduce, EchoError, EchoLayout, EchoRank, EchoRankLayout, ExchangePlan, echo_init_rank, echo_query_rank_layout,
-    echo_rank_decode, echo_rank_quantize, echo_rank_reduce, exchange_all_gather, exchange_all_to_all, exchange_in_process, echo_allreduce_sim, echo_allreduce_sim_host, echo_allreduce_sim_range,
+    echo_rank_decode, echo_rank_quantize, echo_rank_reduce, exchange_all_gather, exchange_all_to_all, exchange_in_process, echo_inject_launch_failure, echo_allreduce_sim, echo_allreduce_sim_host, echo_allreduce_sim_range,
     echo_check_watchdog, echo_free, echo_get_status, echo_init_state,
     echo_phase_gather, echo_phase_quantize, echo_phase_reduce, echo_query_layout, echo_set_quantizer, echo_state_bytes,
     echo_status_string, echo_workspace_bytes, lib,

@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <new>
 
@@ -224,7 +225,11 @@ int launch_bits(Stage stage, int bits, const echo_dev::Args& a, const echo_state
 
 // `pdl` (owners' pass only): this launch directly follows the same call's
 // quantize launch on the stream and may overlap its tail.
+// echo_inject_launch_failure: while set, launches report ECHO_ECUDA instead
+std::atomic<int> g_fail_launches{0};
+
 int launch(Stage stage, int bits, const echo_dev::Args& a, const echo_state* st, cudaStream_t s, bool pdl = false) {
+    if (g_fail_launches.load(std::memory_order_relaxed)) return ECHO_ECUDA;
     switch (st->group) {
         case 32: return launch_bits<32>(stage, bits, a, st, s, pdl);
         case 64: return launch_bits<64>(stage, bits, a, st, s, pdl);
@@ -677,6 +682,10 @@ int echo_rank_decode(void* out, echo_state* st, int bits, echo_stream_t stream) 
     if (int rc = set_device(st)) return rc;
     if (st->P < 2) return ECHO_OK;
     return launch(Stage::Gather, bits, a, st, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int echo_inject_launch_failure(int enable) {
+    return g_fail_launches.exchange(enable ? 1 : 0);
 }
 
 int echo_check_watchdog(echo_state* st, uint32_t limit_us, echo_stream_t stream) {

@@ -115,6 +115,8 @@ def lib() -> ctypes.CDLL:
         L.echo_rank_reduce.restype = I
         L.echo_rank_decode.argtypes = [V, V, I, V]
         L.echo_rank_decode.restype = I
+        L.echo_inject_launch_failure.argtypes = [I]
+        L.echo_inject_launch_failure.restype = I
         L.echo_free.argtypes = [V]
         L.echo_free.restype = I
         L.echo_status_string.argtypes = [I]
@@ -270,6 +272,12 @@ def echo_allreduce_sim_noalloc(inputs: Sequence, outputs: Sequence, state, n: in
 def echo_set_quantizer(st, quantizer: int) -> None:
     """Quantizer form for the handle's later calls (ECHO_QUANT_*)."""
     _check(lib().echo_set_quantizer(st, quantizer), "echo_set_quantizer")
+
+
+def echo_inject_launch_failure(enable: bool) -> bool:
+    """Test hook: while enabled, kernel launches report ECHO_ECUDA (nothing
+    fails on the GPU). Returns the previous setting."""
+    return bool(lib().echo_inject_launch_failure(1 if enable else 0))
 
 
 def echo_free(st) -> None:

@@ -321,6 +321,17 @@ ECHO_API int echo_get_status(echo_state* st, echo_stream_t stream, uint32_t* dev
  */
 ECHO_API int echo_check_watchdog(echo_state* st, uint32_t limit_us, echo_stream_t stream);
 
+/*
+ * Fault-injection hook for tests of callers' error paths (no counterpart on
+ * the pages; part of this library's failure detection). While enabled
+ * (enable != 0), every call that would launch one of the all-reduce kernels
+ * returns ECHO_ECUDA at that launch instead: the kernel is not launched;
+ * work a call enqueues before its first launch (the host-buffer call's first
+ * copies, the no-allocation call's flag clear) stays enqueued. Process-wide,
+ * host-only; nothing on the GPU fails. Returns the previous setting (0 or 1).
+ */
+ECHO_API int echo_inject_launch_failure(int enable);
+
 /* Size of the fixed scratch array used by echo_allreduce_sim_noalloc. It is
  * device memory that every GPU which loads this library holds until the
  * process exits. */

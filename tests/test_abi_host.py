@@ -207,3 +207,10 @@ def test_missing_library_fails_loudly(monkeypatch):
         EE.echo_state_bytes(1024, 2, 128)
     with pytest.raises(RuntimeError, match="missing"):
         EE.EchoAllReduce(1024, 2, device="cpu")
+
+
+def test_launch_failure_hook_toggles(L):
+    assert E.echo_inject_launch_failure(True) is False
+    assert E.echo_inject_launch_failure(True) is True
+    assert E.echo_inject_launch_failure(False) is True
+    assert E.echo_inject_launch_failure(False) is False

@@ -57,3 +57,42 @@ def test_watchdog_argument_checks():
             assert ei.value.status == E.ECHO_EINVAL
     finally:
         gpu.close()
+
+
+def test_injected_launch_failures_reach_the_caller():
+    """With the host hook on, every entry point that launches a kernel returns
+    ECHO_ECUDA (raised as EchoError); nothing fails on the GPU, and with the
+    hook off the next call is correct."""
+    import numpy as np
+    import oracle as O
+    from parity import padded, random_inputs, u16
+    P, n = 4, 10000
+    G = -(-n // 128)
+    x = random_inputs(P, n, 21)
+    ar = E.EchoAllReduce(n, P)
+    rk = E.EchoRank(n, 1, 0)
+    ins = [x[r].cuda() for r in range(P)]
+    outs = [torch.empty_like(t) for t in ins]
+    try:
+        assert E.echo_inject_launch_failure(True) is False
+        try:
+            for fn in (lambda: ar(ins, outs, 4),
+                       lambda: E.echo_phase_quantize(ins, ar.handle, 4, 1.0, 0.05, 0.5, 0.5),
+                       lambda: E.echo_allreduce_sim_range(ins, outs, ar.handle, n, P, 4, 128, 1.0, 0.05, 0.5, 0.5,
+                                                          0, G),
+                       lambda: rk.reduce(ins[0], outs[0], 4)):
+                with pytest.raises(E.EchoError) as ei:
+                    fn()
+                assert ei.value.status == E.ECHO_ECUDA
+        finally:
+            assert E.echo_inject_launch_failure(False) is True
+        ar(ins, outs, 4)
+        el = np.zeros((P, G * 128), np.float32)
+        es = np.zeros((P, G * 128), np.float32)
+        orc = O.echo_allreduce(padded(u16(x), G * 128), n_total=n, group=128, bits=4, e_long=el, e_short=es)
+        assert ar.status() == (E.ECHO_OK, 0)
+        assert np.array_equal(np.stack([u16(o) for o in outs]), orc.y[:, :n])
+    finally:
+        E.echo_inject_launch_failure(False)
+        ar.close()
+        rk.close()
