@@ -1,20 +1,23 @@
 // echo_kernels.cuh -- shared device helpers of the Echo all-reduce
 // simulation, and the scalar per-group paths.
 //
-// The call is three kernels (echo_pipeline.cuh), one per stage of the
-// restructured all-reduce of the Echo explainer ("Echoの仕組み①": all-to-all
-// of 4-bit non-owned segments, high-precision sum at the owner, 4-bit
-// all-gather), with the feedback of "Echoの仕組み②" fused into the passes
-// that read the inputs:
+// The stages of the restructured all-reduce of the Echo explainer
+// ("Echoの仕組み①": all-to-all of 4-bit non-owned segments, high-precision
+// sum at the owner, 4-bit all-gather), with the feedback of "Echoの仕組み②"
+// fused into the passes that read the inputs (kernels in echo_pipeline.cuh):
 //
 //   quantize  every rank's non-owned groups: x' = x + c, group min/max,
 //             fp16 {s, z}, packed codes -> all-to-all payload; residual
 //             x' - x_hat -> both EMAs.
 //   reduce    every group at its owner: x'_owner + dequantized payloads in
 //             rank order (binary32), requantize -> all-gather payload;
-//             residual sum - y -> the owner's EMAs.
-//   gather    every group: dequantize the gathered payload once, write the
-//             bf16 result into all P outputs.
+//             residual sum - y -> the owner's EMAs; in a whole call it also
+//             writes the decoded result into all P outputs (phase 4).
+//   gather    phase 4 on its own: dequantize the gathered payload once and
+//             write the bf16 result into all P outputs (echo_phase_gather;
+//             one rank of a multi-GPU call decodes with k_decode_rank).
+//
+// A call is the first two kernels.
 //
 // This file holds the argument block, the per-group grid (fp16 zero rounded
 // toward -inf from the minimum, fp16 step rounded toward +inf from
