@@ -52,3 +52,21 @@ def test_main_arm_line():
     assert r["bound"] == "hbm" and r["unit"] == "GB/s" and 0 < r["frac"] == pytest.approx(r["achieved"] / r["peak"])
     assert line["e2e"]["value"] > 0 and line["e2e"]["h2d_bytes_per_step"] == 8 * 2048 * 4096 * 2
     assert line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_algorithmic_bytes_match_the_roofline_definition():
+    """B_min = P n (2 in + 2 out + 16 state) + 2 (P - 1) G PB + 2 G PB: 21.0625
+    bytes per element-rank at 4 bits and groups of 128 (PB = 68), 5.0625
+    without state; the two kernels' own shares add up to it less the gather
+    payload's read-back, which the owners' pass does not need."""
+    sys.path.insert(0, ROOT)
+    import bench
+    P, n, g = 8, 1 << 29, 128
+    G = n // g
+    ab = bench.algorithmic_bytes(P, n, g, 4)
+    assert ab["total"] == P * n * 20 + 2 * (P - 1) * G * 68 + 2 * G * 68 == 90_462_748_672
+    assert ab["total"] / (P * n) == 21.0625
+    assert bench.algorithmic_bytes(P, n, g, 4, feedback=False)["total"] / (P * n) == 5.0625
+    assert ab["quantize"] == (P - 1) * G * 2372 and ab["reduce_gather"] == G * 4896
+    assert ab["quantize"] + ab["reduce_gather"] + G * 68 == ab["total"]
+    assert bench.algorithmic_bytes(P, n, g, 8)["total"] / (P * n) == 22.0625
