@@ -55,9 +55,24 @@ MUTANTS = {
     "ties_not_even": [("k = (fmod(lo, 2.0) == 0.0) ? lo : hi;", "k = hi;")],
     "no_minus_zero_fix": [("    mn = mn + 0.0f;\n    mx = mx + 0.0f;\n", "")],
     "no_feedback_add": [("                xp[idx] = xv + c;", "                xp[idx] = xv;")],
+    # evaluation orders: the owner's sum in rank order, the EMA as (1 - a) e + a rho
+    "sum_reverse_order": [("        for (int r = 0; r < P; r++) {\n            size_t base = (size_t)r * (size_t)ld + (size_t)(jl * group);\n            if (r == o) {",
+                           "        for (int r = P - 1; r >= 0; r--) {\n            size_t base = (size_t)r * (size_t)ld + (size_t)(jl * group);\n            if (r == o) {"),
+                          ("                if (r == 0) {\n                    sum[i] = vtmp[i];",
+                           "                if (r == P - 1) {\n                    sum[i] = vtmp[i];")],
+    "sum_owner_first": [("        for (int r = 0; r < P; r++) {\n            size_t base = (size_t)r * (size_t)ld + (size_t)(jl * group);\n            if (r == o) {",
+                         "        for (int rr = 0; rr < P; rr++) {\n            int r = (o + rr) % P;\n            size_t base = (size_t)r * (size_t)ld + (size_t)(jl * group);\n            if (r == o) {"),
+                        ("                if (r == 0) {\n                    sum[i] = vtmp[i];",
+                         "                if (rr == 0) {\n                    sum[i] = vtmp[i];")],
+    "sum_owner_last": [("        for (int r = 0; r < P; r++) {\n            size_t base = (size_t)r * (size_t)ld + (size_t)(jl * group);\n            if (r == o) {",
+                        "        for (int rr = 0; rr < P; rr++) {\n            int r = (o + 1 + rr) % P;\n            size_t base = (size_t)r * (size_t)ld + (size_t)(jl * group);\n            if (r == o) {"),
+                       ("                if (r == 0) {\n                    sum[i] = vtmp[i];",
+                        "                if (rr == 0) {\n                    sum[i] = vtmp[i];")],
+    "ema_incremental_form": [("        float u = keep * e[i];\n        float v = alpha * rho[i];\n        e[i] = u + v;",
+                              "        float d = rho[i] - e[i];\n        float v = alpha * d;\n        e[i] = e[i] + v;\n        (void)keep;")],
 }
 
-PIN_FILES = ["tests/test_oracle_call.py", "tests/test_oracle_quantizer.py", "tests/test_oracle_variants.py",
+PIN_FILES = ["tests/test_oracle_order.py", "tests/test_oracle_call.py", "tests/test_oracle_quantizer.py", "tests/test_oracle_variants.py",
              "tests/test_oracle_chain.py", "tests/test_oracle_convert.py"]
 
 
