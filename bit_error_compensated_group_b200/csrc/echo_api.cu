@@ -31,6 +31,7 @@ struct echo_state {
     cudaEvent_t ev[3];
     bool have_events;
     int rank;              // -1: the single-GPU simulation; else this rank of a multi-GPU call
+    uint64_t wait_ns;      // limit of the kernels' bounded waits (echo_set_wait_limit)
 };
 
 namespace {
@@ -40,6 +41,9 @@ constexpr uint64_t kAlign = 256;
 // GPUs; the shared-memory opt-in of a kernel is made on each device).
 constexpr int kMaxDevices = 64;
 constexpr int64_t kMaxN = int64_t(1) << 40;
+// bounded device-side waits: default limit and the range echo_set_wait_limit accepts
+constexpr uint64_t kDefaultWaitNs = 1000ull * 1000ull * 1000ull;   // 1 s
+constexpr uint32_t kMinWaitUs = 1000u, kMaxWaitUs = 60u * 1000u * 1000u;
 
 uint64_t align_up(uint64_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
@@ -293,6 +297,7 @@ bool make_args(const echo_state* st, int bits, const void* const* inputs, void* 
     a->a_short = aS;
     a->keep_short = 1.0f - aS;
     a->one = 1.0f;
+    a->wait_ns = st->wait_ns;
     return true;
 }
 
@@ -399,6 +404,7 @@ bool make_rank_args(const echo_state* st, int bits, RankPhase phase, const void*
     a->a_short = aS;
     a->keep_short = 1.0f - aS;
     a->one = 1.0f;
+    a->wait_ns = st->wait_ns;
     return true;
 }
 
@@ -462,8 +468,19 @@ int echo_init_state(echo_state** out, int64_t n, int P, int group, int max_bits,
     st->quantizer = ECHO_QUANT_DIRECTED;
     st->have_events = false;
     st->rank = -1;
+    st->wait_ns = kDefaultWaitNs;
     *out = st;
     return ECHO_OK;
+}
+
+int echo_set_wait_limit(echo_state* st, uint32_t limit_us) {
+    if (!st || limit_us < kMinWaitUs || limit_us > kMaxWaitUs) return ECHO_EINVAL;
+    st->wait_ns = 1000ull * limit_us;
+    return ECHO_OK;
+}
+
+uint32_t echo_get_wait_limit(const echo_state* st) {
+    return st ? (uint32_t)(st->wait_ns / 1000ull) : 0u;
 }
 
 int echo_set_quantizer(echo_state* st, int quantizer) {
@@ -646,6 +663,7 @@ int echo_init_rank(echo_state** out, int64_t n, int P, int rank, int group, int 
     st->quantizer = ECHO_QUANT_DIRECTED;
     st->have_events = false;
     st->rank = rank;
+    st->wait_ns = kDefaultWaitNs;
     *out = st;
     return ECHO_OK;
 }
@@ -689,10 +707,11 @@ int echo_inject_launch_failure(int enable) {
 }
 
 int echo_check_watchdog(echo_state* st, uint32_t limit_us, echo_stream_t stream) {
-    if (!st || limit_us < 1 || limit_us > 10000000u) return ECHO_EINVAL;
+    if (!st || limit_us > 10000000u) return ECHO_EINVAL;
     if (int rc = set_device(st)) return rc;
+    const unsigned long long limit_ns = limit_us == 0 ? st->wait_ns : 1000ull * limit_us;
     echo_dev::k_watchdog_check<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        reinterpret_cast<uint32_t*>(st->workspace), 1000ull * limit_us);
+        reinterpret_cast<uint32_t*>(st->workspace), limit_ns);
     return cuda_status(cudaGetLastError());
 }
 
@@ -786,6 +805,7 @@ int echo_allreduce_sim_noalloc(const void* const* inputs, void* const* outputs, 
     st.quantizer = ECHO_QUANT_DIRECTED;
     st.have_events = false;
     st.rank = -1;
+    st.wait_ns = kDefaultWaitNs;
     echo_dev::Args a;
     if (!make_args(&st, bits, inputs, outputs, eta, alpha_long, alpha_short, w, &a)) return ECHO_EINVAL;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -801,6 +821,8 @@ int echo_allreduce_sim_noalloc(const void* const* inputs, void* const* outputs, 
         if (cudaMemcpy(&f, scratch + L.flags_offset, sizeof(f), cudaMemcpyDeviceToHost) != cudaSuccess)
             return ECHO_ECUDA;
         *flags_out = f;
+        if (f & ECHO_FLAG_TIMEOUT) return ECHO_ETIMEOUT;
+        if (f & ECHO_FLAG_RANGE) return ECHO_ERANGE;
     }
     return ECHO_OK;
 }

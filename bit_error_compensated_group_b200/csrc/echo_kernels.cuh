@@ -80,6 +80,9 @@ struct Args {
     long long g_col_base;           // gather payload written at j - g_col_base
     long long g_seg_stride;         // > 0: gathered payload read as [owner][g_seg_stride]
     int out_lo, out_hi;             // gather decode: outputs of ranks [out_lo, out_hi)
+    // limit of every bounded device-side wait (mbarrier waits of the
+    // bulk-copy pipelines), in nanoseconds of the global timer
+    unsigned long long wait_ns;
 };
 
 __device__ __forceinline__ size_t a2a_slot(const Args& a, int r, long long j) {

@@ -12,9 +12,9 @@
 //
 // Synchronization per stage: full[s] (producer arrive + transaction bytes)
 // and empty[s] (one arrive per consumer warp). Every wait is bounded by a
-// wall-clock limit: on expiry the kernel sets ECHO_FLAG_TIMEOUT, stops, and
-// the producer lane waits (again bounded) for the copies it issued before the
-// CTA exits. Partial last groups (not 16-byte sized) take the direct
+// wall-clock limit (Args::wait_ns, the handle's setting, 1 s by default):
+// on expiry the kernel sets ECHO_FLAG_TIMEOUT, stops, and the producer lane
+// waits (again bounded) for the copies it issued before the CTA exits. Partial last groups (not 16-byte sized) take the direct
 // register path of echo_kernels.cuh.
 #pragma once
 
@@ -36,7 +36,6 @@ constexpr int kStagesQuantizeNF = 4;
 constexpr int kStagesReduceNF = 4;
 // dynamic shared memory of a pipelined kernel with NS ring stages
 __host__ __device__ constexpr int pipe_smem(int NS) { return NS * kStageBytes + 2 * NS * 8 + 16; }
-constexpr unsigned long long kWaitLimitNs = 1000ull * 1000ull * 1000ull;   // 1 s
 
 // ------------------------------------------------------------ PTX wrappers
 
@@ -267,7 +266,7 @@ __device__ __forceinline__ void produce(const Args& a, const PipeShared& p, RunW
     for (long long k = blockIdx.x; walker.locate(k, &t, a); k += gridDim.x, ++issued) {
         const int s = (int)(issued % NS);
         const uint32_t use = (uint32_t)(issued / NS);
-        if (issued >= NS && !mbar_wait(&p.empty[s], (use & 1u) ^ 1u, kWaitLimitNs, p.abort)) {
+        if (issued >= NS && !mbar_wait(&p.empty[s], (use & 1u) ^ 1u, a.wait_ns, p.abort)) {
             report_timeout(a, p);
             break;
         }
@@ -301,7 +300,7 @@ __device__ __forceinline__ void produce(const Args& a, const PipeShared& p, RunW
     const long long first = issued > NS ? issued - NS : 0;
     for (long long i = first; i < issued; ++i) {
         const int s = (int)(i % NS);
-        if (!mbar_wait(&p.full[s], (uint32_t)(i / NS) & 1u, kWaitLimitNs, nullptr)) {
+        if (!mbar_wait(&p.full[s], (uint32_t)(i / NS) & 1u, a.wait_ns, nullptr)) {
             atomicOr(a.flags, (unsigned)ECHO_FLAG_TIMEOUT);
         }
     }
@@ -740,7 +739,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
     Tile t;
     for (long long k = blockIdx.x; walker.locate(k, &t, a); k += gridDim.x, ++i) {
         const int s = (int)(i % NS);
-        if (!mbar_wait(&p.full[s], (uint32_t)(i / NS) & 1u, kWaitLimitNs, p.abort)) {
+        if (!mbar_wait(&p.full[s], (uint32_t)(i / NS) & 1u, a.wait_ns, p.abort)) {
             if (lead) {
                 report_timeout(a, p);
                 if (FB) bulk_wait_all();   // this warp's stores still in flight
@@ -1076,7 +1075,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
     Tile t;
     for (long long k = blockIdx.x; walker.locate(k, &t, a); k += gridDim.x, ++i) {
         const int s = (int)(i % NS);
-        if (!mbar_wait(&p.full[s], (uint32_t)(i / NS) & 1u, kWaitLimitNs, p.abort)) {
+        if (!mbar_wait(&p.full[s], (uint32_t)(i / NS) & 1u, a.wait_ns, p.abort)) {
             if ((threadIdx.x & 31) == 0) report_timeout(a, p);
             return;
         }

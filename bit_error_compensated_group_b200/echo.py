@@ -117,6 +117,13 @@ def lib() -> ctypes.CDLL:
         L.echo_rank_decode.restype = I
         L.echo_inject_launch_failure.argtypes = [I]
         L.echo_inject_launch_failure.restype = I
+        L.echo_set_wait_limit.argtypes = [V, ctypes.c_uint32]
+        L.echo_set_wait_limit.restype = I
+        L.echo_get_wait_limit.argtypes = [V]
+        L.echo_get_wait_limit.restype = ctypes.c_uint32
+        L.echo_allreduce_sim_noalloc.argtypes = [PP, PP, V, I64, I, I, I, F, F, F, F,
+                                                 ctypes.POINTER(ctypes.c_uint32), V]
+        L.echo_allreduce_sim_noalloc.restype = I
         L.echo_free.argtypes = [V]
         L.echo_free.restype = I
         L.echo_status_string.argtypes = [I]
@@ -255,18 +262,26 @@ def echo_allreduce_sim_noalloc(inputs: Sequence, outputs: Sequence, state, n: in
     """echo_allreduce_sim for callers that cannot allocate device memory:
     the payloads live in the library's fixed scratch array, there is no
     handle, and the caller passes the EMA state tensor (or None for no
-    feedback). Returns the call's ECHO_FLAG_* bits when `read_flags` (which
-    synchronizes the stream), else None."""
-    f = lib().echo_allreduce_sim_noalloc
-    V, I, I64, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
-    PP = ctypes.POINTER(ctypes.c_void_p)
-    f.argtypes = [PP, PP, V, I64, I, I, I, F, F, F, F, ctypes.POINTER(ctypes.c_uint32), V]
-    f.restype = I
+    feedback). With `read_flags` (which synchronizes the stream) a range or
+    timeout flag raised by the call's kernels raises EchoError (ECHO_ERANGE /
+    ECHO_ETIMEOUT) and the flag bits (0) are returned; without it nothing
+    reports such a failure and None is returned."""
     flags = ctypes.c_uint32(0)
-    rc = f(_ptr_array(inputs), _ptr_array(outputs), _ptr(state), n, P, bits, group, eta, alpha_long, alpha_short,
-           w, ctypes.byref(flags) if read_flags else None, _stream(stream))
+    rc = lib().echo_allreduce_sim_noalloc(_ptr_array(inputs), _ptr_array(outputs), _ptr(state), n, P, bits, group,
+                                          eta, alpha_long, alpha_short, w,
+                                          ctypes.byref(flags) if read_flags else None, _stream(stream))
     _check(rc, "echo_allreduce_sim_noalloc")
     return int(flags.value) if read_flags else None
+
+
+def echo_set_wait_limit(st, limit_us: int) -> None:
+    """Limit of the kernels' bounded device waits for the handle's later
+    calls (1 ms .. 60 s; default 1 s)."""
+    _check(lib().echo_set_wait_limit(st, limit_us), "echo_set_wait_limit")
+
+
+def echo_get_wait_limit(st) -> int:
+    return int(lib().echo_get_wait_limit(st))
 
 
 def echo_set_quantizer(st, quantizer: int) -> None:

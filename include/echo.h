@@ -310,12 +310,32 @@ ECHO_API int echo_allreduce_sim_host(const void* const* host_inputs, void* host_
 ECHO_API int echo_get_status(echo_state* st, echo_stream_t stream, uint32_t* device_flags);
 
 /*
+ * Limit of the kernels' bounded device-side waits for the later calls of a
+ * handle (no counterpart on the pages; part of this library's failure
+ * detection). Every wait of the bulk-copy pipelines (a consumer waiting for a
+ * staged tile, the producer waiting for a free slot or for its own copies to
+ * land) gives up after this long, sets ECHO_FLAG_TIMEOUT and ends the kernel
+ * early; that call's results are then undefined. The default, 1 s, is far
+ * above any wait of a healthy call; a caller that shares the GPU with other
+ * contexts time-sliced for long periods may raise it.
+ *   limit_us   1000 .. 60 000 000 (1 ms .. 60 s)
+ * Host-only, takes effect at the handle's next launch. ECHO_EINVAL on a NULL
+ * handle or a limit out of range (the setting is then unchanged).
+ * echo_allreduce_sim_noalloc, which has no handle, always uses the default.
+ */
+ECHO_API int echo_set_wait_limit(echo_state* st, uint32_t limit_us);
+
+/* The handle's wait limit in microseconds (0 for a NULL handle). */
+ECHO_API uint32_t echo_get_wait_limit(const echo_state* st);
+
+/*
  * Failure-detection self-check (no counterpart on the pages; part of this
  * library's error reporting). Launches one thread that waits, with the same
  * bounded wait the bulk-copy pipelines use, on a barrier that nothing ever
- * completes. After limit_us microseconds (1 .. 10^7) the wait gives up, the
- * kernel sets ECHO_FLAG_TIMEOUT in st's flag word and returns; the next
- * echo_get_status returns ECHO_ETIMEOUT and the context stays usable.
+ * completes. After limit_us microseconds (1 .. 10^7; 0: the handle's wait
+ * limit, see echo_set_wait_limit) the wait gives up, the kernel sets
+ * ECHO_FLAG_TIMEOUT in st's flag word and returns; the next echo_get_status
+ * returns ECHO_ETIMEOUT and the context stays usable.
  * Asynchronous on `stream`. ECHO_EINVAL on a NULL handle or a limit out of
  * range, ECHO_ECUDA when the launch fails.
  */
@@ -362,7 +382,12 @@ ECHO_API int echo_inject_launch_failure(int enable);
  *              before the first call and keeps it between calls.
  *   flags_out  NULL, or a host word that receives this call's ECHO_FLAG_*
  *              bits; when given, the call synchronizes `stream` before
- *              returning.
+ *              returning and maps the bits to its return code as
+ *              echo_get_status does: ECHO_ETIMEOUT when ECHO_FLAG_TIMEOUT is
+ *              set, else ECHO_ERANGE when ECHO_FLAG_RANGE is set. Without
+ *              flags_out nothing reports a range or timeout failure of the
+ *              call: there is no handle to query, and the next call clears
+ *              the flag word.
  * Limit: the payloads of the message must fit the scratch:
  *   echo_query_layout(n, P, group, bits, bits).workspace_bytes, about
  *   (P + 1) * ceil(n / group) * (group * bits / 8 + 4) bytes, must not exceed
@@ -377,7 +402,9 @@ ECHO_API int echo_inject_launch_failure(int enable);
  *   call's payloads; each call clears the flag word before its kernels run.
  *   Calls that overlap on the GPU (on streams with no ordering between them)
  *   race on the scratch and give undefined results: order them.
- * Errors: those of echo_allreduce_sim, plus ECHO_ENOSPACE.
+ * Errors: those of echo_allreduce_sim, plus ECHO_ENOSPACE; with flags_out,
+ *   also ECHO_ERANGE and ECHO_ETIMEOUT (data-dependent, after the call ran).
+ * Waits: the kernels' bounded waits use the default limit (1 s).
  */
 ECHO_API int echo_allreduce_sim_noalloc(const void* const* inputs, void* const* outputs, void* state_dev,
                                         int64_t n, int P, int bits, int group, float eta, float alpha_long,

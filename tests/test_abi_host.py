@@ -99,11 +99,14 @@ def test_calls_reject_missing_handle(L):
     assert L.echo_phase_gather(arr, None, 4, None) == E.ECHO_EINVAL
     assert L.echo_get_status(None, None, None) == E.ECHO_EINVAL
     assert L.echo_set_quantizer(None, E.ECHO_QUANT_NEAREST) == E.ECHO_EINVAL
+    assert L.echo_set_wait_limit(None, 1000000) == E.ECHO_EINVAL
+    assert L.echo_get_wait_limit(None) == 0
+    assert L.echo_check_watchdog(None, 0, None) == E.ECHO_EINVAL
     assert L.echo_free(None) == E.ECHO_OK
 
 
 def test_status_strings(L):
-    for code in range(5):
+    for code in range(6):
         assert E.echo_status_string(code)
     assert E.echo_status_string(99) == "unknown status"
 

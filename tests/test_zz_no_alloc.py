@@ -8,9 +8,10 @@ cudaMalloc/cudaFree. The no-allocation entry point keeps the payloads in a
 fixed scratch array inside the library, so such a caller passes only its
 inputs, outputs and EMA state. These tests call it through the C ABI and
 check that two calls in a row give exactly what the ordinary, workspace-based
-echo_allreduce_sim gives (outputs bit-identical, EMA state within the usual
-1e-6 relative bar -- in fact identical), and that a message too large for the
-scratch is refused.
+echo_allreduce_sim gives and what the oracle gives (outputs bit-identical,
+EMA state within the usual 1e-6 relative bar -- in fact identical), that a
+value outside the fp16 parameter range is reported through the call's return
+code, and that a message too large for the scratch is refused.
 
 This file is collected last on purpose: it runs alone or after everything
 else, and the shared scratch must not depend on what ran before.
@@ -19,10 +20,11 @@ import numpy as np
 import pytest
 import torch
 
+import oracle as O
 import workloads as W
 import bit_error_compensated_group_b200 as E
 from bit_error_compensated_group_b200 import echo as EE
-from parity import assert_state_close, u16
+from parity import assert_state_close, padded, u16
 
 pytestmark = pytest.mark.gpu
 
@@ -48,6 +50,10 @@ def test_noalloc_matches_workspace_entry_point(P, n, group, bits, feedback):
     if feedback:
         state_na = torch.zeros(E.echo_state_bytes(n, P, group) // 4, dtype=torch.float32, device="cuda")
     kw = dict(eta=1.0, alpha_long=0.05, alpha_short=0.5, w=0.5)
+    G = -(-n // group)
+    x_host = padded(np.stack([u16(t) for t in ins]), G * group)
+    el = np.zeros((P, G * group), np.float32) if feedback else None
+    es = np.zeros((P, G * group), np.float32) if feedback else None
     try:
         for call in range(2):
             ref(ins, out_ref, bits, **kw)
@@ -55,8 +61,10 @@ def test_noalloc_matches_workspace_entry_point(P, n, group, bits, feedback):
                                                   kw["alpha_long"], kw["alpha_short"], kw["w"])
             rc, ref_flags = ref.status()
             assert flags == 0 and ref_flags == 0 and rc == E.ECHO_OK
+            orc = O.echo_allreduce(x_host, n_total=n, group=group, bits=bits, e_long=el, e_short=es, **kw)
             for r in range(P):
                 assert np.array_equal(u16(out_na[r]), u16(out_ref[r])), f"call {call} rank {r}"
+                assert np.array_equal(u16(out_na[r]), orc.y[r, :n]), f"call {call} rank {r} vs oracle"
             if feedback:
                 got = state_na.cpu().numpy()
                 want = ref.state.cpu().numpy()
@@ -64,8 +72,32 @@ def test_noalloc_matches_workspace_entry_point(P, n, group, bits, feedback):
                 g3, w3 = got.reshape(P, 2, S)[:, :, :n], want.reshape(P, 2, S)[:, :, :n]
                 assert_state_close(g3, w3, f"EMA state call {call}")
                 assert np.array_equal(g3, w3)
+                o3 = np.stack([el[:, :n], es[:, :n]], axis=1)
+                assert_state_close(g3, o3, f"EMA state call {call} vs oracle")
     finally:
         ref.close()
+
+
+def test_noalloc_reports_range_violations_in_its_return_code():
+    """A value beyond the fp16 range (here 2^17 in rank 1's input) cannot get
+    fp16 parameters: the kernels raise the range flag, and with a flag word
+    requested the call returns ECHO_ERANGE (there is no handle to ask later).
+    The next call on ordinary inputs is clean again: each call clears the
+    flag word first."""
+    P, n, group, bits = 2, 4096, 128, 4
+    ins = _inputs(P, n, 77)
+    ins[1][300] = 2.0 ** 17
+    outs = [torch.empty_like(t) for t in ins]
+    with pytest.raises(E.EchoError) as ei:
+        EE.echo_allreduce_sim_noalloc(ins, outs, None, n, P, bits, group, 1.0, 0.05, 0.5, 0.5)
+    assert ei.value.status == EE.ECHO_ERANGE
+    ins[1][300] = 1.0
+    assert EE.echo_allreduce_sim_noalloc(ins, outs, None, n, P, bits, group, 1.0, 0.05, 0.5, 0.5) == 0
+    # without a flag word nothing reads the flags: the call itself succeeds
+    ins[1][300] = 2.0 ** 17
+    assert EE.echo_allreduce_sim_noalloc(ins, outs, None, n, P, bits, group, 1.0, 0.05, 0.5, 0.5,
+                                         read_flags=False) is None
+    torch.cuda.synchronize()
 
 
 def test_noalloc_refuses_messages_beyond_the_scratch():
