@@ -10,9 +10,14 @@ Metric: GB/s of bf16 input (all P ranks' inputs) per second.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
-With N > 1 (launched by torchrun, one process per GPU) every rank runs its own
-independent 1 GB call (the simulation shards by message, no collective on the
-data path): weak scaling, value = all ranks' input bytes / max-over-ranks time.
+With N > 1 (launched by torchrun, one process per GPU) the one 1 GB message
+is split across the GPUs by group columns (``--split columns``, the default):
+rank k runs echo_allreduce_sim_range on columns [floor(kG/N), floor((k+1)G/N))
+of the same message -- every column is independent, so there is no collective
+on the data path -- and value = the message's input bytes / max-over-ranks
+time (strong scaling). ``--split messages`` instead gives every GPU its own
+independent 1 GB message (weak scaling, value = all ranks' input bytes /
+max-over-ranks time).
 
 ``--impl reference`` times the oracle (plain C, single thread) on the host on a
 bounded sample of group columns of the same workload, rank 0 only.
@@ -35,9 +40,13 @@ if ROOT not in sys.path:
 METRIC = "Echo 4-bit all-reduce sim GB/s of bf16 input (P=8, 1 GB); % HBM roofline"
 FALLBACK_HBM_GBS = 6650.0
 
-# group columns of the workload timed on the host (one oracle call each)
+# group columns of the workload timed on the host (one oracle call each):
+# single thread, and on all cores (a chunk of columns per worker process)
 CPU_BASELINE_COLS = 1 << 17
-REFERENCE_STEP_COLS = 1 << 14
+CPU_BASELINE_COLS_PER_CORE = 1 << 13
+CPU_BASELINE_COLS_MAX = 1 << 18
+REFERENCE_STEP_COLS_PER_CORE = 1 << 11
+REFERENCE_STEP_COLS_MAX = 1 << 17
 
 
 _TOKENS = None   # --tokens: a smaller message of the same shape family (profiling only)
@@ -240,28 +249,130 @@ def cpu_sample_rate(cols, seed=123):
     return P * m * 2 / dt / 1e9, dt, P * m
 
 
+# ------------------------------------------------------------ the oracle on all host cores
+#
+# The oracle stays single-threaded and unchanged; the sample's group columns
+# are cut into one contiguous chunk per worker process (spawned, so no CUDA
+# state is inherited), every column being independent. Inputs sit in shared
+# memory; each worker copies its chunk, waits at a barrier with the others,
+# then runs the oracle on its columns. Elapsed = latest end - earliest start.
+
+def _oracle_worker(wid, shm_name, shape, barrier, tasks, results):
+    import numpy as np
+    from multiprocessing import shared_memory
+    import oracle as O
+    shm = shared_memory.SharedMemory(name=shm_name)
+    try:
+        x_all = np.ndarray(shape, dtype=np.uint16, buffer=shm.buf)
+        while True:
+            task = tasks.get()
+            if task is None:
+                break
+            lo, hi, j0, n_total, group, bits, fb = task
+            x = np.ascontiguousarray(x_all[:, lo * group:hi * group])
+            el = np.zeros(x.shape, np.float32)
+            es = np.zeros(x.shape, np.float32)
+            barrier.wait(timeout=120)
+            t0 = time.perf_counter()
+            if hi > lo:
+                O.echo_allreduce(x, n_total=n_total, group=group, bits=bits, e_long=el, e_short=es, eta=fb[0],
+                                 alpha_long=fb[1], alpha_short=fb[2], w=fb[3], j0=j0 + lo, jc=hi - lo)
+            results.put((wid, t0, time.perf_counter()))
+    finally:
+        del x_all
+        shm.close()
+
+
+class OraclePool:
+    """`workers` spawned processes, each running the oracle on its own chunk
+    of the sampled group columns of the workload."""
+
+    def __init__(self, workers, cols):
+        import multiprocessing as mp
+        import numpy as np
+        import torch
+        from multiprocessing import shared_memory
+        import workloads as W
+        w = _workload()
+        self.w = w
+        self.workers = workers
+        G = -(-w.n // w.group)
+        self.cols = min(cols, w.n // w.group)          # full groups only
+        self.j0 = G // 2 - self.cols // 2                # straddles an owner boundary at P = 8
+        m = self.cols * w.group
+        self.shm = shared_memory.SharedMemory(create=True, size=w.P * m * 2)
+        x = np.ndarray((w.P, m), dtype=np.uint16, buffer=self.shm.buf)
+        for r in range(w.P):
+            x[r] = W.bf16_bits(W.student_t3_unit_f32(m, W.seed_of(w.cid, 7, r)).to(torch.bfloat16))
+        del x
+        ctx = mp.get_context("spawn")
+        self.barrier = ctx.Barrier(workers)
+        self.results = ctx.Queue()
+        self.tasks = [ctx.Queue() for _ in range(workers)]
+        self.procs = [ctx.Process(target=_oracle_worker, daemon=True,
+                                  args=(k, self.shm.name, (w.P, m), self.barrier, self.tasks[k], self.results))
+                      for k in range(workers)]
+        for pr in self.procs:
+            pr.start()
+
+    def run(self):
+        """One pass over the sample on all workers: (GB/s of bf16 input,
+        seconds, element-ranks)."""
+        w = self.w
+        fb = (w.eta, w.alpha_long, w.alpha_short, w.w)
+        for k in range(self.workers):
+            lo, hi = k * self.cols // self.workers, (k + 1) * self.cols // self.workers
+            self.tasks[k].put((lo, hi, self.j0, w.n, w.group, w.bits, fb))
+        got = [self.results.get(timeout=600) for _ in range(self.workers)]
+        dt = max(g[2] for g in got) - min(g[1] for g in got)
+        er = w.P * self.cols * w.group
+        return er * 2 / dt / 1e9, dt, er
+
+    def close(self):
+        for q in self.tasks:
+            q.put(None)
+        for pr in self.procs:
+            pr.join(timeout=30)
+        self.shm.close()
+        self.shm.unlink()
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
 def run_reference(args):
+    """The oracle as it stands, on all the host's cores: each step one pass
+    of the worker processes over a bounded sample of group columns."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     w = _workload()
-    cols = REFERENCE_STEP_COLS
-    for _ in range(args.warmup):
-        cpu_sample_rate(cols)
-    times = []
-    for _ in range(args.steps):
-        _, dt, er = cpu_sample_rate(cols)
-        times.append(dt)
+    cores = host_cores()
+    cols = min(REFERENCE_STEP_COLS_PER_CORE * cores, REFERENCE_STEP_COLS_MAX)
+    pool = OraclePool(cores, cols)
+    try:
+        for _ in range(args.warmup):
+            pool.run()
+        times = []
+        for _ in range(args.steps):
+            _, dt, er = pool.run()
+            times.append(dt)
+    finally:
+        pool.close()
     tot = sum(times)
-    er = w.P * cols * w.group
     value = args.steps * er * 2 / tot / 1e9
-    sample = f"{cols} of {-(-w.n // w.group)} group columns x P={w.P} per step ({er} element-ranks)"
+    sample = (f"{pool.cols} of {-(-w.n // w.group)} group columns x P={w.P} per step ({er} element-ranks), "
+              f"{cores} worker processes of the single-threaded oracle, one column chunk each")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic", "config": _config(w),
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -295,20 +406,30 @@ def run_gpu(args):
 
     w = _workload()
     P, n, group, bits = w.P, w.n, w.group, w.bits
+    G = -(-n // group)
+    split_cols = world > 1 and args.split == "columns"
+    c0, c1 = E.column_window(rank, world, G) if split_cols else (0, G)
     ar = E.EchoAllReduce(n, P, group, bits, feedback=_FEEDBACK, device=dev)
     inputs = []
     for r in range(P):
-        inputs.append(W.rank_input(w, r, site=rank, device=dev))   # each GPU its own message
+        # columns: every GPU holds the same message (it touches only its
+        # window); messages: each GPU its own message
+        inputs.append(W.rank_input(w, r, site=0 if split_cols else rank, device=dev))
     outputs = [torch.empty_like(t) for t in inputs]
     stream = torch.cuda.current_stream(dev)
     h = ar.handle
     fb = (w.eta, w.alpha_long, w.alpha_short, w.w)
 
-    # one step = one echo_allreduce_sim call: the non-owners' quantize pass,
-    # then the owners' pass (a programmatic dependent of the first, which also
-    # decodes into all P outputs); events only at the step boundaries
+    # one step = one echo_allreduce_sim call (with a column split: the
+    # echo_allreduce_sim_range call on this GPU's window): the non-owners'
+    # quantize pass, then the owners' pass (a programmatic dependent of the
+    # first, which also decodes into all P outputs); events only at the step
+    # boundaries
     def call():
-        E.echo_allreduce_sim(inputs, outputs, h, n, P, bits, group, *fb, stream=stream)
+        if split_cols:
+            E.echo_allreduce_sim_range(inputs, outputs, h, n, P, bits, group, *fb, c0, c1, stream=stream)
+        else:
+            E.echo_allreduce_sim(inputs, outputs, h, n, P, bits, group, *fb, stream=stream)
 
     # the same two kernels through the phase entry points with an event
     # between them: the per-kernel split for the roofline, in a pass of its own
@@ -344,21 +465,25 @@ def run_gpu(args):
     total_ms = t0.elapsed_time(t1)
     max_ms = max_over_ranks(total_ms, world, dev)
 
+    # the per-kernel split (phase entry points over the whole message): with
+    # a column split every GPU would time the whole message, so it is left out
     phase_steps = max(3, min(args.steps, 10))
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(phase_steps)]
-    for i in range(phase_steps):
-        step(evs[i])
-    barrier()
-    per_phase = {"quantize": 0.0, "reduce_gather": 0.0}
-    for e in evs:
-        per_phase["quantize"] += e[0].elapsed_time(e[1])
-        per_phase["reduce_gather"] += e[1].elapsed_time(e[2])
+    per_phase = None
+    if not split_cols:
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(phase_steps)]
+        for i in range(phase_steps):
+            step(evs[i])
+        barrier()
+        per_phase = {"quantize": 0.0, "reduce_gather": 0.0}
+        for e in evs:
+            per_phase["quantize"] += e[0].elapsed_time(e[1])
+            per_phase["reduce_gather"] += e[1].elapsed_time(e[2])
 
     # the same message without feedback state (x' = x, no EMA traffic): its
     # time and the difference, the cost of compensation (the pages quote
     # 0.90 ms per 1 GB message on 8 A100s, fused into the entry pass)
     variant = None
-    if not args.no_variants and _FEEDBACK:
+    if not args.no_variants and _FEEDBACK and not split_cols:
         nf = E.EchoAllReduce(n, P, group, bits, feedback=False, device=dev)
         nf_steps = max(3, min(args.steps, 10))
 
@@ -392,7 +517,7 @@ def run_gpu(args):
     # the other quantizer forms (the ablations' variants) on the same call,
     # feedback on: the nearest and integer-zero forms clamp each code
     forms = None
-    if not args.no_variants and _FEEDBACK:
+    if not args.no_variants and _FEEDBACK and not split_cols:
         forms = {}
         q_steps = max(3, min(args.steps, 10))
         for name, q in (("nearest", E.ECHO_QUANT_NEAREST), ("int_zero", E.ECHO_QUANT_INT_ZERO)):
@@ -413,7 +538,7 @@ def run_gpu(args):
     # the early-site 8-bit mode on the same message, feedback on (one code
     # per byte: 22.06 algorithmic bytes per element-rank instead of 21.06)
     int8 = None
-    if not args.no_variants and _FEEDBACK:
+    if not args.no_variants and _FEEDBACK and not split_cols:
         a8 = E.EchoAllReduce(n, P, group, 8, feedback=True, device=dev)
         i8_steps = max(3, min(args.steps, 10))
 
@@ -454,18 +579,48 @@ def run_gpu(args):
     e2e = None
     host_in = host_out = None
     if not args.no_e2e:
-        # every rank pins P + 1 message buffers; the leg runs only if all could
-        # (a collective decision, so that every rank takes the same steps)
+        # every rank pins P + 1 message buffers (its window's, with a column
+        # split); the leg runs only if all could (a collective decision, so
+        # that every rank takes the same steps)
         why = None
+        hn = min(c1 * group, n) - c0 * group if split_cols else n
         try:
-            host_in = [torch.empty(n, dtype=torch.bfloat16, pin_memory=True) for _ in range(P)]
-            host_out = torch.empty(n, dtype=torch.bfloat16, pin_memory=True)
+            host_in = [torch.empty(hn, dtype=torch.bfloat16, pin_memory=True) for _ in range(P)]
+            host_out = torch.empty(hn, dtype=torch.bfloat16, pin_memory=True)
         except (RuntimeError, MemoryError) as exc:
             host_in = host_out = None
             why = f"pinned host buffers: {exc}".splitlines()[0][:200]
         if max_over_ranks(0.0 if why is None else 1.0, world, dev) > 0.0:
             e2e = {"unavailable": why or "another rank could not pin its host buffers"}
             host_in = host_out = None
+    if host_in is not None and split_cols:
+        # a column split: this GPU's window of the inputs in, its window of
+        # the result out, around the window's call (serialised on one stream)
+        e0, e1 = c0 * group, min(c1 * group, n)   # the pinned buffers hold just this window
+        e2e_steps = max(1, min(args.steps, 4))
+        for r in range(P):
+            host_in[r].copy_(inputs[r][e0:e1])
+
+        def e2e_step():
+            for r in range(P):
+                inputs[r][e0:e1].copy_(host_in[r], non_blocking=True)
+            call()
+            host_out.copy_(outputs[0][e0:e1], non_blocking=True)
+
+        e2e_step()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        b.record(stream)
+        barrier()
+        e2e_ms = max_over_ranks(a.elapsed_time(b), world, dev) / e2e_steps
+        e2e = {"value": P * n * 2 / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": P * n * 2, "d2h_bytes_per_step": n * 2,
+               "ms_per_step": e2e_ms, "steps": e2e_steps,
+               "call": "echo_allreduce_sim_range on each GPU's window, host copies of the window around it"}
+        host_in = host_out = None
     if host_in is not None:
         e2e_steps = max(1, min(args.steps, 4))
         for r in range(P):
@@ -485,7 +640,6 @@ def run_gpu(args):
         b.record(stream)
         barrier()
         e2e_ms = max_over_ranks(a.elapsed_time(b), world, dev) / e2e_steps
-        G = -(-n // group)
         chunk = args.e2e_chunk if args.e2e_chunk > 0 else -(-G // 16)
         e2e = {"value": weak_scaling_gbs(world, P * n * 2, e2e_ms), "unit": "GB/s",
                "h2d_bytes_per_step": P * n * 2, "d2h_bytes_per_step": n * 2,
@@ -495,28 +649,50 @@ def run_gpu(args):
 
     if rank == 0:
         ms = max_ms / args.steps
-        value = weak_scaling_gbs(world, P * n * 2, ms)
         peak, peak_kind = _peak_hbm()
         ab = algorithmic_bytes(P, n, group, bits, feedback=_FEEDBACK)
-        q_ms = per_phase["quantize"] / phase_steps
-        achieved = ab["quantize"] / (q_ms * 1e-3) / 1e9
         traffic = _measured_traffic() if _FEEDBACK else None
+        cfg = _config(w)
+        if split_cols:
+            # strong scaling: the one message's bytes in the slowest GPU's time;
+            # the roofline is the whole call's, per GPU (each moves 1/N of it)
+            value = P * n * 2 / (ms * 1e-3) / 1e9
+            per_gpu = ab["total"] / world / (ms * 1e-3) / 1e9
+            cfg.update(split="columns", windows=[list(E.column_window(k, world, G)) for k in range(world)])
+            roof = {"bound": "hbm", "kernel": "call (both kernels, one GPU's window)", "achieved": per_gpu,
+                    "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": per_gpu / peak, "traffic": None,
+                    "algorithmic_bytes": ab["total"] // world}
+            phases = None
+        else:
+            value = weak_scaling_gbs(world, P * n * 2, ms)
+            q_ms = per_phase["quantize"] / phase_steps
+            achieved = ab["quantize"] / (q_ms * 1e-3) / 1e9
+            if world > 1:
+                cfg.update(split="messages")
+            roof = {"bound": "hbm", "kernel": "k_quantize", "achieved": achieved, "peak": peak,
+                    "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
+                    "traffic_source": "ncu capture of a 4096-token case, scaled to the full launch by the "
+                                      "rank-groups processed (x32)",
+                    "algorithmic_bytes": ab["quantize"]}
+            phases = {k: v / phase_steps for k, v in per_phase.items()}
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": _config(w),
-            "roofline": {"bound": "hbm", "kernel": "k_quantize", "achieved": achieved, "peak": peak,
-                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
-                         "algorithmic_bytes": ab["quantize"]},
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "strong" if split_cols else "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": cfg,
+            "roofline": roof,
             "roofline_call": {"bytes": ab["total"], "achieved": ab["total"] / (ms * 1e-3) / 1e9,
                               "frac": ab["total"] / (ms * 1e-3) / 1e9 / peak},
-            "phases_ms": {k: v / phase_steps for k, v in per_phase.items()},
-            "phases_steps": phase_steps,
-            "elements_per_s": world * P * n / (ms * 1e-3),
-            "gpu_launches": 2 * args.steps if P >= 2 else args.steps,   # the timed echo_allreduce_sim calls
+            "phases_ms": phases,
+            "phases_steps": phase_steps if phases is not None else 0,
+            "elements_per_s": (1 if split_cols else world) * P * n / (ms * 1e-3),
+            "gpu_launches": 2 * args.steps if P >= 2 else args.steps,   # the timed calls' two kernels
             "clocks": clock_info, "status": rc, "flags": flags,
             "e2e": e2e,
         }
+        if split_cols:
+            line["roofline_call"] = {"bytes": ab["total"], "achieved": ab["total"] / (ms * 1e-3) / 1e9,
+                                     "frac_of_n_gpus": ab["total"] / (ms * 1e-3) / 1e9 / (peak * world)}
         if variant is not None:
             line["no_feedback"] = variant
             line["compensation_ms"] = ms - variant["ms_per_step"]
@@ -525,10 +701,20 @@ def run_gpu(args):
         if int8 is not None:
             line["int8"] = int8
         if world == 1 and not args.no_cpu_baseline:
-            gbs, dt, er = cpu_sample_rate(CPU_BASELINE_COLS)
-            line["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                                    "sample": f"{er // (P * group)} group columns x P={P} "
-                                              f"({er} element-ranks, {dt:.1f} s, single thread)"}
+            cores = host_cores()
+            pool = OraclePool(cores, min(CPU_BASELINE_COLS_PER_CORE * cores, CPU_BASELINE_COLS_MAX))
+            try:
+                gbs, dt, er = pool.run()
+            finally:
+                pool.close()
+            line["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                                    "sample": f"{er // (P * group)} group columns x P={P} ({er} element-ranks, "
+                                              f"{dt:.2f} s on {cores} worker processes of the single-threaded "
+                                              f"oracle, one column chunk each)"}
+            gbs1, dt1, er1 = cpu_sample_rate(CPU_BASELINE_COLS)
+            line["cpu_baseline_1core"] = {"value": gbs1, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                          "sample": f"{er1 // (P * group)} group columns x P={P} "
+                                                    f"({er1} element-ranks, {dt1:.1f} s, single thread)"}
         print(json.dumps(line), flush=True)
     ar.close()
     if world > 1:
@@ -840,6 +1026,9 @@ def main():
                     help="print one rank's kernel times of a multi-GPU call (rank 0 of P = 8, 1 GB) instead")
     ap.add_argument("--workloads", action="store_true",
                     help="print every workload's GPU and oracle time per call instead of the main line")
+    ap.add_argument("--split", choices=["columns", "messages"], default="columns",
+                    help="with N > 1 GPUs: split the one message by group columns (strong scaling, default) "
+                         "or give every GPU its own message (weak scaling)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="tokens per rank (default 131072, the 1 GB message); smaller values are for profiling")
     args = ap.parse_args()

@@ -8,7 +8,7 @@ and raises if the library is missing.
 from .echo import (  # noqa: F401
     ECHO_EINVAL, ECHO_ECUDA, ECHO_ENOSPACE, ECHO_ERANGE, ECHO_ETIMEOUT, ECHO_FLAG_RANGE, ECHO_FLAG_TIMEOUT,
     ECHO_MAX_RANKS, ECHO_NOALLOC_SCRATCH_BYTES, ECHO_OK, ECHO_QUANT_DIRECTED, ECHO_QUANT_INT_ZERO, ECHO_QUANT_NEAREST,
-    EchoAllReduce, EchoError, EchoLayout, EchoRank, EchoRankLayout, ExchangePlan,
+    EchoAllReduce, EchoError, EchoLayout, EchoRank, EchoRankLayout, ExchangePlan, column_window,
     echo_allreduce_sim, echo_allreduce_sim_host, echo_allreduce_sim_noalloc, echo_allreduce_sim_range,
     echo_check_watchdog, echo_free, echo_get_status, echo_get_wait_limit, echo_init_rank, echo_init_state,
     echo_inject_launch_failure, echo_phase_gather, echo_phase_quantize, echo_phase_reduce, echo_query_layout,

@@ -202,6 +202,18 @@ def echo_allreduce_sim_range(inputs: Sequence, outputs: Sequence, st, n: int, P:
                                           _stream(stream)), "echo_allreduce_sim_range")
 
 
+def column_window(rank: int, world: int, G: int):
+    """Group columns ``[c0, c1)`` that GPU ``rank`` of ``world`` takes when one
+    message is split across GPUs: contiguous ranges ``[floor(rank G / world),
+    floor((rank + 1) G / world))``. They tile ``[0, G)`` in rank order; each
+    GPU runs ``echo_allreduce_sim_range`` on its window of the same message
+    (every column is independent: all P ranks' group j, their payloads and
+    EMA rows), so no collective is needed on the data path."""
+    if world < 1 or not 0 <= rank < world or G < 0:
+        raise ValueError("column_window: need 0 <= rank < world and G >= 0")
+    return rank * G // world, (rank + 1) * G // world
+
+
 def _host_ptr(t) -> int:
     if isinstance(t, int):
         return t

@@ -23,6 +23,7 @@ def _last_json(out: str) -> dict:
 
 
 def test_reference_arm_line():
+    sys.path.insert(0, ROOT)
     env = dict(os.environ, RANK="0", WORLD_SIZE="1")
     out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "0"],
                          cwd=ROOT, env=env, capture_output=True, text=True, timeout=600, check=True).stdout
@@ -32,7 +33,8 @@ def test_reference_arm_line():
                 "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
         assert key in line, key
     assert line["value"] > 0 and line["cpu_baseline"]["value"] == line["value"]
-    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
+    import bench
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == bench.host_cores()
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
     assert line["config"]["workload"] == "p8_1GB_student_t"
 
@@ -51,7 +53,9 @@ def test_main_arm_line():
     r = line["roofline"]
     assert r["bound"] == "hbm" and r["unit"] == "GB/s" and 0 < r["frac"] == pytest.approx(r["achieved"] / r["peak"])
     assert line["e2e"]["value"] > 0 and line["e2e"]["h2d_bytes_per_step"] == 8 * 2048 * 4096 * 2
-    assert line["cpu_baseline"]["kind"] == "oracle"
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["cpu_baseline_1core"]["cores"] == 1
+    assert line["scaling"] == "weak" and line["roofline"]["traffic_source"]
 
 
 def test_algorithmic_bytes_match_the_roofline_definition():

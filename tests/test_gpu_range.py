@@ -233,3 +233,38 @@ def test_host_call_forms(to_host, streams):
             compare(gpu, orc, el, es, n, G, P, p, True, f"{streams} call {c}")
     finally:
         gpu.close()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_column_split_across_gpus(world):
+    """The benchmark's split of one message over N GPUs, on one GPU: N
+    separate handles (each with its own EMA state and workspace, as on
+    separate GPUs) run echo_allreduce_sim_range on their column windows
+    (column_window); their windows of the outputs and state, put together,
+    are the oracle's whole call, twice in a row."""
+    P, n, group = 8, 8192 * 5 + 77, 128
+    p = Params()
+    G = -(-n // group)
+    ld = G * group
+    x = random_inputs(P, n, 4242, 1.5)
+    xb = padded(u16(x), ld)
+    el, es = np.zeros((P, ld), np.float32), np.zeros((P, ld), np.float32)
+    gpus = [GpuEcho(P, n) for _ in range(world)]
+    try:
+        wins = [E.column_window(k, world, G) for k in range(world)]
+        for g in gpus:
+            g.set_inputs(x)
+            g.set_state(el, es)
+        for call in range(2):
+            for g, (c0, c1) in zip(gpus, wins):
+                run_windows(g, p, [(c0, c1)])
+            orc = O.echo_allreduce(xb, n_total=n, group=group, bits=4, e_long=el, e_short=es)
+            for g, (c0, c1) in zip(gpus, wins):
+                assert g.status() == (E.ECHO_OK, 0)
+                sl = slice(c0 * group, min(c1 * group, n))
+                assert np.array_equal(g.outputs_u16()[:, sl], orc.y[:, sl]), (call, c0, c1)
+                gl, gs = g.state()
+                assert np.array_equal(gl[:, sl], el[:, sl]) and np.array_equal(gs[:, sl], es[:, sl]), (call, c0, c1)
+    finally:
+        for g in gpus:
+            g.close()
