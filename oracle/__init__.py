@@ -73,6 +73,8 @@ def lib() -> ctypes.CDLL:
             P, P, P, P, P, P, P, P,
         ]
         L.oracle_echo_allreduce_q.restype = ctypes.c_int
+        L.oracle_bf16_allreduce.argtypes = [ctypes.c_int, ctypes.c_longlong, P, P]
+        L.oracle_bf16_allreduce.restype = None
         _lib = L
     return _lib
 
@@ -224,3 +226,14 @@ def echo_allreduce(x: np.ndarray, *, n_total: int, group: int, bits: int,
 
 def library_path() -> str:
     return os.path.abspath(_build.LIB)
+
+
+def bf16_allreduce(x: np.ndarray) -> np.ndarray:
+    """The 16-bit baseline all-reduce over the rows of ``x`` ([P][n] uint16
+    bf16 bit patterns): every row of the result is bf16_rn of the binary32
+    sum in rank order."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    P, n = x.shape
+    y = np.zeros((P, n), np.uint16)
+    lib().oracle_bf16_allreduce(P, n, _ptr(x), _ptr(y))
+    return y

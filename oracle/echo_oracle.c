@@ -77,6 +77,13 @@
  *      codes clamp(rint(v * inv) + zp, 0, Q); dequantization (code - zp) * s,
  *      exact in binary32. The parameter pair carries {s, zp} with zp as an
  *      unsigned 16-bit integer in place of z.
+ *
+ * The 16-bit baseline the pages compare Echo against ([ABS]; [EXP] results
+ * table: "16-bit NCCL all-reduce"), simulated the same way over P virtual
+ * ranks: every rank receives bf16_rn(sum_r float(x_r)), the binary32 sum in
+ * rank order 0, 1, ..., P-1 (R15: the pages fix neither the order nor the
+ * accumulation precision of that all-reduce; this reading takes the same
+ * order and precision as R6, so that the two differ only by quantization).
  */
 #include <math.h>
 #include <stdint.h>
@@ -725,4 +732,29 @@ int oracle_echo_allreduce(int P, long long n_total, int group, int bits,
     return oracle_echo_allreduce_q(P, n_total, group, bits, ORACLE_Q_DIRECTED, j0, jc, x, y, e_long, e_short,
                                    eta, alpha_long, alpha_short, w, a2a_codes, a2a_params, gather_codes,
                                    gather_params, xprime, rho, passes, flags);
+}
+
+/* ------------------------------------------------------------------ */
+/* The 16-bit baseline all-reduce (reading R15)                         */
+/* ------------------------------------------------------------------ */
+
+/* x: P rows of n bf16 bit patterns (row r at x + r * n); y: P rows of n, every
+ * row receives the same bf16 result. */
+void oracle_bf16_allreduce(int P, long long n, const uint16_t* x, uint16_t* y)
+{
+    for (long long i = 0; i < n; i++) {
+        float sum = 0.0f;
+        for (int r = 0; r < P; r++) {
+            float v = oracle_bf16_to_f32(x[(size_t)r * (size_t)n + (size_t)i]);
+            if (r == 0) {
+                sum = v;
+            } else {
+                sum = sum + v;
+            }
+        }
+        uint16_t out = oracle_f32_to_bf16(sum);
+        for (int r = 0; r < P; r++) {
+            y[(size_t)r * (size_t)n + (size_t)i] = out;
+        }
+    }
 }

@@ -68,11 +68,15 @@ MUTANTS = {
                         "        for (int rr = 0; rr < P; rr++) {\n            int r = (o + 1 + rr) % P;\n            size_t base = (size_t)r * (size_t)ld + (size_t)(jl * group);\n            if (r == o) {"),
                        ("                if (r == 0) {\n                    sum[i] = vtmp[i];",
                         "                if (rr == 0) {\n                    sum[i] = vtmp[i];")],
+    "bf16_baseline_reverse_order": [("        for (int r = 0; r < P; r++) {\n            float v = oracle_bf16_to_f32(x[(size_t)r * (size_t)n + (size_t)i]);\n            if (r == 0) {",
+                                     "        for (int r = P - 1; r >= 0; r--) {\n            float v = oracle_bf16_to_f32(x[(size_t)r * (size_t)n + (size_t)i]);\n            if (r == P - 1) {")],
+    "bf16_baseline_drops_a_rank": [("            float v = oracle_bf16_to_f32(x[(size_t)r * (size_t)n + (size_t)i]);\n            if (r == 0) {",
+                                    "            float v = r == P - 1 && P > 1 ? 0.0f : oracle_bf16_to_f32(x[(size_t)r * (size_t)n + (size_t)i]);\n            if (r == 0) {")],
     "ema_incremental_form": [("        float u = keep * e[i];\n        float v = alpha * rho[i];\n        e[i] = u + v;",
                               "        float d = rho[i] - e[i];\n        float v = alpha * d;\n        e[i] = e[i] + v;\n        (void)keep;")],
 }
 
-PIN_FILES = ["tests/test_oracle_order.py", "tests/test_oracle_call.py", "tests/test_oracle_quantizer.py", "tests/test_oracle_variants.py",
+PIN_FILES = ["tests/test_oracle_order.py", "tests/test_oracle_bf16.py", "tests/test_oracle_call.py", "tests/test_oracle_quantizer.py", "tests/test_oracle_variants.py",
              "tests/test_oracle_chain.py", "tests/test_oracle_convert.py"]
 
 
