@@ -285,26 +285,34 @@ def _oracle_worker(wid, shm_name, shape, barrier, tasks, results):
 
 class OraclePool:
     """`workers` spawned processes, each running the oracle on its own chunk
-    of the sampled group columns of the workload."""
+    of group columns: by default a sample of `cols` columns of the benchmark
+    workload; with `x` (a [P][cols * group] bf16-bit array of workload `w`,
+    columns from `j0`), those columns."""
 
-    def __init__(self, workers, cols):
+    def __init__(self, workers, cols, w=None, x=None, j0=None):
         import multiprocessing as mp
         import numpy as np
         import torch
         from multiprocessing import shared_memory
         import workloads as W
-        w = _workload()
+        w = _workload() if w is None else w
         self.w = w
         self.workers = workers
         G = -(-w.n // w.group)
-        self.cols = min(cols, w.n // w.group)          # full groups only
-        self.j0 = G // 2 - self.cols // 2                # straddles an owner boundary at P = 8
+        if x is None:
+            self.cols = min(cols, w.n // w.group)          # full groups only
+            self.j0 = G // 2 - self.cols // 2                # straddles an owner boundary at P = 8
+        else:
+            self.cols, self.j0 = cols, j0
         m = self.cols * w.group
         self.shm = shared_memory.SharedMemory(create=True, size=w.P * m * 2)
-        x = np.ndarray((w.P, m), dtype=np.uint16, buffer=self.shm.buf)
+        xs = np.ndarray((w.P, m), dtype=np.uint16, buffer=self.shm.buf)
         for r in range(w.P):
-            x[r] = W.bf16_bits(W.student_t3_unit_f32(m, W.seed_of(w.cid, 7, r)).to(torch.bfloat16))
-        del x
+            if x is None:
+                xs[r] = W.bf16_bits(W.student_t3_unit_f32(m, W.seed_of(w.cid, 7, r)).to(torch.bfloat16))
+            else:
+                xs[r] = x[r]
+        del xs
         ctx = mp.get_context("spawn")
         self.barrier = ctx.Barrier(workers)
         self.results = ctx.Queue()
@@ -315,14 +323,14 @@ class OraclePool:
         for pr in self.procs:
             pr.start()
 
-    def run(self):
-        """One pass over the sample on all workers: (GB/s of bf16 input,
+    def run(self, bits=None):
+        """One pass over the columns on all workers: (GB/s of bf16 input,
         seconds, element-ranks)."""
         w = self.w
         fb = (w.eta, w.alpha_long, w.alpha_short, w.w)
         for k in range(self.workers):
             lo, hi = k * self.cols // self.workers, (k + 1) * self.cols // self.workers
-            self.tasks[k].put((lo, hi, self.j0, w.n, w.group, w.bits, fb))
+            self.tasks[k].put((lo, hi, self.j0, w.n, w.group, w.bits if bits is None else bits, fb))
         got = [self.results.get(timeout=600) for _ in range(self.workers)]
         dt = max(g[2] for g in got) - min(g[1] for g in got)
         er = w.P * self.cols * w.group
@@ -854,6 +862,8 @@ def run_workloads(args):
             G = -(-n // group)
             x = np.zeros((P, G * group), np.uint16)
             x[:, :n] = W.bf16_bits(W.inputs(w, 0, "cpu"))
+            cores = host_cores()
+            pool = OraclePool(min(cores, G), G, w=w, x=x, j0=0) if G > 1 else None
             for bits in widths:
                 el = np.zeros((P, G * group), np.float32)
                 es = np.zeros((P, G * group), np.float32)
@@ -863,8 +873,109 @@ def run_workloads(args):
                 dt = time.perf_counter() - t0
                 entry["per_call"][f"int{bits}"]["oracle_ms"] = dt * 1e3
                 entry["per_call"][f"int{bits}"]["oracle_cores"] = 1
+                if pool is not None:
+                    _, dtn, _ = pool.run(bits)
+                    entry["per_call"][f"int{bits}"]["oracle_ms_all_cores"] = dtn * 1e3
+                    entry["per_call"][f"int{bits}"]["oracle_all_cores"] = pool.workers
+            if pool is not None:
+                pool.close()
         out[w.name] = entry
     print(json.dumps({"workloads": out, "peak_gbs": peak, "peak_kind": peak_kind, "data": "synthetic"}), flush=True)
+
+
+def run_background(args):
+    """The background-traffic study on one GPU (the Echo abstract and the
+    explainer's results section: the gain over a 16-bit all-reduce grows
+    with competing traffic). For each load level L (% duty cycle of an HBM
+    copy running on its own stream: copy for L % of every 100 us period,
+    sleep for the rest), the Echo call (with and without feedback) and the
+    16-bit baseline all-reduce of the same message are timed on the main
+    stream while the copy runs. The copy's own bandwidth is measured alone
+    and during the timed calls."""
+    import torch
+    import workloads as W
+    import bit_error_compensated_group_b200 as E
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = _workload()
+    P, n, group, bits = w.P, w.n, w.group, w.bits
+    fb = (w.eta, w.alpha_long, w.alpha_short, w.w)
+    peak, peak_kind = _peak_hbm()
+    inputs = [W.rank_input(w, r, 0, dev) for r in range(P)]
+    outputs = [torch.empty_like(t) for t in inputs]
+    ar = E.EchoAllReduce(n, P, group, bits, feedback=True, device=dev)
+    nf = E.EchoAllReduce(n, P, group, bits, feedback=False, device=dev)
+    bg_bytes = 2 << 30
+    src = torch.randint(0, 255, (bg_bytes,), dtype=torch.uint8, device=dev)
+    dst = torch.empty_like(src)
+    moved = torch.zeros(1, dtype=torch.int64, device=dev)
+    main, side = torch.cuda.current_stream(dev), torch.cuda.Stream(dev)
+    steps = max(3, args.steps)
+    calls = {
+        "echo": lambda: E.echo_allreduce_sim(inputs, outputs, ar.handle, n, P, bits, group, *fb, stream=main),
+        "echo_no_feedback": lambda: E.echo_allreduce_sim(inputs, outputs, nf.handle, n, P, bits, group, *fb,
+                                                          stream=main),
+        "bf16": lambda: E.echo_bf16_allreduce_sim(inputs, outputs, n, P, stream=main),
+    }
+    for f in calls.values():                      # warm-up without load
+        for _ in range(args.warmup):
+            f()
+    torch.cuda.synchronize(dev)
+    # the foreground time at no load, to size the copy's duration
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(main)
+    for f in calls.values():
+        for _ in range(steps + 1):
+            f()
+    b.record(main)
+    torch.cuda.synchronize(dev)
+    window_us = int(a.elapsed_time(b) * 1e3)
+    period_us = 100
+    levels = [int(v) for v in str(args.background).split(",") if v.strip()]
+    out = {"loads_pct": levels, "period_us": period_us}
+    for key in list(calls) + ["background_alone", "background_during"]:
+        out[key] = []
+    for lv in levels:
+        # the copy alone: its bandwidth at this duty cycle
+        moved.zero_()
+        alone_us = 20000
+        E.echo_background_traffic(src, dst, 10 * lv, period_us, alone_us, moved, stream=side)
+        torch.cuda.synchronize(dev)
+        out["background_alone"].append(int(moved.item()) / (alone_us * 1e-6) / 1e9)
+        # the calls while the copy runs (its duration covers them even if they slow down 4x)
+        moved.zero_()
+        dur_us = 4 * window_us + 20000
+        E.echo_background_traffic(src, dst, 10 * lv, period_us, dur_us, moved, stream=side)
+        for key, f in calls.items():
+            f()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(main)
+            for _ in range(steps):
+                f()
+            e1.record(main)
+            e1.synchronize()
+            out[key].append(e0.elapsed_time(e1) / steps)
+        torch.cuda.synchronize(dev)
+        out["background_during"].append(int(moved.item()) / (dur_us * 1e-6) / 1e9 if lv else 0.0)
+    for key in calls:
+        base = out[key][levels.index(0)] if 0 in levels else out[key][0]
+        out[key + "_slowdown"] = [t / base for t in out[key]]
+    out["bf16_over_echo"] = [bt / et for bt, et in zip(out["bf16"], out["echo"])]
+    out["bf16_over_echo_no_feedback"] = [bt / et for bt, et in zip(out["bf16"], out["echo_no_feedback"])]
+    ab = algorithmic_bytes(P, n, group, bits)
+    out["algorithmic_bytes"] = {"echo": ab["total"],
+                                "echo_no_feedback": algorithmic_bytes(P, n, group, bits, feedback=False)["total"],
+                                "bf16": 2 * P * n * 2}
+    ar.close()
+    nf.close()
+    rc = 0
+    print(json.dumps({"background": out, "unit": "ms per call", "steps": steps, "warmup": args.warmup,
+                      "config": _config(w), "peak_gbs": peak, "peak_kind": peak_kind, "data": "synthetic",
+                      "status": rc}), flush=True)
+
+
+def _chunk_counts(args):
+    return [int(c) for c in str(args.chunks).split(",") if c.strip()]
 
 
 def run_ranks(args):
@@ -923,12 +1034,40 @@ def run_ranks(args):
         nbytes = [(G - seg) * (2 * group + st * group + pb),                        # x, EMAs, send row
                   seg * (2 * group + st * group + (P - 1) * pb + pb),               # x, EMAs, received rows, gather send
                   G * (pb + 2 * group)]                                            # gathered rows, output
+        # the same kernels of rank 0 cut into column chunks (the chunked call's
+        # compute side; its exchanges need P GPUs and are not timed here)
+        per_chunks = {}
+        for chunks in _chunk_counts(args):
+            if chunks == 1:
+                continue
+            cevs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+            for i in range(args.warmup + steps):
+                e = cevs[i - args.warmup] if i >= args.warmup else None
+                if e:
+                    e[0].record(s)
+                for c in range(chunks):
+                    r0.quantize_chunk(xs[0], c, chunks, bits, *fb)
+                if e:
+                    e[1].record(s)
+                for c in range(chunks):
+                    r0.reduce_chunk(xs[0], ys[0], c, chunks, bits, *fb)
+                if e:
+                    e[2].record(s)
+                for c in range(chunks):
+                    r0.decode_chunk(ys[0], c, chunks, bits)
+                if e:
+                    e[3].record(s)
+            torch.cuda.synchronize(dev)
+            cms = [sum(e[k].elapsed_time(e[k + 1]) for e in cevs) / steps for k in range(3)]
+            per_chunks[str(chunks)] = {"phases_ms": {"quantize": cms[0], "reduce": cms[1], "decode": cms[2]},
+                                       "ms": sum(cms)}
         rc, flags = r0.status()
         out["feedback" if feedback else "no_feedback"] = {
             "phases_ms": {"quantize": ms[0], "reduce": ms[1], "decode": ms[2]}, "ms": sum(ms),
             "algorithmic_bytes": {"quantize": nbytes[0], "reduce": nbytes[1], "decode": nbytes[2]},
             "roofline_frac": {k: b / (t * 1e-3) / 1e9 / peak for k, b, t in zip(("quantize", "reduce", "decode"),
                                                                                nbytes, ms)},
+            "chunked_kernels": per_chunks,
             "status": rc, "flags": flags}
         for rk in ranks:
             rk.close()
@@ -948,8 +1087,10 @@ def run_dist(args):
     comparison): under torchrun, P = world size, one rank per GPU, each with
     its own 1 GB bf16 message (the same workload as the main line; rank r's
     input is the workload's rank r). Times, on each rank's stream and as the
-    max over ranks, EchoRank.allreduce with and without feedback and
-    torch.distributed.all_reduce (SUM) of the same bf16 tensor."""
+    max over ranks, EchoRank.allreduce with and without feedback -- whole,
+    and cut into each of --chunks column chunks with chunk c's exchanges
+    overlapping chunk c + 1's kernels -- and torch.distributed.all_reduce
+    (SUM) of the same bf16 tensor."""
     import torch
     import torch.distributed as dist
     import workloads as W
@@ -985,9 +1126,12 @@ def run_dist(args):
         return max_over_ranks(a.elapsed_time(b) / steps, world, dev)
 
     out = {}
+    comm = torch.cuda.Stream(dev)
     for feedback in (True, False):
         er = E.EchoRank(n, world, rank, group, bits, feedback, device=dev)
-        out["echo_feedback" if feedback else "echo_no_feedback"] = timed(lambda: er.allreduce(x, y, bits, *fb))
+        for chunks in _chunk_counts(args):
+            key = ("echo_feedback" if feedback else "echo_no_feedback") + ("" if chunks == 1 else f"_chunks{chunks}")
+            out[key] = timed(lambda: er.allreduce(x, y, bits, *fb, chunks=chunks, comm_stream=comm))
         rc, flags = er.status()
         er.close()
         del er
@@ -996,8 +1140,8 @@ def run_dist(args):
     out["nccl_bf16_all_reduce"] = timed(lambda: dist.all_reduce(z))
     if rank == 0:
         line = {"dist": {k: {"ms_per_call": v, "gbs_bf16_per_rank": n * 2 / (v * 1e-3) / 1e9} for k, v in out.items()},
-                "speedup_vs_nccl_bf16": {k: out["nccl_bf16_all_reduce"] / out[k] for k in ("echo_feedback",
-                                                                                         "echo_no_feedback")},
+                "speedup_vs_nccl_bf16": {k: out["nccl_bf16_all_reduce"] / v for k, v in out.items()
+                                         if k.startswith("echo")},
                 "n_gpus": world, "P": world, "steps": steps, "warmup": args.warmup,
                 "config": {"workload": w.name, "n": n, "group": group, "bits": bits}, "data": "synthetic"}
         print(json.dumps(line), flush=True)
@@ -1026,6 +1170,10 @@ def main():
                     help="print one rank's kernel times of a multi-GPU call (rank 0 of P = 8, 1 GB) instead")
     ap.add_argument("--workloads", action="store_true",
                     help="print every workload's GPU and oracle time per call instead of the main line")
+    ap.add_argument("--background", default=None,
+                    help="background-traffic study: comma-separated load levels in %% (e.g. 0,25,50,75,100)")
+    ap.add_argument("--chunks", default="1,4,16",
+                    help="--dist / --ranks: column-chunk counts of the multi-GPU call (comma-separated)")
     ap.add_argument("--split", choices=["columns", "messages"], default="columns",
                     help="with N > 1 GPUs: split the one message by group columns (strong scaling, default) "
                          "or give every GPU its own message (weak scaling)")
@@ -1043,6 +1191,8 @@ def main():
         run_workloads(args)
     elif args.ranks:
         run_ranks(args)
+    elif args.background is not None:
+        run_background(args)
     elif args.dist:
         run_dist(args)
     else:

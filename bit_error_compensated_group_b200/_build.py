@@ -16,7 +16,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libecho_b200.so")
 SOURCES = ["echo_api.cu"]
-HEADERS = ["echo_kernels.cuh", "echo_pipeline.cuh"]
+HEADERS = ["echo_kernels.cuh", "echo_pipeline.cuh", "echo_traffic.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = [

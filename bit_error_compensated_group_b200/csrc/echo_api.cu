@@ -13,6 +13,7 @@
 #include "echo.h"
 #include "echo_kernels.cuh"
 #include "echo_pipeline.cuh"
+#include "echo_traffic.cuh"
 
 struct echo_state {
     int64_t n;
@@ -104,9 +105,10 @@ enum class Stage { Quantize, Reduce, Gather };
 // An upper bound on the tiles a pipelined launch walks: the runs (2 per rank
 // for quantize, 1 per owner for reduce) cut into tiles of `tile_groups`.
 int64_t tile_bound(Stage stage, const echo_dev::Args& a, int tile_groups) {
-    const int64_t cols = a.c1 - a.c0;   // the call's group-column window
+    int64_t cols = a.c1 - a.c0;   // the call's group-column window
+    if (a.chunk_k > 0) cols = cols / a.chunk_k + a.P;   // every owner's part of one chunk
     const int64_t groups = stage == Stage::Quantize ? (int64_t)(a.P - 1) * cols : cols;
-    const int64_t runs = stage == Stage::Quantize ? 2 * (int64_t)a.P : a.P;
+    const int64_t runs = stage == Stage::Quantize ? (a.chunk_k > 0 ? (int64_t)a.P * a.P : 2 * (int64_t)a.P) : a.P;
     return groups / tile_groups + runs + 1;
 }
 
@@ -408,6 +410,19 @@ bool make_rank_args(const echo_state* st, int bits, RankPhase phase, const void*
     return true;
 }
 
+// One chunk of a chunked rank call: chunk `chunk` of `chunks` of every
+// owner's segment; the partial last group (the last group of the last
+// owner's segment) belongs to the last chunk.
+bool set_chunk(echo_dev::Args* a, const echo_state* st, int chunk, int chunks) {
+    if (chunks < 1 || chunks > ECHO_MAX_CHUNKS || chunk < 0 || chunk >= chunks) return false;
+    if (chunks == 1) return true;   // the whole call
+    a->chunk_i = chunk;
+    a->chunk_k = chunks;
+    const int64_t full = st->n / st->group;
+    a->tail = (full < st->G && chunk == chunks - 1) ? 1 : 0;
+    return true;
+}
+
 bool sim_handle(const echo_state* st) { return st && st->rank < 0; }
 bool rank_handle(const echo_state* st) { return st && st->rank >= 0; }
 
@@ -668,20 +683,21 @@ int echo_init_rank(echo_state** out, int64_t n, int P, int rank, int group, int 
     return ECHO_OK;
 }
 
-int echo_rank_quantize(const void* x, echo_state* st, int bits, float eta, float alpha_long, float alpha_short,
-                       float w, echo_stream_t stream) {
+int echo_rank_quantize_chunk(const void* x, echo_state* st, int bits, float eta, float alpha_long,
+                             float alpha_short, float w, int chunk, int chunks, echo_stream_t stream) {
     if (!rank_handle(st) || !x || !valid_bits(bits) || bits > st->max_bits) return ECHO_EINVAL;
     if (!valid_feedback(eta, alpha_long, alpha_short, w)) return ECHO_EINVAL;
     echo_dev::Args a;
     if (!make_rank_args(st, bits, RankPhase::Quantize, x, nullptr, eta, alpha_long, alpha_short, w, &a))
         return ECHO_EINVAL;
+    if (!set_chunk(&a, st, chunk, chunks)) return ECHO_EINVAL;
     if (int rc = set_device(st)) return rc;
     if (st->P < 2) return ECHO_OK;
     return launch(Stage::Quantize, bits, a, st, reinterpret_cast<cudaStream_t>(stream));
 }
 
-int echo_rank_reduce(const void* x, void* out, echo_state* st, int bits, float eta, float alpha_long,
-                     float alpha_short, float w, echo_stream_t stream) {
+int echo_rank_reduce_chunk(const void* x, void* out, echo_state* st, int bits, float eta, float alpha_long,
+                           float alpha_short, float w, int chunk, int chunks, echo_stream_t stream) {
     if (!rank_handle(st) || !x || !valid_bits(bits) || bits > st->max_bits) return ECHO_EINVAL;
     if (st->P == 1 && !out) return ECHO_EINVAL;
     if (!valid_feedback(eta, alpha_long, alpha_short, w)) return ECHO_EINVAL;
@@ -689,17 +705,115 @@ int echo_rank_reduce(const void* x, void* out, echo_state* st, int bits, float e
     if (!make_rank_args(st, bits, RankPhase::Reduce, x, st->P == 1 ? out : nullptr, eta, alpha_long, alpha_short,
                         w, &a))
         return ECHO_EINVAL;
+    if (!set_chunk(&a, st, chunk, chunks)) return ECHO_EINVAL;
     if (int rc = set_device(st)) return rc;
     return launch(Stage::Reduce, bits, a, st, reinterpret_cast<cudaStream_t>(stream));
 }
 
-int echo_rank_decode(void* out, echo_state* st, int bits, echo_stream_t stream) {
+int echo_rank_decode_chunk(void* out, echo_state* st, int bits, int chunk, int chunks, echo_stream_t stream) {
     if (!rank_handle(st) || !out || !valid_bits(bits) || bits > st->max_bits) return ECHO_EINVAL;
     echo_dev::Args a;
     if (!make_rank_args(st, bits, RankPhase::Decode, nullptr, out, 0.0f, 0.0f, 0.0f, 0.0f, &a)) return ECHO_EINVAL;
+    if (!set_chunk(&a, st, chunk, chunks)) return ECHO_EINVAL;
     if (int rc = set_device(st)) return rc;
     if (st->P < 2) return ECHO_OK;
     return launch(Stage::Gather, bits, a, st, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int echo_rank_quantize(const void* x, echo_state* st, int bits, float eta, float alpha_long, float alpha_short,
+                       float w, echo_stream_t stream) {
+    return echo_rank_quantize_chunk(x, st, bits, eta, alpha_long, alpha_short, w, 0, 1, stream);
+}
+
+int echo_rank_reduce(const void* x, void* out, echo_state* st, int bits, float eta, float alpha_long,
+                     float alpha_short, float w, echo_stream_t stream) {
+    return echo_rank_reduce_chunk(x, out, st, bits, eta, alpha_long, alpha_short, w, 0, 1, stream);
+}
+
+int echo_rank_decode(void* out, echo_state* st, int bits, echo_stream_t stream) {
+    return echo_rank_decode_chunk(out, st, bits, 0, 1, stream);
+}
+
+int echo_query_chunk(int64_t n, int P, int group, int owner, int chunk, int chunks, int64_t* first,
+                     int64_t* count) {
+    if (!first || !count || !valid_sizes(n, P, group) || owner < 0 || owner >= P) return ECHO_EINVAL;
+    if (chunks < 1 || chunks > ECHO_MAX_CHUNKS || chunk < 0 || chunk >= chunks) return ECHO_EINVAL;
+    const int64_t G = (n + group - 1) / group;
+    const int64_t len = (int64_t)(owner + 1) * G / P - (int64_t)owner * G / P;
+    const int64_t b = (int64_t)chunk * len / chunks, e = (int64_t)(chunk + 1) * len / chunks;
+    *first = b;
+    *count = e - b;
+    return ECHO_OK;
+}
+
+namespace {
+
+// SM count of the current device, looked up once per device.
+int device_sms(int* dev_out) {
+    static int sms[kMaxDevices];
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+    if (sms[dev] == 0) {
+        int c = 0;
+        if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        sms[dev] = c;
+    }
+    *dev_out = dev;
+    return sms[dev];
+}
+
+}  // namespace
+
+int echo_bf16_allreduce_sim(const void* const* inputs, void* const* outputs, int64_t n, int P,
+                            echo_stream_t stream) {
+    if (!inputs || !outputs || n < 1 || n >= kMaxN || P < 1 || P > ECHO_MAX_RANKS) return ECHO_EINVAL;
+    echo_dev::Args a;
+    std::memset(&a, 0, sizeof(a));
+    for (int r = 0; r < P; ++r) {
+        if (!inputs[r] || !outputs[r] || !aligned(inputs[r], 16) || !aligned(outputs[r], 16)) return ECHO_EINVAL;
+        a.in[r] = static_cast<const uint16_t*>(inputs[r]);
+        a.out[r] = static_cast<uint16_t*>(outputs[r]);
+    }
+    a.n = n;
+    a.P = P;
+    if (g_fail_launches.load(std::memory_order_relaxed)) return ECHO_ECUDA;
+    int dev = 0;
+    const int sms = device_sms(&dev);
+    if (sms == 0) return ECHO_ECUDA;
+    static int per_sm[kMaxDevices];
+    if (per_sm[dev] == 0) {
+        int b = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, echo_dev::k_bf16_allreduce_sim, echo_dev::kBf16Threads,
+                                                          0) != cudaSuccess || b < 1)
+            b = 1;
+        per_sm[dev] = b;
+    }
+    const int64_t need = (n / 8 + echo_dev::kBf16Threads - 1) / echo_dev::kBf16Threads;
+    const int grid = (int)(need < (int64_t)sms * per_sm[dev] ? (need > 0 ? need : 1) : (int64_t)sms * per_sm[dev]);
+    echo_dev::k_bf16_allreduce_sim<<<grid, echo_dev::kBf16Threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+    return cuda_status(cudaGetLastError());
+}
+
+int echo_background_traffic(const void* src, void* dst, size_t bytes, uint32_t duty_permille, uint32_t period_us,
+                            uint32_t duration_us, unsigned long long* moved_dev, echo_stream_t stream) {
+    if (!src || !dst || !aligned(src, 16) || !aligned(dst, 16) || bytes < 16 || bytes % 16 != 0) return ECHO_EINVAL;
+    const uintptr_t s0 = reinterpret_cast<uintptr_t>(src), d0 = reinterpret_cast<uintptr_t>(dst);
+    if (s0 < d0 + bytes && d0 < s0 + bytes) return ECHO_EINVAL;   // overlapping buffers
+    if (duty_permille > 1000 || period_us < 10 || period_us > 1000000 || duration_us < 1 ||
+        duration_us > 60000000u)
+        return ECHO_EINVAL;
+    if (moved_dev && !aligned(moved_dev, 8)) return ECHO_EINVAL;
+    if (duty_permille == 0) return ECHO_OK;   // no traffic: nothing to launch
+    if (g_fail_launches.load(std::memory_order_relaxed)) return ECHO_ECUDA;
+    int dev = 0;
+    const int sms = device_sms(&dev);
+    if (sms == 0) return ECHO_ECUDA;
+    const unsigned long long period_ns = 1000ull * period_us;
+    const unsigned long long on_ns = period_ns * duty_permille / 1000ull;
+    echo_dev::k_background_traffic<<<sms, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint4*>(src), static_cast<uint4*>(dst), (long long)(bytes / 16), on_ns, period_ns,
+        1000ull * duration_us, moved_dev);
+    return cuda_status(cudaGetLastError());
 }
 
 int echo_inject_launch_failure(int enable) {

@@ -83,7 +83,27 @@ struct Args {
     // limit of every bounded device-side wait (mbarrier waits of the
     // bulk-copy pipelines), in nanoseconds of the global timer
     unsigned long long wait_ns;
+    // chunk_k > 0: one rank of a multi-GPU call runs chunk chunk_i of
+    // chunk_k: of every owner's segment only its chunk_i-th part,
+    // [sb + floor(chunk_i len / chunk_k), sb + floor((chunk_i + 1) len / chunk_k))
+    // (len = the segment's groups), so that each chunk's exchanges are
+    // balanced over the owners
+    int chunk_i, chunk_k;
 };
+
+// Owner s's segment [sb, se) of G groups over P ranks, or, in a chunked call,
+// that segment's part for chunk chunk_i of chunk_k.
+__device__ __forceinline__ void segment_part(const Args& a, int s, long long* b, long long* e) {
+    const long long sb = (long long)s * a.G / a.P, se = (long long)(s + 1) * a.G / a.P;
+    if (a.chunk_k > 0) {
+        const long long len = se - sb;
+        *b = sb + (long long)a.chunk_i * len / a.chunk_k;
+        *e = sb + (long long)(a.chunk_i + 1) * len / a.chunk_k;
+    } else {
+        *b = sb;
+        *e = se;
+    }
+}
 
 __device__ __forceinline__ size_t a2a_slot(const Args& a, int r, long long j) {
     return (size_t)(r - a.a2a_rank_base) * (size_t)a.a2a_stride + (size_t)(j - a.a2a_col_base);

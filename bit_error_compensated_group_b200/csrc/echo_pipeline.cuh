@@ -160,37 +160,53 @@ struct RunWalker {
     // rather than held in registers.
     int kind;
     int run;            // current run index
+    int cur_rank;       // the rank of the current run
     long long base;     // first tile index of the current run
     long long run_j0, run_len;
 
-    // run `run` before clipping: kind 0, rank r = run / 2: [0, lo) for even
+    // run `run` before clipping. Kind 0, rank r = run / 2: [0, lo) for even
     // runs, [hi, G) for odd; kind 1: [lo, hi) of rank `run`, where [lo, hi)
-    // is that rank's owned segment. Clipped to the call's full-group window
-    // [c0, c1) (a partial last group takes the kernels' scalar path).
+    // is that rank's owned segment. In a chunked call (chunk_k > 0) kind 0
+    // has a run per (rank r = run / P, owner s = run % P): owner s's part of
+    // the chunk, empty for s = r; kind 1 the owned segment's part. Clipped to
+    // the call's full-group window [c0, c1) (a partial last group takes the
+    // kernels' scalar path).
     __device__ __forceinline__ void load_run(const Args& a) {
-        const int r = kind == 0 ? run >> 1 : run;
-        const long long lo = (long long)r * a.G / a.P, hi = (long long)(r + 1) * a.G / a.P;
         long long b, e;
-        if (kind == 1) {
-            b = lo;
-            e = hi;
-        } else if ((run & 1) == 0) {
-            b = 0;
-            e = lo;
+        if (a.chunk_k > 0) {
+            const int r = kind == 0 ? run / a.P : run;
+            const int s = kind == 0 ? run - r * a.P : run;
+            cur_rank = r;
+            segment_part(a, s, &b, &e);
+            if (kind == 0 && s == r) e = b;
         } else {
-            b = hi;
-            e = a.G;
+            const int r = kind == 0 ? run >> 1 : run;
+            cur_rank = r;
+            const long long lo = (long long)r * a.G / a.P, hi = (long long)(r + 1) * a.G / a.P;
+            if (kind == 1) {
+                b = lo;
+                e = hi;
+            } else if ((run & 1) == 0) {
+                b = 0;
+                e = lo;
+            } else {
+                b = hi;
+                e = a.G;
+            }
         }
         b = max(b, a.c0);
         e = min(e, a.c1);
         run_j0 = b;
         run_len = max(0LL, e - b);
     }
-    __device__ __forceinline__ int runs(const Args& a) const { return kind == 0 ? 2 * a.rank_hi : a.rank_hi; }
-    __device__ __forceinline__ int rank_of_run() const { return kind == 0 ? (run >> 1) : run; }
+    __device__ __forceinline__ int runs_per_rank(const Args& a) const {
+        return kind == 1 ? 1 : (a.chunk_k > 0 ? a.P : 2);
+    }
+    __device__ __forceinline__ int runs(const Args& a) const { return runs_per_rank(a) * a.rank_hi; }
+    __device__ __forceinline__ int rank_of_run() const { return cur_rank; }
 
-    __device__ __forceinline__ RunWalker(int kind_, const Args& a)
-        : kind(kind_), run(kind_ == 0 ? 2 * a.rank_lo : a.rank_lo), base(0) {
+    __device__ __forceinline__ RunWalker(int kind_, const Args& a) : kind(kind_), cur_rank(0), base(0) {
+        run = runs_per_rank(a) * a.rank_lo;
         if (run < runs(a)) load_run(a);
     }
 
@@ -230,12 +246,14 @@ __device__ __forceinline__ PipeShared pipe_shared(uint8_t* smem) {
     return p;
 }
 
+// `consumers`: the warps that release each stage (all consumer warps, or one
+// half of them when the halves take alternate tiles)
 template <int NS>
-__device__ __forceinline__ void pipe_init(const PipeShared& p) {
+__device__ __forceinline__ void pipe_init(const PipeShared& p, int consumers = kConsumerWarps) {
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(&p.full[s], 1);
-            mbar_init(&p.empty[s], kConsumerWarps);
+            mbar_init(&p.empty[s], consumers);
         }
         *p.abort = 0;
         mbar_fence_init();
@@ -798,12 +816,49 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
 
 // One owned group of a tile with feedback (x, e_long, e_short staged): 8
 // consecutive elements per lane, like the quantize pass.
+constexpr int kReduceRankBatch = 8;   // ranks whose payload loads are issued together
+// the simulation's owners' pass: load the next tile's first payload batch
+// while the current tile is computed
+constexpr bool kReducePrefetch = false;
+
+// The payload loads of ranks [r0, r0 + RB) for lane t's 8 elements of group
+// j: one code word (two at 8 bits) and the group's parameter word per rank;
+// zeros for the owner's own slot, ranks past P and inactive lanes.
+template <int GROUP, int BITS, bool RK, int RB>
+__device__ __forceinline__ void load_payload8(const Args& a, int o, long long j, int t, bool act, int r0,
+                                              uint32_t (&cw)[RB][BITS / 4], uint32_t (&pw)[RB]) {
+    constexpr int CB = GROUP * BITS / 8, CW = BITS / 4;
+#pragma unroll
+    for (int k = 0; k < RB; ++k) {
+        const int r = r0 + k;
+#pragma unroll
+        for (int c = 0; c < CW; ++c) cw[k][c] = 0u;
+        pw[k] = 0u;
+        if (act && r < a.P && r != o) {
+            const size_t slot = a2a_slot_t<RK>(a, r, j);
+            const uint8_t* codes = a.a2a_codes + slot * CB;
+            if (BITS == 4) {
+                cw[k][0] = *reinterpret_cast<const uint32_t*>(codes + 4 * t);
+            } else {
+                const uint2 v = *reinterpret_cast<const uint2*>(codes + 8 * t);
+                cw[k][0] = v.x;
+                cw[k][CW - 1] = v.y;
+            }
+            pw[k] = a.a2a_params[slot];
+        }
+    }
+}
+
+// `cw0` / `pw0`: the first batch's payload words, already loaded by the
+// caller (for the next tile while the previous one was computed); later
+// batches (P > RB) are loaded here.
 template <int GROUP, int BITS, int QM, bool RK>
 __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* st, const Tile& t, int gi,
-                                                  bool act) {
+                                                  bool act, const uint32_t (&cw0)[kReduceRankBatch][BITS / 4],
+                                                  const uint32_t (&pw0)[kReduceRankBatch]) {
     using LN = Lane<GROUP>;
     constexpr int L = LN::L, Q = (1 << BITS) - 1, CB = GROUP * BITS / 8;
-    constexpr int RB = 8;          // ranks whose payload loads are issued together
+    constexpr int RB = kReduceRankBatch;
     constexpr int CW = BITS / 4;   // 32-bit code words per lane (8 codes)
     const LN ln;
     const int o = t.rank;
@@ -815,39 +870,27 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
     float2 xo[4], acc[4];
 #pragma unroll
     for (int p = 0; p < 4; ++p) xo[p] = acc[p] = make_float2(0.0f, 0.0f);
-    // binary32 sum in rank order 0..P-1: own x' unquantized, others decoded.
-    // The payload loads of a batch of RB ranks are issued together; the first
-    // batch's go out before the staged x and EMAs are read, so that their
-    // latency overlaps the feedback injection.
+    if (act) {
+        load_x8c_smem(xs + e0, xo);
+        float2 el[4], es[4];
+        load_f8_smem(els, e0, e0 + 4, el);
+        load_f8_smem(ess, e0, e0 + 4, es);
+#pragma unroll
+        for (int p = 0; p < 4; ++p) xo[p] = inject2(xo[p], el[p], es[p], a);
+    }
+    // binary32 sum in rank order 0..P-1: own x' unquantized, others decoded
     for (int r0 = 0; r0 < a.P; r0 += RB) {
         uint32_t cw[RB][CW];
         uint32_t pw[RB];
+        if (r0 == 0) {
 #pragma unroll
-        for (int k = 0; k < RB; ++k) {
-            const int r = r0 + k;
+            for (int k = 0; k < RB; ++k) {
+                pw[k] = pw0[k];
 #pragma unroll
-            for (int c = 0; c < CW; ++c) cw[k][c] = 0u;
-            pw[k] = 0u;
-            if (act && r < a.P && r != o) {
-                const size_t slot = a2a_slot_t<RK>(a, r, j);
-                const uint8_t* codes = a.a2a_codes + slot * CB;
-                if (BITS == 4) {
-                    cw[k][0] = *reinterpret_cast<const uint32_t*>(codes + 4 * ln.t);
-                } else {
-                    const uint2 v = *reinterpret_cast<const uint2*>(codes + 8 * ln.t);
-                    cw[k][0] = v.x;
-                    cw[k][CW - 1] = v.y;
-                }
-                pw[k] = a.a2a_params[slot];
+                for (int c = 0; c < CW; ++c) cw[k][c] = cw0[k][c];
             }
-        }
-        if (r0 == 0 && act) {
-            load_x8c_smem(xs + e0, xo);
-            float2 el[4], es[4];
-            load_f8_smem(els, e0, e0 + 4, el);
-            load_f8_smem(ess, e0, e0 + 4, es);
-#pragma unroll
-            for (int p = 0; p < 4; ++p) xo[p] = inject2(xo[p], el[p], es[p], a);
+        } else {
+            load_payload8<GROUP, BITS, RK, RB>(a, o, j, ln.t, act, r0, cw, pw);
         }
 #pragma unroll
         for (int k = 0; k < RB; ++k) {
@@ -922,6 +965,159 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
     float* el_g = state_row_t<RK>(a, o) + j * GROUP + e0;
     store_f8_cs(el_g, nl);
     store_f8_cs(el_g + a.S, ns);
+}
+
+// One owned group of a tile with feedback, 16 elements per lane: lane t of
+// the group's L = GROUP / 16 lanes holds the 8-element chunks t and t + L
+// (each chunk's shared-memory reads by 8 lanes cover one contiguous span).
+// Against 8 elements per lane, the per-group work -- range reduction, fp16
+// parameters, each incoming payload's parameter word and slot address -- is
+// shared by twice the elements; a 2048-element tile is one pass of four warps.
+template <int GROUP, int BITS, int QM, bool RK>
+__device__ __forceinline__ void reduce_tile_group16(const Args& a, const uint8_t* st, const Tile& t, int gi,
+                                                    bool act) {
+    using LN = Lane16<GROUP>;
+    constexpr int L = LN::L, Q = (1 << BITS) - 1, CB = GROUP * BITS / 8;
+    constexpr int RB = BITS == 4 ? 8 : 4;   // ranks whose payload loads are issued together
+    constexpr int CW = BITS / 4;            // 32-bit code words per 8-element chunk
+    const LN ln;
+    const int o = t.rank;
+    const long long j = t.j0 + gi;
+    const uint16_t* xs = reinterpret_cast<const uint16_t*>(st) + gi * GROUP;
+    const float* els = reinterpret_cast<const float*>(st + kTileElems * 2) + gi * GROUP;
+    const float* ess = reinterpret_cast<const float*>(st + kTileElems * 6) + gi * GROUP;
+    float2 xo[8], acc[8];
+#pragma unroll
+    for (int p = 0; p < 8; ++p) xo[p] = acc[p] = make_float2(0.0f, 0.0f);
+    // binary32 sum in rank order 0..P-1: own x' unquantized, others decoded.
+    // The first batch's payload loads go out before the staged x and EMAs
+    // are read, so that their latency overlaps the feedback injection.
+    for (int r0 = 0; r0 < a.P; r0 += RB) {
+        uint32_t cw[RB][2 * CW];
+        uint32_t pw[RB];
+#pragma unroll
+        for (int k = 0; k < RB; ++k) {
+            const int r = r0 + k;
+            pw[k] = 0u;
+#pragma unroll
+            for (int c = 0; c < 2 * CW; ++c) cw[k][c] = 0u;
+            if (act && r < a.P && r != o) {
+                const size_t slot = a2a_slot_t<RK>(a, r, j);
+                const uint8_t* codes = a.a2a_codes + slot * CB;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    if (BITS == 4) {
+                        cw[k][h] = *reinterpret_cast<const uint32_t*>(codes + 4 * ln.chunk(h));
+                    } else {
+                        const uint2 v = *reinterpret_cast<const uint2*>(codes + 8 * ln.chunk(h));
+                        cw[k][2 * h] = v.x;
+                        cw[k][2 * h + 1] = v.y;
+                    }
+                }
+                pw[k] = a.a2a_params[slot];
+            }
+        }
+        if (r0 == 0 && act) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int e0 = 8 * ln.chunk(h);
+                float2 el[4], es[4];
+                load_x8c_smem(xs + e0, &xo[4 * h]);
+                load_f8_smem(els, e0, e0 + 4, el);
+                load_f8_smem(ess, e0, e0 + 4, es);
+#pragma unroll
+                for (int p = 0; p < 4; ++p) xo[4 * h + p] = inject2(xo[4 * h + p], el[p], es[p], a);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < RB; ++k) {
+            const int r = r0 + k;
+            if (r >= a.P) break;
+            float2 term[8];
+            if (r == o) {
+#pragma unroll
+                for (int p = 0; p < 8; ++p) term[p] = xo[p];
+            } else {
+                const float sk = param_s(pw[k]);
+                const float2 s2 = splat(sk);
+                const float2 z2 = splat(param_zf<QM>(pw[k], sk));
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    float2 q[4];
+                    unpack_codes8<BITS>(&cw[k][h * CW], q);
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) term[4 * h + p] = fma2_rn(q[p], s2, z2);
+                }
+            }
+#pragma unroll
+            for (int p = 0; p < 8; ++p) acc[p] = (r == 0) ? term[p] : add2_rn(acc[p], term[p]);
+        }
+    }
+    float lmin = __int_as_float(0x7f800000), lmax = -__int_as_float(0x7f800000);
+    if (act) {
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+            lmin = nan_min3(lmin, acc[p].x, acc[p].y);
+            lmax = nan_max3(lmax, acc[p].x, acc[p].y);
+        }
+    }
+    uint32_t yb[8];   // bf16 pairs of the result
+    if (a.P >= 2) {
+        const GridP g = make_grid_p<L, Q, QM>(lmin, lmax);
+        raise_flags(a, act && g.bad);
+        if (!act) return;
+        uint8_t* codes = a.g_codes + (size_t)(j - a.g_col_base) * CB;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float2 e[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                e[p] = encode2<QM, Q>(acc[4 * h + p], g, a);
+                yb[4 * h + p] = bf16x2_rn(fma2_rn(add2_rn(e[p], splat(-kMagic)), g.s, g.z));
+            }
+            const uint2 pk = pack_codes8<BITS>(e);
+            if (BITS == 4) *reinterpret_cast<uint32_t*>(codes + 4 * ln.chunk(h)) = pk.x;
+            else *reinterpret_cast<uint2*>(codes + 8 * ln.chunk(h)) = pk;
+        }
+        if (ln.t == 0) a.g_params[j - a.g_col_base] = g.param;
+        if (a.write_outputs) {
+            // phase 4 in the owner's pass: every rank's output gets the decoded
+            // requantized sum -- the same bits a decode of the gathered payload gives
+            for (int r = 0; r < a.P; ++r) {
+                uint16_t* y = a.out[r] + j * GROUP;
+                __stcs(reinterpret_cast<uint4*>(y + 8 * ln.chunk(0)), make_uint4(yb[0], yb[1], yb[2], yb[3]));
+                __stcs(reinterpret_cast<uint4*>(y + 8 * ln.chunk(1)), make_uint4(yb[4], yb[5], yb[6], yb[7]));
+            }
+        }
+    } else {
+        // a single rank sends nothing: its output is its own x'
+        raise_flags(a, act && !(lmin >= -65504.0f && lmax <= 65504.0f));
+        if (!act) return;
+#pragma unroll
+        for (int p = 0; p < 8; ++p) yb[p] = bf16x2_rn(acc[p]);
+        uint16_t* y = a.out[0] + j * GROUP;
+        *reinterpret_cast<uint4*>(y + 8 * ln.chunk(0)) = make_uint4(yb[0], yb[1], yb[2], yb[3]);
+        *reinterpret_cast<uint4*>(y + 8 * ln.chunk(1)) = make_uint4(yb[4], yb[5], yb[6], yb[7]);
+    }
+    float* el_g = state_row_t<RK>(a, o) + j * GROUP;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int e0 = 8 * ln.chunk(h);
+        float2 el[4], es[4], nl[4], ns[4];
+        load_f8_smem(els, e0, e0 + 4, el);
+        load_f8_smem(ess, e0, e0 + 4, es);
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            // rho = acc - float(y): flip the sign bits of the bf16 pair, then widen exactly
+            const uint32_t ny = yb[4 * h + p] ^ 0x80008000u;
+            const float2 rho = add2_rn(acc[4 * h + p],
+                                       make_float2(__uint_as_float(ny << 16), __uint_as_float(ny & 0xffff0000u)));
+            nl[p] = ema2(el[p], rho, a.keep_long, a.a_long, a);
+            ns[p] = ema2(es[p], rho, a.keep_short, a.a_short, a);
+        }
+        store_f8_cs(el_g + e0, nl);
+        store_f8_cs(el_g + a.S + e0, ns);
+    }
 }
 
 // The owner's pass without feedback, 16 elements per lane (chunks t and
@@ -1048,13 +1244,21 @@ __device__ __forceinline__ void reduce_tile_group_nf(const Args& a, const uint8_
     }
 }
 
+// Two CTAs of kPipeThreads per SM: 96 registers per thread (each SM
+// sub-partition's 16384 registers then hold its share of the 18 warps).
 template <int GROUP, int BITS, bool FB, int QM, bool RK = false>
 __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
     constexpr int M = FB ? 1 : kReduceSubtilesNF;
     constexpr int NS = FB ? kStagesReduceFB : kStagesReduceNF;
+    // One rank of a multi-GPU call with feedback: 16 elements per lane, the
+    // two halves of the consumer warps taking alternate tiles (each stage is
+    // released by one half). The simulation with feedback: 8 elements per
+    // lane, all consumer warps on every tile. Without feedback: 16 elements
+    // per lane, two passes of all warps over a 4-sub-tile stage.
+    constexpr bool HALVES = FB && RK;
     const PipeShared p = pipe_shared<NS>(smem);
-    pipe_init<NS>(p);
+    pipe_init<NS>(p, HALVES ? kConsumerWarps / 2 : kConsumerWarps);
     const int warp = threadIdx.x >> 5;
     RunWalker<GROUP, M> walker(1, a);
     if (warp == kConsumerWarps) {
@@ -1066,31 +1270,92 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
     // the payload, the flag word and the outputs: only once the quantize pass
     // is complete (an output may be the same buffer as an input it reads)
     griddep_wait();
-    // with feedback: 8 elements per lane, one pass per tile; without: 16 per
-    // lane, two passes over the 4-sub-tile stage
-    constexpr int GPW = FB ? Lane<GROUP>::GPW : Lane16<GROUP>::GPW;
-    constexpr int PASSES = FB ? 1 : M * kTileElems / (kConsumerWarps * 32 * 16);
-    const int gi = warp * GPW + (FB ? Lane<GROUP>().sub : Lane16<GROUP>().sub);
-    long long i = 0;
+    const bool lead = (threadIdx.x & 31) == 0;
     Tile t;
-    for (long long k = blockIdx.x; walker.locate(k, &t, a); k += gridDim.x, ++i) {
-        const int s = (int)(i % NS);
-        if (!mbar_wait(&p.full[s], (uint32_t)(i / NS) & 1u, a.wait_ns, p.abort)) {
-            if ((threadIdx.x & 31) == 0) report_timeout(a, p);
-            return;
-        }
-        const uint8_t* stage = p.stages + (size_t)s * kStageBytes;
-        if (FB) {
-            reduce_tile_group<GROUP, BITS, QM, RK>(a, stage, t, gi, gi < t.count);
-        } else {
-#pragma unroll 1
-            for (int m = 0; m < PASSES; ++m) {
-                const int g = gi + m * kConsumerWarps * GPW;
-                reduce_tile_group_nf<GROUP, BITS, QM, RK>(a, stage, t, g, g < t.count);
+    if (FB && !RK && kReducePrefetch) {
+        // The simulation: the first batch of a tile's payload loads is issued
+        // while the previous tile is computed (registers carry it), so their
+        // latency hides behind that work instead of stalling the tile.
+        constexpr int CW = BITS / 4;
+        const int gi = warp * Lane<GROUP>::GPW + Lane<GROUP>().sub;
+        const int lt = Lane<GROUP>().t;
+        long long k = blockIdx.x, i = 0;
+        bool have = walker.locate(k, &t, a);
+        uint32_t cw[kReduceRankBatch][CW], pw[kReduceRankBatch];
+        if (have) load_payload8<GROUP, BITS, RK, kReduceRankBatch>(a, t.rank, t.j0 + gi, lt, gi < t.count, 0, cw, pw);
+        while (have) {
+            const int s = (int)(i % NS);
+            if (!mbar_wait(&p.full[s], (uint32_t)(i / NS) & 1u, a.wait_ns, p.abort)) {
+                if (lead) report_timeout(a, p);
+                return;
             }
+            Tile tn;
+            const bool have_next = walker.locate(k + gridDim.x, &tn, a);
+            uint32_t cwn[kReduceRankBatch][CW], pwn[kReduceRankBatch];
+            load_payload8<GROUP, BITS, RK, kReduceRankBatch>(a, tn.rank, tn.j0 + gi, lt, have_next && gi < tn.count,
+                                                            0, cwn, pwn);
+            reduce_tile_group<GROUP, BITS, QM, RK>(a, p.stages + (size_t)s * kStageBytes, t, gi, gi < t.count, cw,
+                                                   pw);
+            __syncwarp();
+            if (lead) mbar_arrive(&p.empty[s]);
+#pragma unroll
+            for (int q = 0; q < kReduceRankBatch; ++q) {
+                pw[q] = pwn[q];
+#pragma unroll
+                for (int c = 0; c < CW; ++c) cw[q][c] = cwn[q][c];
+            }
+            t = tn;
+            have = have_next;
+            k += gridDim.x;
+            ++i;
         }
-        __syncwarp();
-        if ((threadIdx.x & 31) == 0) mbar_arrive(&p.empty[s]);
+    } else if (FB && !RK) {
+        // The simulation, payload loads issued at the start of each tile
+        constexpr int CW = BITS / 4;
+        const int gi = warp * Lane<GROUP>::GPW + Lane<GROUP>().sub;
+        const int lt = Lane<GROUP>().t;
+        long long i = 0;
+        for (long long k = blockIdx.x; walker.locate(k, &t, a); k += gridDim.x, ++i) {
+            const int s = (int)(i % NS);
+            uint32_t cw[kReduceRankBatch][CW], pw[kReduceRankBatch];
+            load_payload8<GROUP, BITS, RK, kReduceRankBatch>(a, t.rank, t.j0 + gi, lt, gi < t.count, 0, cw, pw);
+            if (!mbar_wait(&p.full[s], (uint32_t)(i / NS) & 1u, a.wait_ns, p.abort)) {
+                if (lead) report_timeout(a, p);
+                return;
+            }
+            reduce_tile_group<GROUP, BITS, QM, RK>(a, p.stages + (size_t)s * kStageBytes, t, gi, gi < t.count, cw,
+                                                   pw);
+            __syncwarp();
+            if (lead) mbar_arrive(&p.empty[s]);
+        }
+    } else {
+        constexpr int GPW = Lane16<GROUP>::GPW;
+        constexpr int HALF = kConsumerWarps / 2;
+        constexpr int PASSES = FB ? 1 : M * kTileElems / (kConsumerWarps * 32 * 16);
+        constexpr int STEP = HALVES ? 2 : 1;
+        static_assert(!HALVES || HALF * GPW * GROUP == kTileElems, "a tile is one pass of half the consumer warps");
+        const int half = HALVES ? warp / HALF : 0;
+        const int gi = (HALVES ? warp % HALF : warp) * GPW + Lane16<GROUP>().sub;
+        long long i = half;
+        for (long long k = blockIdx.x + half * gridDim.x; walker.locate(k, &t, a); k += STEP * gridDim.x, i += STEP) {
+            const int s = (int)(i % NS);
+            if (!mbar_wait(&p.full[s], (uint32_t)(i / NS) & 1u, a.wait_ns, p.abort)) {
+                if (lead) report_timeout(a, p);
+                return;
+            }
+            const uint8_t* stage = p.stages + (size_t)s * kStageBytes;
+            if (FB) {
+                reduce_tile_group16<GROUP, BITS, QM, RK>(a, stage, t, gi, gi < t.count);
+            } else {
+#pragma unroll 1
+                for (int m = 0; m < PASSES; ++m) {
+                    const int g = gi + m * kConsumerWarps * GPW;
+                    reduce_tile_group_nf<GROUP, BITS, QM, RK>(a, stage, t, g, g < t.count);
+                }
+            }
+            __syncwarp();
+            if (lead) mbar_arrive(&p.empty[s]);
+        }
     }
     if (a.tail && blockIdx.x == gridDim.x - 1 && warp == 0) {
         const long long j = a.G - 1;
@@ -1178,15 +1443,20 @@ __global__ void __launch_bounds__(kGatherThreads) k_gather_tma(const Args a) {
 
 // Phase 4 on one rank of a multi-GPU call: every group of the gathered
 // payload (P owner segments, each padded to g_seg_stride groups) decoded into
-// this rank's output. With a single output there is no tile to share between
+// this rank's output (a.out[a.out_lo]). With a single output there is no tile to share between
 // stores, so each thread decodes E-element chunks straight from registers:
-// the loads of U chunks (code words and parameter word each) are issued
-// together, then each chunk leaves in one streaming store (32 bytes at
-// E = 16 when the output is 32-byte aligned, else 16-byte stores). Chunk c
-// covers elements [E c, E c + E) of group c / (GROUP / E). A CTA walks tiles
-// of U * blockDim consecutive chunks, so a thread's chunks only move
-// forward: the owner of a group is found by advancing an index over the
-// segment starts kept in shared memory (no division per chunk).
+// the loads of U chunks (one code load and the parameter word each) are
+// issued together, then each chunk leaves in one 32-byte streaming store
+// (16-byte stores when the output is not 32-byte aligned).
+//
+// Work layout: owner o's run is its segment (in a chunked call, the chunk's
+// part of it) clipped to the call's full-group window; a run is cut into
+// tiles of TG consecutive groups, and the tiles of all runs are numbered in
+// owner order. A CTA walks tiles k = blockIdx.x,
+// + gridDim.x, ...: per tile the owner, the first group and the first slot in
+// the gathered rows are uniform, so per chunk only 32-bit offsets inside the
+// tile are computed. The runs' bounds and tile prefix sums are set up once
+// per CTA in shared memory (one thread per owner, then a warp scan).
 constexpr int kDecodeThreads = 256;
 constexpr int kDecodeUnroll = 8;
 constexpr int kDecodeElems = 16;
@@ -1197,50 +1467,90 @@ __device__ __forceinline__ void store_v8_cs(void* p, uint4 lo, uint4 hi) {
                  : "memory");
 }
 
+// 16 consecutive codes of a group: 8 bytes at 4 bits (x, y), 16 at 8 bits
+template <int BITS>
+__device__ __forceinline__ uint4 load_codes16(const uint8_t* p) {
+    if (BITS == 4) {
+        const uint2 v = *reinterpret_cast<const uint2*>(p);
+        return make_uint4(v.x, v.y, 0u, 0u);
+    }
+    return *reinterpret_cast<const uint4*>(p);
+}
+
 template <int GROUP, int BITS, int QM>
 __global__ void __launch_bounds__(kDecodeThreads) k_decode_rank(const Args a) {
-    constexpr int E = kDecodeElems, H = E / 8, L = GROUP / E, CB = GROUP * BITS / 8, U = kDecodeUnroll;
-    static_assert(E == 8 || E == 16, "chunk of 8 or 16 elements");
-    __shared__ long long seg_start[ECHO_MAX_RANKS + 1];
-    for (int s = threadIdx.x; s <= a.P; s += blockDim.x) seg_start[s] = (long long)s * a.G / a.P;
+    constexpr int E = kDecodeElems, L = GROUP / E, CB = GROUP * BITS / 8, U = kDecodeUnroll;
+    constexpr int CHUNK_BYTES = E * BITS / 8;
+    constexpr int TG = U * kDecodeThreads / L;   // groups per tile
+    static_assert(E == 16 && GROUP % E == 0, "16-element chunks");
+    static_assert(ECHO_MAX_RANKS <= 64, "one warp scans the owners' tile counts");
+    __shared__ long long run_b[ECHO_MAX_RANKS], run_e[ECHO_MAX_RANKS], run_slot[ECHO_MAX_RANKS];
+    __shared__ long long tile_pre[ECHO_MAX_RANKS + 1];
+    const int tid = threadIdx.x;
+    if (tid < a.P) {
+        const long long sb = (long long)tid * a.G / a.P;
+        long long pb, pe;
+        segment_part(a, tid, &pb, &pe);   // the segment, or its part for this chunk
+        const long long b = max(pb, a.c0), e = max(b, min(pe, a.c1));
+        run_b[tid] = b;
+        run_e[tid] = e;
+        run_slot[tid] = (long long)tid * a.g_seg_stride + (b - sb);
+        tile_pre[tid + 1] = (e - b + TG - 1) / TG;   // this owner's tile count, summed below
+    }
     __syncthreads();
-    const long long c_begin = a.c0 * L, c_end = a.c1 * L;   // the window's full groups
-    const long long tile_chunks = (long long)U * blockDim.x;
+    if (tid < 32) {   // inclusive scan of the tile counts: lane l holds owners 2l and 2l + 1
+        const int o0 = 2 * tid, o1 = 2 * tid + 1;
+        const long long c0 = o0 < a.P ? tile_pre[o0 + 1] : 0, c1 = o1 < a.P ? tile_pre[o1 + 1] : 0;
+        long long incl = c0 + c1;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const long long v = __shfl_up_sync(kFull, incl, d);
+            if (tid >= d) incl += v;
+        }
+        if (o0 < a.P) tile_pre[o0 + 1] = incl - c1;
+        if (o1 < a.P) tile_pre[o1 + 1] = incl;
+        if (tid == 0) tile_pre[0] = 0;
+    }
+    __syncthreads();
+    const long long ntiles = tile_pre[a.P];
+    // one output (this rank's); 32-byte stores when it is 32-byte aligned
+    uint16_t* const out = a.out[a.out_lo];
+    const bool v8 = (reinterpret_cast<uintptr_t>(out) & 31) == 0;
     int o = 0;
-    for (long long base = c_begin + blockIdx.x * tile_chunks; base < c_end; base += gridDim.x * tile_chunks) {
-        uint2 w[U][H];
+    for (long long k = blockIdx.x; k < ntiles; k += gridDim.x) {
+        while (k >= tile_pre[o + 1]) ++o;
+        const long long off = (k - tile_pre[o]) * TG;
+        const long long j0 = run_b[o] + off;
+        // chunk lc of the tile: group lc / L, its part lc % L, so its codes
+        // start lc * CHUNK_BYTES after the tile's first group's, its output
+        // lc * E elements after the tile's first element
+        const int nchunks = (int)min((long long)TG, run_e[o] - j0) * L;
+        const uint8_t* codes = a.g_codes + (size_t)(run_slot[o] + off) * CB;
+        const uint32_t* params = a.g_params + (run_slot[o] + off);
+        uint16_t* const y = out + j0 * GROUP;
+        uint4 w[U];
         uint32_t pw[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const long long c = base + u * blockDim.x + threadIdx.x;
-#pragma unroll
-            for (int h = 0; h < H; ++h) w[u][h] = make_uint2(0u, 0u);
-            pw[u] = 0u;
-            if (c < c_end) {
-                const long long j = c / L;
-                while (j >= seg_start[o + 1]) ++o;
-                const size_t gs = (size_t)((long long)o * a.g_seg_stride + j - seg_start[o]);
-                const uint8_t* codes = a.g_codes + gs * CB;
-#pragma unroll
-                for (int h = 0; h < H; ++h) w[u][h] = load_codes8<BITS>(codes, (int)(c % L) * H + h);
-                pw[u] = a.g_params[gs];
+            const int lc = u * kDecodeThreads + tid;
+            if (lc < nchunks) {
+                w[u] = load_codes16<BITS>(codes + lc * CHUNK_BYTES);
+                pw[u] = params[lc / L];
             }
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const long long c = base + u * blockDim.x + threadIdx.x;
-            if (c < c_end) {
-                uint4 y[H];
-#pragma unroll
-                for (int h = 0; h < H; ++h) y[h] = decode8_bf16<BITS, QM>(w[u][h], pw[u]);
-                for (int r = a.out_lo; r < a.out_hi; ++r) {
-                    uint16_t* dst = a.out[r] + (long long)E * c;
-                    if (E == 16 && (reinterpret_cast<uintptr_t>(a.out[r]) & 31) == 0) {
-                        store_v8_cs(dst, y[0], y[H - 1]);
-                    } else {
-#pragma unroll
-                        for (int h = 0; h < H; ++h) __stcs(reinterpret_cast<uint4*>(dst + 8 * h), y[h]);
-                    }
+            const int lc = u * kDecodeThreads + tid;
+            if (lc < nchunks) {
+                const uint4 y0 = decode8_bf16<BITS, QM>(make_uint2(w[u].x, BITS == 4 ? 0u : w[u].y), pw[u]);
+                const uint4 y1 = decode8_bf16<BITS, QM>(BITS == 4 ? make_uint2(w[u].y, 0u) : make_uint2(w[u].z, w[u].w),
+                                                        pw[u]);
+                uint16_t* dst = y + lc * E;
+                if (v8) {
+                    store_v8_cs(dst, y0, y1);
+                } else {
+                    __stcs(reinterpret_cast<uint4*>(dst), y0);
+                    __stcs(reinterpret_cast<uint4*>(dst + 8), y1);
                 }
             }
         }
@@ -1253,11 +1563,9 @@ __global__ void __launch_bounds__(kDecodeThreads) k_decode_rank(const Args a) {
         const uint4 v = decode8_bf16<BITS, QM>(w, a.g_params[gs]);
         const uint32_t yb[4] = {v.x, v.y, v.z, v.w};
         const long long e = j * GROUP + 8 * threadIdx.x;
-        for (int r = a.out_lo; r < a.out_hi; ++r) {
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-                if (e + k < a.n) a.out[r][e + k] = (uint16_t)(yb[k >> 1] >> (16 * (k & 1)));
-        }
+        for (int k = 0; k < 8; ++k)
+            if (e + k < a.n) out[e + k] = (uint16_t)(yb[k >> 1] >> (16 * (k & 1)));
     }
 }
 

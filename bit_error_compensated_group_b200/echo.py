@@ -20,6 +20,7 @@ ECHO_NOALLOC_SCRATCH_BYTES = 16 << 20
 ECHO_FLAG_RANGE = 1
 ECHO_FLAG_TIMEOUT = 2
 ECHO_MAX_RANKS = 64
+ECHO_MAX_CHUNKS = 4096
 ECHO_QUANT_DIRECTED, ECHO_QUANT_NEAREST, ECHO_QUANT_INT_ZERO = 0, 1, 2
 
 LIB_PATH = _build.LIB
@@ -115,6 +116,19 @@ def lib() -> ctypes.CDLL:
         L.echo_rank_reduce.restype = I
         L.echo_rank_decode.argtypes = [V, V, I, V]
         L.echo_rank_decode.restype = I
+        L.echo_rank_quantize_chunk.argtypes = [V, V, I, F, F, F, F, I, I, V]
+        L.echo_rank_quantize_chunk.restype = I
+        L.echo_rank_reduce_chunk.argtypes = [V, V, V, I, F, F, F, F, I, I, V]
+        L.echo_rank_reduce_chunk.restype = I
+        L.echo_rank_decode_chunk.argtypes = [V, V, I, I, I, V]
+        L.echo_rank_decode_chunk.restype = I
+        L.echo_query_chunk.argtypes = [I64, I, I, I, I, I, ctypes.POINTER(I64), ctypes.POINTER(I64)]
+        L.echo_query_chunk.restype = I
+        L.echo_bf16_allreduce_sim.argtypes = [PP, PP, I64, I, V]
+        L.echo_bf16_allreduce_sim.restype = I
+        L.echo_background_traffic.argtypes = [V, V, ctypes.c_size_t, ctypes.c_uint32, ctypes.c_uint32,
+                                              ctypes.c_uint32, V, V]
+        L.echo_background_traffic.restype = I
         L.echo_inject_launch_failure.argtypes = [I]
         L.echo_inject_launch_failure.restype = I
         L.echo_set_wait_limit.argtypes = [V, ctypes.c_uint32]
@@ -286,6 +300,25 @@ def echo_allreduce_sim_noalloc(inputs: Sequence, outputs: Sequence, state, n: in
     return int(flags.value) if read_flags else None
 
 
+def echo_bf16_allreduce_sim(inputs: Sequence, outputs: Sequence, n: int, P: int, stream=None) -> None:
+    """The 16-bit baseline all-reduce over P virtual ranks (rank-ordered
+    binary32 sum, bf16 result into every output)."""
+    _check(lib().echo_bf16_allreduce_sim(_ptr_array(inputs), _ptr_array(outputs), n, P, _stream(stream)),
+           "echo_bf16_allreduce_sim")
+
+
+def echo_background_traffic(src, dst, duty_permille: int, period_us: int, duration_us: int, moved=None,
+                            stream=None) -> None:
+    """Competing HBM traffic: copy src -> dst (same size, bytes a multiple of
+    16) for the duty cycle of every period, for duration_us of wall-clock
+    time. `moved`: an int64 CUDA tensor that accumulates the bytes moved."""
+    if src.numel() * src.element_size() != dst.numel() * dst.element_size():
+        raise ValueError("echo_background_traffic: src and dst differ in size")
+    _check(lib().echo_background_traffic(_ptr(src), _ptr(dst), src.numel() * src.element_size(), duty_permille,
+                                         period_us, duration_us, _ptr(moved), _stream(stream)),
+           "echo_background_traffic")
+
+
 def echo_set_wait_limit(st, limit_us: int) -> None:
     """Limit of the kernels' bounded device waits for the handle's later
     calls (1 ms .. 60 s; default 1 s)."""
@@ -399,6 +432,32 @@ def echo_rank_decode(out, st, bits: int, stream=None) -> None:
     _check(lib().echo_rank_decode(_ptr(out), st, bits, _stream(stream)), "echo_rank_decode")
 
 
+def echo_rank_quantize_chunk(x, st, bits: int, eta: float, alpha_long: float, alpha_short: float, w: float,
+                             chunk: int, chunks: int, stream=None) -> None:
+    _check(lib().echo_rank_quantize_chunk(_ptr(x), st, bits, eta, alpha_long, alpha_short, w, chunk, chunks,
+                                          _stream(stream)), "echo_rank_quantize_chunk")
+
+
+def echo_rank_reduce_chunk(x, out, st, bits: int, eta: float, alpha_long: float, alpha_short: float, w: float,
+                           chunk: int, chunks: int, stream=None) -> None:
+    _check(lib().echo_rank_reduce_chunk(_ptr(x), _ptr(out), st, bits, eta, alpha_long, alpha_short, w, chunk,
+                                        chunks, _stream(stream)), "echo_rank_reduce_chunk")
+
+
+def echo_rank_decode_chunk(out, st, bits: int, chunk: int, chunks: int, stream=None) -> None:
+    _check(lib().echo_rank_decode_chunk(_ptr(out), st, bits, chunk, chunks, _stream(stream)),
+           "echo_rank_decode_chunk")
+
+
+def echo_query_chunk(n: int, P: int, group: int, owner: int, chunk: int, chunks: int):
+    """(first, count): owner's part of chunk `chunk` of `chunks`, in groups,
+    relative to the owner's first group."""
+    first, count = ctypes.c_int64(), ctypes.c_int64()
+    _check(lib().echo_query_chunk(n, P, group, owner, chunk, chunks, ctypes.byref(first), ctypes.byref(count)),
+           "echo_query_chunk")
+    return int(first.value), int(count.value)
+
+
 class ExchangePlan:
     """Views of one rank's workspace for the two exchanges of a multi-GPU
     call and their split sizes, in the argument order of
@@ -430,6 +489,37 @@ class ExchangePlan:
         self.gsend_params = i32(L.gsend_params_offset, sm)
         self.grecv_codes = u8(L.grecv_codes_offset, P * sm * cb)
         self.grecv_params = i32(L.grecv_params_offset, P * sm)
+        self._args = (n, P, rank, group, cb, sm)
+        self._segs = segs
+        self._seg_begin = [int(echo_query_rank_layout(n, P, s, group, max_bits, bits).seg_begin) for s in range(P)]
+        self._chunks = {}
+
+    def chunk_pieces(self, chunk: int, chunks: int):
+        """Views of this rank's buffers for chunk `chunk` of `chunks` (the
+        layout echo_rank_quantize_chunk & co. document): per peer, what to
+        send and where to receive, as (codes, params) view pairs.
+
+        a2a_send[s] / a2a_recv[r]: this rank's send slots for owner s's part;
+        the slots of this owner's recv row r where rank r's part lands.
+        ag_send: this owner's part of its gsend buffer; ag_recv[o]: the slots
+        of gathered row o where owner o's part lands."""
+        key = (chunk, chunks)
+        if key not in self._chunks:
+            n, P, rank, group, cb, sm = self._args
+            parts = [echo_query_chunk(n, P, group, s, chunk, chunks) for s in range(P)]
+            seg = self._segs[rank]
+            f_me, c_me = parts[rank]
+
+            def cp(codes, params, slot, count):
+                return codes[slot * cb:(slot + count) * cb], params[slot:slot + count]
+
+            a2a_send = [cp(self.send_codes, self.send_params, self._seg_begin[s] + parts[s][0], parts[s][1])
+                        for s in range(P)]
+            a2a_recv = [cp(self.recv_codes, self.recv_params, r * seg + f_me, c_me) for r in range(P)]
+            ag_send = cp(self.gsend_codes, self.gsend_params, f_me, c_me)
+            ag_recv = [cp(self.grecv_codes, self.grecv_params, o * sm + parts[o][0], parts[o][1]) for o in range(P)]
+            self._chunks[key] = (a2a_send, a2a_recv, ag_send, ag_recv)
+        return self._chunks[key]
 
 
 def exchange_all_to_all(plan: ExchangePlan, group=None) -> None:
@@ -446,6 +536,41 @@ def exchange_all_gather(plan: ExchangePlan, group=None) -> None:
     import torch.distributed as dist
     dist.all_gather_into_tensor(plan.grecv_codes, plan.gsend_codes, group=group)
     dist.all_gather_into_tensor(plan.grecv_params, plan.gsend_params, group=group)
+
+
+def exchange_chunk(plan: ExchangePlan, step: str, chunk: int, chunks: int, rank: int, group=None):
+    """One chunk's exchange as point-to-point sends and receives (the pieces
+    of a chunk are not contiguous across peers, and their sizes differ by a
+    group or so): `step` "all_to_all" sends this rank's part for every other
+    owner and receives every other rank's part of its own segment;
+    "all_gather" sends its own part to every other rank, receives every other
+    owner's part, and copies its own part into its gathered row. Enqueued on
+    the current stream; returns the requests (their wait() orders that
+    stream after the transfers)."""
+    import torch.distributed as dist
+    a2a_send, a2a_recv, ag_send, ag_recv = plan.chunk_pieces(chunk, chunks)
+    P = len(a2a_send)
+    ops = []
+    for peer in range(P):
+        if peer == rank:
+            continue
+        if step == "all_to_all":
+            pieces = ((a2a_send[peer], a2a_recv[peer]),)
+        elif step == "all_gather":
+            pieces = ((ag_send, ag_recv[peer]),)
+        else:
+            raise ValueError(step)
+        for send, recv in pieces:
+            for k in range(2):   # codes, then parameter words
+                if send[k].numel():
+                    ops.append(dist.P2POp(dist.isend, send[k], peer, group))
+                if recv[k].numel():
+                    ops.append(dist.P2POp(dist.irecv, recv[k], peer, group))
+    if step == "all_gather":
+        for k in range(2):
+            if ag_send[k].numel():
+                ag_recv[rank][k].copy_(ag_send[k])
+    return dist.batch_isend_irecv(ops) if ops else []
 
 
 class EchoRank:
@@ -481,17 +606,43 @@ class EchoRank:
     def decode(self, out, bits=4, stream=None) -> None:
         echo_rank_decode(out, self.handle, bits, stream)
 
-    def allreduce(self, x, out, bits=4, eta=1.0, alpha_long=0.05, alpha_short=0.5, w=0.5, group=None) -> None:
-        """Steps 1-5 on torch's current stream, with the process group's
-        collectives in between (every rank of the group calls this)."""
+    def quantize_chunk(self, x, chunk, chunks, bits=4, eta=1.0, alpha_long=0.05, alpha_short=0.5, w=0.5,
+                       stream=None) -> None:
+        echo_rank_quantize_chunk(x, self.handle, bits, eta, alpha_long, alpha_short, w, chunk, chunks, stream)
+
+    def reduce_chunk(self, x, out, chunk, chunks, bits=4, eta=1.0, alpha_long=0.05, alpha_short=0.5, w=0.5,
+                     stream=None) -> None:
+        echo_rank_reduce_chunk(x, out, self.handle, bits, eta, alpha_long, alpha_short, w, chunk, chunks, stream)
+
+    def decode_chunk(self, out, chunk, chunks, bits=4, stream=None) -> None:
+        echo_rank_decode_chunk(out, self.handle, bits, chunk, chunks, stream)
+
+    def allreduce(self, x, out, bits=4, eta=1.0, alpha_long=0.05, alpha_short=0.5, w=0.5, group=None,
+                  chunks: int = 1, comm_stream=None) -> None:
+        """Steps 1-5 with the process group's exchanges in between (every rank
+        of the group calls this). chunks = 1: on torch's current stream, the
+        collectives between the kernels. chunks > 1: the call in column
+        chunks (see echo_rank_quantize_chunk), chunk c's exchanges on
+        `comm_stream` (a new stream if None) overlapping chunk c + 1's
+        kernels on the current stream, ordered by CUDA events; the current
+        stream continues once the last chunk is decoded."""
         fb = (eta, alpha_long, alpha_short, w)
-        self.quantize(x, bits, *fb)
-        if self.P > 1:
-            exchange_all_to_all(self.plan(bits), group)
-        self.reduce(x, out, bits, *fb)
-        if self.P > 1:
-            exchange_all_gather(self.plan(bits), group)
-            self.decode(out, bits)
+        if chunks <= 1 or self.P == 1:
+            self.quantize(x, bits, *fb)
+            if self.P > 1:
+                exchange_all_to_all(self.plan(bits), group)
+            self.reduce(x, out, bits, *fb)
+            if self.P > 1:
+                exchange_all_gather(self.plan(bits), group)
+                self.decode(out, bits)
+            return
+        plan = self.plan(bits)
+
+        def comm(step, c):
+            for req in exchange_chunk(plan, step, c, chunks, self.rank, group):
+                req.wait()
+
+        run_chunked([self], [x], [out], bits, fb, chunks, comm, comm_stream)
 
     def ema_views(self):
         """(e_long [n], e_short [n]) of this rank."""
@@ -512,6 +663,50 @@ class EchoRank:
             self.close()
         except Exception:
             pass
+
+
+def run_chunked(ranks: Sequence["EchoRank"], xs: Sequence, outs: Sequence, bits: int, fb, chunks: int, comm,
+                comm_stream=None) -> None:
+    """The chunked schedule of a multi-GPU call for the ranks this process
+    drives (one per process on P GPUs; all P of them on one GPU in tests and
+    one-GPU benchmarks). Compute stream = torch's current stream; chunk c's
+    all-to-all runs on the communication stream once its quantize is done,
+    its reduce once that all-to-all is done, its all-gather once the reduce
+    is done, its decode once the all-gather is done; the compute stream
+    issues quantize(c), reduce(c - 1), decode(c - 2) in turn, so one chunk's
+    transfers overlap the neighbouring chunks' kernels. `comm(step, c)`
+    enqueues chunk c's exchange on the current stream (called with the
+    communication stream current)."""
+    compute = torch.cuda.current_stream()
+    cs = comm_stream if comm_stream is not None else torch.cuda.Stream(device=compute.device)
+    ev = {name: [torch.cuda.Event() for _ in range(chunks)] for name in ("q", "a", "r", "g")}
+    cs.wait_stream(compute)   # the inputs and the previous call's work
+    for t in range(chunks + 2):
+        c = t
+        if c < chunks:
+            for rk, x in zip(ranks, xs):
+                rk.quantize_chunk(x, c, chunks, bits, *fb, stream=compute)
+            ev["q"][c].record(compute)
+            with torch.cuda.stream(cs):
+                cs.wait_event(ev["q"][c])
+                comm("all_to_all", c)
+                ev["a"][c].record(cs)
+        c = t - 1
+        if 0 <= c < chunks:
+            compute.wait_event(ev["a"][c])
+            for rk, x in zip(ranks, xs):
+                rk.reduce_chunk(x, None, c, chunks, bits, *fb, stream=compute)
+            ev["r"][c].record(compute)
+            with torch.cuda.stream(cs):
+                cs.wait_event(ev["r"][c])
+                comm("all_gather", c)
+                ev["g"][c].record(cs)
+        c = t - 2
+        if 0 <= c < chunks:
+            compute.wait_event(ev["g"][c])
+            for rk, y in zip(ranks, outs):
+                rk.decode_chunk(y, c, chunks, bits, stream=compute)
+    compute.wait_stream(cs)
 
 
 def exchange_in_process(plans: Sequence[ExchangePlan], step: str) -> None:
@@ -540,3 +735,25 @@ def exchange_in_process(plans: Sequence[ExchangePlan], step: str) -> None:
                     recv[s * k:(s + 1) * k].copy_(send)
     else:
         raise ValueError(step)
+
+
+def exchange_chunk_in_process(plans: Sequence[ExchangePlan], step: str, chunk: int, chunks: int) -> None:
+    """exchange_chunk for P ranks held by one process on one device:
+    stream-ordered copies of the same pieces (tests and one-GPU benchmarks)."""
+    pieces = [pl.chunk_pieces(chunk, chunks) for pl in plans]
+    P = len(plans)
+    for dst in range(P):
+        for src in range(P):
+            if step == "all_to_all":
+                if src == dst:
+                    continue
+                send, recv = pieces[src][0][dst], pieces[dst][1][src]
+            elif step == "all_gather":
+                send, recv = pieces[src][2], pieces[dst][3][src]
+            else:
+                raise ValueError(step)
+            for k in range(2):
+                if send[k].numel() != recv[k].numel():
+                    raise ValueError("chunk pieces of different messages")
+                if send[k].numel():
+                    recv[k].copy_(send[k])

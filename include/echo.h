@@ -505,6 +505,97 @@ ECHO_API int echo_rank_reduce(const void* x, void* out, echo_state* st, int bits
  * writes the reduced result (n bf16) into `out`. Nothing to do when P == 1. */
 ECHO_API int echo_rank_decode(void* out, echo_state* st, int bits, echo_stream_t stream);
 
+/*
+ * Chunked calls of one rank: the explainer ("Echoの仕組み①") hides
+ * quantization behind the transfers with a tiled pipeline. Here a call is cut
+ * into `chunks` column chunks so that the caller can overlap chunk c's
+ * exchanges with chunk c + 1's kernels (on two streams ordered by events;
+ * nothing in these kernels waits on another GPU).
+ *
+ * Chunk c of `chunks` takes, of every owner s's segment of len(s) groups,
+ * the part [floor(c len(s) / chunks), floor((c + 1) len(s) / chunks)),
+ * relative to the segment's first group (echo_query_chunk), so that every
+ * owner receives 1/chunks of its segment in each chunk's all-to-all. The
+ * partial last group (the last group of the last owner's segment) belongs to
+ * the last chunk. Running chunks 0 .. chunks-1 of the three phases, each
+ * chunk's exchanges between them, gives, bit for bit, the unchunked call.
+ *
+ *   echo_rank_quantize_chunk  phases 1, 2, 5 for this rank's non-owned groups
+ *                             of the chunk: the send row's slots of every
+ *                             owner's part
+ *   all-to-all of the chunk   (caller) to owner s: send slots
+ *                             [seg_begin(s) + first(s), + count(s)); owner s
+ *                             puts what rank r sent at recv row r, slots
+ *                             [first(s), first(s) + count(s))
+ *   echo_rank_reduce_chunk    phases 1, 3, 5 for this rank's own part
+ *   all-gather of the chunk   (caller) owner o's gsend slots
+ *                             [first(o), first(o) + count(o)) to every rank's
+ *                             gathered row o, same slots
+ *   echo_rank_decode_chunk    phase 4 for every owner's part
+ * (first/count from echo_query_chunk; codes are count * code_bytes bytes at
+ * slot * code_bytes, parameter words count words at slot.)
+ *
+ *   chunk, chunks   0 <= chunk < chunks <= ECHO_MAX_CHUNKS; chunks = 1 is the
+ *                   unchunked call (echo_rank_quantize & co. are these with
+ *                   chunk 0 of 1)
+ * Other arguments and errors as for the unchunked calls; ECHO_EINVAL for a
+ * chunk out of range.
+ */
+#define ECHO_MAX_CHUNKS 4096
+
+ECHO_API int echo_rank_quantize_chunk(const void* x, echo_state* st, int bits, float eta, float alpha_long,
+                                      float alpha_short, float w, int chunk, int chunks, echo_stream_t stream);
+ECHO_API int echo_rank_reduce_chunk(const void* x, void* out, echo_state* st, int bits, float eta,
+                                    float alpha_long, float alpha_short, float w, int chunk, int chunks,
+                                    echo_stream_t stream);
+ECHO_API int echo_rank_decode_chunk(void* out, echo_state* st, int bits, int chunk, int chunks,
+                                    echo_stream_t stream);
+
+/*
+ * Owner `owner`'s part of chunk `chunk` of `chunks`: *first = the part's
+ * first group relative to the segment's first group, *count = its groups
+ * (0 when the segment has fewer groups than chunks). Host-only, no device
+ * call. ECHO_EINVAL for bad sizes, an owner outside [0, P) or a chunk out of
+ * range.
+ */
+ECHO_API int echo_query_chunk(int64_t n, int P, int group, int owner, int chunk, int chunks, int64_t* first,
+                              int64_t* count);
+
+/*
+ * ------------------------------------------------------------------------
+ * The background-traffic study (the Echo abstract and the explainer's
+ * results section "実測性能と精度": Echo's gain over a 16-bit all-reduce
+ * grows with competing traffic). On one GPU the simulated transport is HBM,
+ * so the competing traffic is an HBM copy on another stream.
+ *
+ * echo_bf16_allreduce_sim: the 16-bit baseline all-reduce simulated over P
+ * virtual ranks like echo_allreduce_sim: every outputs[r] (n bf16) receives
+ * bf16_rn of the binary32 sum of inputs[0..P-1] in rank order -- no
+ * quantization, no state. Buffers as for echo_allreduce_sim (device, 16-byte
+ * aligned; an output may be its own input). Asynchronous on `stream`.
+ * ECHO_EINVAL on a bad size or pointer, ECHO_ECUDA on a launch error.
+ */
+ECHO_API int echo_bf16_allreduce_sim(const void* const* inputs, void* const* outputs, int64_t n, int P,
+                                     echo_stream_t stream);
+
+/*
+ * echo_background_traffic: competing HBM traffic for duration_us
+ * microseconds of wall-clock time: one CTA per SM copies src to dst (bytes,
+ * a multiple of 16, 16-byte aligned, not overlapping; the copy wraps around)
+ * during the first duty_permille / 1000 of every period_us and sleeps for
+ * the rest. The kernel ends by itself when the duration has passed, whatever
+ * else runs; it waits on nothing. When moved_dev is not NULL (8-byte aligned
+ * device word) the bytes read and written are added to it. duty_permille 0
+ * launches nothing.
+ *   duty_permille 0 .. 1000, period_us 10 .. 10^6, duration_us 1 .. 6*10^7
+ * Asynchronous on `stream` (give it a stream of its own so that it overlaps
+ * the measured calls). ECHO_EINVAL on bad arguments, ECHO_ECUDA on a launch
+ * error.
+ */
+ECHO_API int echo_background_traffic(const void* src, void* dst, size_t bytes, uint32_t duty_permille,
+                                     uint32_t period_us, uint32_t duration_us, unsigned long long* moved_dev,
+                                     echo_stream_t stream);
+
 /* Release the host handle and the events echo_allreduce_sim_host created
  * for it (never the caller's device buffers). NULL is a no-op. */
 ECHO_API int echo_free(echo_state* st);

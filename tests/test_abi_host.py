@@ -162,7 +162,55 @@ def test_rank_calls_reject_bad_arguments(L):
     assert L.echo_rank_quantize(4096, None, 4, 1.0, 0.05, 0.5, 0.5, None) == E.ECHO_EINVAL
     assert L.echo_rank_reduce(4096, 4096, None, 4, 1.0, 0.05, 0.5, 0.5, None) == E.ECHO_EINVAL
     assert L.echo_rank_decode(4096, None, 4, None) == E.ECHO_EINVAL
+    assert L.echo_rank_quantize_chunk(4096, None, 4, 1.0, 0.05, 0.5, 0.5, 0, 2, None) == E.ECHO_EINVAL
+    assert L.echo_rank_reduce_chunk(4096, 4096, None, 4, 1.0, 0.05, 0.5, 0.5, 0, 2, None) == E.ECHO_EINVAL
+    assert L.echo_rank_decode_chunk(4096, None, 4, 0, 2, None) == E.ECHO_EINVAL
     assert h.value is None
+
+
+@pytest.mark.parametrize("n,P,g", [(1000, 3, 64), (1 << 29, 8, 128), (3 * 128, 4, 128), (777, 5, 32)])
+@pytest.mark.parametrize("chunks", [1, 2, 3, 7, 64])
+def test_chunk_parts_tile_each_segment(L, n, P, g, chunks):
+    """Every owner's parts of chunks 0 .. chunks-1 tile its segment in
+    order, their sizes differ by at most one group, and the last group of
+    the message (in the last owner's segment) is in the last chunk."""
+    G = -(-n // g)
+    for s in range(P):
+        seg = int(E.echo_query_rank_layout(n, P, s, g, 4, 4).seg_groups)
+        parts = [E.echo_query_chunk(n, P, g, s, c, chunks) for c in range(chunks)]
+        assert parts[0][0] == 0 and sum(c for _, c in parts) == seg
+        for (f0, c0), (f1, _) in zip(parts, parts[1:]):
+            assert f0 + c0 == f1
+        sizes = [c for _, c in parts]
+        assert max(sizes) - min(sizes) <= 1
+    if G >= P:
+        f, c = E.echo_query_chunk(n, P, g, P - 1, chunks - 1, chunks)
+        seg_last = int(E.echo_query_rank_layout(n, P, P - 1, g, 4, 4).seg_groups)
+        assert f + c == seg_last and c >= 1
+
+
+def test_traffic_calls_reject_bad_arguments(L):
+    arr = (ctypes.c_void_p * 2)(4096, 8192)
+    assert L.echo_bf16_allreduce_sim(arr, arr, 0, 2, None) == E.ECHO_EINVAL        # n < 1
+    assert L.echo_bf16_allreduce_sim(arr, arr, 100, 65, None) == E.ECHO_EINVAL     # P > 64
+    bad = (ctypes.c_void_p * 2)(4096, 8200)
+    assert L.echo_bf16_allreduce_sim(bad, arr, 100, 2, None) == E.ECHO_EINVAL      # misaligned
+    assert L.echo_bf16_allreduce_sim(None, arr, 100, 2, None) == E.ECHO_EINVAL
+    bt = L.echo_background_traffic
+    assert bt(4096, 4096 + 256, 1024, 500, 100, 1000, None, None) == E.ECHO_EINVAL    # overlapping
+    assert bt(4096, 1 << 20, 1000, 500, 100, 1000, None, None) == E.ECHO_EINVAL       # not a multiple of 16
+    assert bt(4096, 1 << 20, 1024, 1001, 100, 1000, None, None) == E.ECHO_EINVAL      # duty > 1000
+    assert bt(4096, 1 << 20, 1024, 500, 5, 1000, None, None) == E.ECHO_EINVAL         # period too short
+    assert bt(4096, 1 << 20, 1024, 500, 100, 0, None, None) == E.ECHO_EINVAL          # no duration
+    assert bt(4096, 1 << 20, 1024, 0, 100, 1000, None, None) == E.ECHO_OK             # duty 0: nothing to launch
+
+
+def test_chunk_query_rejects_bad_arguments(L):
+    f, c = ctypes.c_int64(), ctypes.c_int64()
+    for args in ((1000, 3, 64, 3, 0, 2), (1000, 3, 64, -1, 0, 2), (1000, 3, 64, 0, 2, 2), (1000, 3, 64, 0, 0, 0),
+                 (1000, 3, 64, 0, 0, E.ECHO_MAX_CHUNKS + 1), (0, 3, 64, 0, 0, 1), (1000, 3, 48, 0, 0, 1)):
+        assert L.echo_query_chunk(*args, ctypes.byref(f), ctypes.byref(c)) == E.ECHO_EINVAL, args
+    assert L.echo_query_chunk(1000, 3, 64, 0, 0, 1, None, ctypes.byref(c)) == E.ECHO_EINVAL
 
 
 def test_header_is_c_and_links(L, tmp_path):

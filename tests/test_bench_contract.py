@@ -74,3 +74,16 @@ def test_algorithmic_bytes_match_the_roofline_definition():
     assert ab["quantize"] == (P - 1) * G * 2372 and ab["reduce_gather"] == G * 4896
     assert ab["quantize"] + ab["reduce_gather"] + G * 68 == ab["total"]
     assert bench.algorithmic_bytes(P, n, g, 8)["total"] / (P * n) == 22.0625
+
+
+@pytest.mark.gpu
+def test_background_study_line():
+    out = subprocess.run([sys.executable, "bench.py", "--tokens", "2048", "--steps", "3", "--warmup", "2",
+                          "--background", "0,50,100"], cwd=ROOT, capture_output=True, text=True, timeout=900,
+                         check=True).stdout
+    bg = _last_json(out)["background"]
+    assert bg["loads_pct"] == [0, 50, 100]
+    for key in ("echo", "echo_no_feedback", "bf16", "background_alone"):
+        assert len(bg[key]) == 3 and all(v > 0 for v in bg[key][1:]), key
+    assert bg["echo_slowdown"][0] == 1.0 and bg["background_alone"][0] == 0.0
+    assert bg["background_alone"][2] > bg["background_alone"][1] > 0

@@ -158,3 +158,81 @@ def test_rank_range_flag(bad, rank):
     finally:
         for rk in ranks:
             rk.close()
+
+
+CHUNK_CASES = [
+    # P, n, group, bits, feedback, chunks
+    (2, 4096 * 3 + 5, 128, 4, True, 3),                # partial last group
+    (3, 1000, 64, 8, True, 2),
+    (8, 8192 * 3 + 77, 128, 4, True, 4),               # partial last group, owner parts of unequal size
+    (8, 8192 * 3 + 77, 128, 4, False, 7),
+    (8, 50000, 32, 4, True, 16),
+    (4, 3 * 128, 128, 4, True, 3),                     # G < P: empty segments and empty parts
+    (64, 3 * 64 * 128 + 17, 128, 4, True, 2),          # largest P
+    (64, 200 * 128, 128, 4, True, 5),                  # more chunks than some owners have groups
+]
+
+
+@pytest.mark.parametrize("P,n,group,bits,feedback,chunks", CHUNK_CASES)
+def test_chunked_ranks_match_the_oracle(P, n, group, bits, feedback, chunks):
+    """The chunked schedule (run_chunked): chunk c's exchanges, emulated by
+    copies of the chunk's pieces on a second stream, overlap the kernels of
+    the neighbouring chunks on the compute stream, ordered by events only.
+    Every rank's output and EMA rows match the oracle's whole call bit for
+    bit over two calls."""
+    p = Params(bits=bits, group=group, w=0.3, alpha_long=0.1, alpha_short=0.6)
+    fb = (p.eta, p.alpha_long, p.alpha_short, p.w)
+    G = -(-n // group)
+    ld = G * group
+    ranks = [E.EchoRank(n, P, r, group, max(bits, 4), feedback) for r in range(P)]
+    try:
+        x = random_inputs(P, n, 29 * P + n, 2.0)
+        xs = [x[r].cuda() for r in range(P)]
+        outs = [torch.full_like(t, 3.0) for t in xs]
+        el = es = None
+        if feedback:
+            el0, es0 = seeded_state(P, n, n + 7 * P)
+            for r in range(P):
+                L, S = ranks[r].ema_views()
+                L.copy_(torch.from_numpy(el0[r]))
+                S.copy_(torch.from_numpy(es0[r]))
+            el, es = padded(el0, ld), padded(es0, ld)
+        plans = [rk.plan(bits) for rk in ranks]
+        comm_stream = torch.cuda.Stream()
+
+        def comm(step, c):
+            E.exchange_chunk_in_process(plans, step, c, chunks)
+
+        xb = padded(u16(x), ld)
+        for call in range(2):
+            E.run_chunked(ranks, xs, outs, bits, fb, chunks, comm, comm_stream)
+            orc = O.echo_allreduce(xb, n_total=n, group=group, bits=bits, e_long=el, e_short=es, eta=p.eta,
+                                   alpha_long=p.alpha_long, alpha_short=p.alpha_short, w=p.w)
+            flags = 0
+            for rk in ranks:
+                flags |= rk.status()[1]
+            assert flags == orc.flags
+            for r in range(P):
+                assert np.array_equal(u16(outs[r]), orc.y[r, :n]), f"call {call}: output of rank {r}"
+                if feedback:
+                    L, S = ranks[r].ema_views()
+                    assert np.array_equal(L.cpu().numpy(), el[r, :n]), f"call {call}: e_long of rank {r}"
+                    assert np.array_equal(S.cpu().numpy(), es[r, :n]), f"call {call}: e_short of rank {r}"
+    finally:
+        for rk in ranks:
+            rk.close()
+
+
+def test_chunk_arguments_are_checked():
+    rk = E.EchoRank(4096, 2, 0)
+    try:
+        x = torch.zeros(4096, dtype=torch.bfloat16, device="cuda")
+        for chunk, chunks in ((0, 0), (2, 2), (-1, 3), (0, E.ECHO_MAX_CHUNKS + 1)):
+            with pytest.raises(E.EchoError) as ei:
+                rk.quantize_chunk(x, chunk, chunks)
+            assert ei.value.status == E.ECHO_EINVAL
+            with pytest.raises(E.EchoError) as ei:
+                rk.decode_chunk(x, chunk, chunks)
+            assert ei.value.status == E.ECHO_EINVAL
+    finally:
+        rk.close()

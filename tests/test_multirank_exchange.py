@@ -5,7 +5,11 @@ layout). Every byte a rank sends is tagged with (sender, group, byte), so
 the test checks that each owner receives exactly the payload of its segment
 from every rank, in rank order, and every rank every owner's requantized
 segment. No kernel runs here; the kernels' side of the same layout is
-checked against the oracle on the GPU (tests/test_gpu_ranks.py)."""
+checked against the oracle on the GPU (tests/test_gpu_ranks.py).
+
+The chunked call's exchanges (exchange_chunk: point-to-point pieces of every
+owner's part of a chunk, in the order the chunked schedule issues them) must
+deliver the same bytes, chunk after chunk, as the whole exchanges."""
 import os
 import socket
 
@@ -30,7 +34,7 @@ def _tag_param(r, j):
     return 1_000_000 * (r + 1) + j
 
 
-def _worker(rank, world, port, n, group, bits, q):
+def _worker(rank, world, port, n, group, bits, chunks, q):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     import sys
     sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
@@ -52,10 +56,23 @@ def _worker(rank, world, port, n, group, bits, q):
         for k in range(seg):
             plan.gsend_codes[k * cb:(k + 1) * cb] = _tag_codes(rank, b0 + k, cb).to(torch.uint8) ^ 0x55
             plan.gsend_params[k] = -_tag_param(rank, b0 + k)
-        E.exchange_all_to_all(plan)
-        E.exchange_all_gather(plan)
+        if chunks == 1:
+            E.exchange_all_to_all(plan)
+            E.exchange_all_gather(plan)
+        else:
+            # the order of the chunked schedule: all-to-all of chunk t, then
+            # all-gather of chunk t - 1
+            for t in range(chunks + 1):
+                if t < chunks:
+                    for req in E.exchange_chunk(plan, "all_to_all", t, chunks, rank):
+                        req.wait()
+                if t >= 1:
+                    for req in E.exchange_chunk(plan, "all_gather", t - 1, chunks, rank):
+                        req.wait()
         bad = []
         for r in range(P):
+            if chunks > 1 and r == rank:
+                continue          # the chunked exchange does not send an owner its own row (never read)
             for k in range(seg):
                 j = b0 + k
                 got = plan.recv_codes[(r * seg + k) * cb:(r * seg + k + 1) * cb].to(torch.int64)
@@ -76,16 +93,20 @@ def _worker(rank, world, port, n, group, bits, q):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,n,group,bits", [
-    (3, 1000, 64, 4),        # G = 16: segments of 5, 5 and 6 groups
-    (2, 777, 32, 8),         # partial last group
-    (4, 3 * 128, 128, 4),    # G = 3 < P: one rank owns nothing
+@pytest.mark.parametrize("world,n,group,bits,chunks", [
+    (3, 1000, 64, 4, 1),        # G = 16: segments of 5, 5 and 6 groups
+    (2, 777, 32, 8, 1),         # partial last group
+    (4, 3 * 128, 128, 4, 1),    # G = 3 < P: one rank owns nothing
+    (2, 777, 32, 8, 3),         # chunked: parts of 8 and 9 groups in thirds
+    (3, 1000, 64, 4, 4),        # chunked: more chunks than some parts have groups
+    (4, 5000, 32, 4, 5),
+    (4, 3 * 128, 128, 4, 2),    # chunked with an empty segment
 ])
-def test_exchange_delivers_each_segment(world, n, group, bits):
+def test_exchange_delivers_each_segment(world, n, group, bits, chunks):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, n, group, bits, q)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, n, group, bits, chunks, q)) for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
