@@ -942,10 +942,14 @@ def run_background(args):
         E.echo_background_traffic(src, dst, 10 * lv, period_us, alone_us, moved, stream=side)
         torch.cuda.synchronize(dev)
         out["background_alone"].append(int(moved.item()) / (alone_us * 1e-6) / 1e9)
-        # the calls while the copy runs (its duration covers them even if they slow down 4x)
+        # the calls while the copy runs (its duration covers them even if they
+        # slow down 3x); the copy's bandwidth during the calls is estimated
+        # from its total bytes less what it moved alone after them
         moved.zero_()
-        dur_us = 4 * window_us + 20000
+        dur_us = 3 * window_us + 20000
         E.echo_background_traffic(src, dst, 10 * lv, period_us, dur_us, moved, stream=side)
+        w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        w0.record(main)
         for key, f in calls.items():
             f()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -955,8 +959,12 @@ def run_background(args):
             e1.record(main)
             e1.synchronize()
             out[key].append(e0.elapsed_time(e1) / steps)
+        w1.record(main)
         torch.cuda.synchronize(dev)
-        out["background_during"].append(int(moved.item()) / (dur_us * 1e-6) / 1e9 if lv else 0.0)
+        busy_s = w0.elapsed_time(w1) * 1e-3
+        alone_gbs = out["background_alone"][-1]
+        during = (int(moved.item()) / 1e9 - alone_gbs * max(0.0, dur_us * 1e-6 - busy_s)) / busy_s if lv else 0.0
+        out["background_during"].append(max(0.0, during))
     for key in calls:
         base = out[key][levels.index(0)] if 0 in levels else out[key][0]
         out[key + "_slowdown"] = [t / base for t in out[key]]

@@ -796,7 +796,9 @@ int echo_bf16_allreduce_sim(const void* const* inputs, void* const* outputs, int
 
 int echo_background_traffic(const void* src, void* dst, size_t bytes, uint32_t duty_permille, uint32_t period_us,
                             uint32_t duration_us, unsigned long long* moved_dev, echo_stream_t stream) {
-    if (!src || !dst || !aligned(src, 16) || !aligned(dst, 16) || bytes < 16 || bytes % 16 != 0) return ECHO_EINVAL;
+    if (!src || !dst || !aligned(src, 16) || !aligned(dst, 16) || bytes < (size_t)echo_dev::kBgChunk ||
+        bytes % echo_dev::kBgChunk != 0)
+        return ECHO_EINVAL;
     const uintptr_t s0 = reinterpret_cast<uintptr_t>(src), d0 = reinterpret_cast<uintptr_t>(dst);
     if (s0 < d0 + bytes && d0 < s0 + bytes) return ECHO_EINVAL;   // overlapping buffers
     if (duty_permille > 1000 || period_us < 10 || period_us > 1000000 || duration_us < 1 ||
@@ -810,9 +812,16 @@ int echo_background_traffic(const void* src, void* dst, size_t bytes, uint32_t d
     if (sms == 0) return ECHO_ECUDA;
     const unsigned long long period_ns = 1000ull * period_us;
     const unsigned long long on_ns = period_ns * duty_permille / 1000ull;
-    echo_dev::k_background_traffic<<<sms, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        static_cast<const uint4*>(src), static_cast<uint4*>(dst), (long long)(bytes / 16), on_ns, period_ns,
-        1000ull * duration_us, moved_dev);
+    static int smem_set[kMaxDevices];
+    if (!smem_set[dev]) {
+        if (cudaFuncSetAttribute(echo_dev::k_background_traffic, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 echo_dev::kBgSmem) != cudaSuccess)
+            return ECHO_ECUDA;
+        smem_set[dev] = 1;
+    }
+    echo_dev::k_background_traffic<<<sms, 32, echo_dev::kBgSmem, reinterpret_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint8_t*>(src), static_cast<uint8_t*>(dst), (long long)(bytes / echo_dev::kBgChunk), on_ns,
+        period_ns, 1000ull * duration_us, moved_dev);
     return cuda_status(cudaGetLastError());
 }
 

@@ -151,37 +151,34 @@ struct Tile {
     int count;
 };
 
-template <int GROUP, int M = 1>
+template <int GROUP, int M = 1, bool RK = false>
 struct RunWalker {
     static constexpr int T = M * kTileElems / GROUP;   // groups per tile (M sub-tiles)
     // kind 0: non-owned runs of the ranks [rank_lo, rank_hi) (quantize); kind
-    // 1: the owned runs of those ranks (reduce).
+    // 1: the owned runs of those ranks (reduce). RK: one rank of a multi-GPU
+    // call (rank_hi = rank_lo + 1), whose calls may be chunked.
     // G, P and the window are read from the kernel arguments when needed
     // rather than held in registers.
     int kind;
     int run;            // current run index
-    int cur_rank;       // the rank of the current run
     long long base;     // first tile index of the current run
     long long run_j0, run_len;
 
     // run `run` before clipping. Kind 0, rank r = run / 2: [0, lo) for even
     // runs, [hi, G) for odd; kind 1: [lo, hi) of rank `run`, where [lo, hi)
-    // is that rank's owned segment. In a chunked call (chunk_k > 0) kind 0
-    // has a run per (rank r = run / P, owner s = run % P): owner s's part of
-    // the chunk, empty for s = r; kind 1 the owned segment's part. Clipped to
-    // the call's full-group window [c0, c1) (a partial last group takes the
-    // kernels' scalar path).
+    // is that rank's owned segment. In a chunked rank call (chunk_k > 0)
+    // kind 0 has a run per owner s = run - P rank_lo: owner s's part of the
+    // chunk, empty for the rank's own segment; kind 1 the owned segment's
+    // part. Clipped to the call's full-group window [c0, c1) (a partial last
+    // group takes the kernels' scalar path).
     __device__ __forceinline__ void load_run(const Args& a) {
         long long b, e;
-        if (a.chunk_k > 0) {
-            const int r = kind == 0 ? run / a.P : run;
-            const int s = kind == 0 ? run - r * a.P : run;
-            cur_rank = r;
+        if (RK && a.chunk_k > 0) {
+            const int s = kind == 0 ? run - a.P * a.rank_lo : run;
             segment_part(a, s, &b, &e);
-            if (kind == 0 && s == r) e = b;
+            if (kind == 0 && s == a.rank_lo) e = b;
         } else {
             const int r = kind == 0 ? run >> 1 : run;
-            cur_rank = r;
             const long long lo = (long long)r * a.G / a.P, hi = (long long)(r + 1) * a.G / a.P;
             if (kind == 1) {
                 b = lo;
@@ -200,12 +197,14 @@ struct RunWalker {
         run_len = max(0LL, e - b);
     }
     __device__ __forceinline__ int runs_per_rank(const Args& a) const {
-        return kind == 1 ? 1 : (a.chunk_k > 0 ? a.P : 2);
+        return kind == 1 ? 1 : ((RK && a.chunk_k > 0) ? a.P : 2);
     }
     __device__ __forceinline__ int runs(const Args& a) const { return runs_per_rank(a) * a.rank_hi; }
-    __device__ __forceinline__ int rank_of_run() const { return cur_rank; }
+    __device__ __forceinline__ int rank_of_run(const Args& a) const {
+        return RK ? a.rank_lo : (kind == 0 ? (run >> 1) : run);
+    }
 
-    __device__ __forceinline__ RunWalker(int kind_, const Args& a) : kind(kind_), cur_rank(0), base(0) {
+    __device__ __forceinline__ RunWalker(int kind_, const Args& a) : kind(kind_), base(0) {
         run = runs_per_rank(a) * a.rank_lo;
         if (run < runs(a)) load_run(a);
     }
@@ -216,7 +215,7 @@ struct RunWalker {
             const long long nt = (run_len + T - 1) / T;
             if (k < base + nt) {
                 const long long off = (k - base) * T;
-                t->rank = rank_of_run();
+                t->rank = rank_of_run(a);
                 t->j0 = run_j0 + off;
                 t->count = (int)min((long long)T, run_len - off);
                 return true;
@@ -277,7 +276,7 @@ __device__ __forceinline__ void report_timeout(const Args& a, const PipeShared& 
 // stores keep the memory system busier, ran 3.54 -> 3.78 ms with it and goes
 // without).
 template <int GROUP, int M, int NS, bool RK, int PF_CB = 0>
-__device__ __forceinline__ void produce(const Args& a, const PipeShared& p, RunWalker<GROUP, M>& walker,
+__device__ __forceinline__ void produce(const Args& a, const PipeShared& p, RunWalker<GROUP, M, RK>& walker,
                                         bool with_state) {
     long long issued = 0;
     Tile t;
@@ -740,7 +739,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
     griddep_launch_dependents();
     pipe_init<NS>(p);
     const int warp = threadIdx.x >> 5;
-    RunWalker<GROUP, M> walker(0, a);
+    RunWalker<GROUP, M, RK> walker(0, a);
     if (warp == kConsumerWarps) {
         if ((threadIdx.x & 31) == 0) produce<GROUP, M, NS, RK>(a, p, walker, FB);
         return;
@@ -1260,7 +1259,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
     const PipeShared p = pipe_shared<NS>(smem);
     pipe_init<NS>(p, HALVES ? kConsumerWarps / 2 : kConsumerWarps);
     const int warp = threadIdx.x >> 5;
-    RunWalker<GROUP, M> walker(1, a);
+    RunWalker<GROUP, M, RK> walker(1, a);
     if (warp == kConsumerWarps) {
         // the owned groups' x and EMAs: the quantize pass writes neither, so
         // the producer may stage them while that pass is still running

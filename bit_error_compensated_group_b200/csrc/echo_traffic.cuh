@@ -9,13 +9,16 @@
 //                         virtual ranks: every rank's output is the bf16
 //                         rounding of the binary32 sum of the P bf16 inputs
 //                         in rank order (no quantization, no state);
-//   k_background_traffic  competing HBM traffic: a copy that runs for a duty
-//                         cycle of every period and sleeps for the rest, for
-//                         a fixed wall-clock time, on its own stream.
+//   k_background_traffic  competing HBM traffic: a bulk (TMA) copy that runs
+//                         for a duty cycle of every period and sleeps for the
+//                         rest, for a fixed wall-clock time, on its own
+//                         stream.
 #pragma once
 
 #include <cuda_bf16.h>
 #include <stdint.h>
+
+#include "echo_pipeline.cuh"
 
 namespace echo_dev {
 
@@ -73,48 +76,75 @@ __global__ void __launch_bounds__(kBf16Threads) k_bf16_allreduce_sim(const Args 
     }
 }
 
-__device__ __forceinline__ unsigned long long traffic_ns() {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
+// Competing HBM traffic: one warp per CTA, one CTA per SM; its lane 0
+// copies 16 KB chunks of src to dst through a 2-slot shared-memory ring with
+// bulk copies (the TMA engine: loads complete on an mbarrier, stores are
+// bulk-async groups), so a few registers and 32 KB of shared memory per SM
+// keep 32 KB in flight per SM and the kernel fits beside the all-reduce's
+// own CTAs. The copy runs during the first on_ns of every period_ns and
+// pauses (ring drained, thread asleep) for the rest, until duration_ns have
+// passed since the CTA started -- a fixed wall-clock bound: the kernel ends
+// by itself whatever else runs. Chunk c of the CTA is global chunk
+// blockIdx.x + c * gridDim.x, wrapping around src. Bytes read and written
+// are added to *moved (when not null).
+constexpr int kBgChunk = 16384;
+constexpr int kBgSlots = 2;
+constexpr int kBgSmem = kBgChunk * kBgSlots;
+constexpr unsigned long long kBgWaitNs = 1000ull * 1000ull * 1000ull;   // 1 s, never reached by a landing load
 
-// Competing HBM traffic. Every thread walks the n16 16-byte words of src
-// with the grid stride (wrapping around), copying them to dst during the
-// first on_ns of every period_ns and sleeping for the rest, until
-// duration_ns have passed since the CTA started (a fixed wall-clock bound:
-// the kernel ends by itself whatever else runs). The bytes copied are added
-// to *moved (when not null), one atomic per warp.
-__global__ void __launch_bounds__(256) k_background_traffic(const uint4* src, uint4* dst, long long n16,
-                                                            unsigned long long on_ns, unsigned long long period_ns,
-                                                            unsigned long long duration_ns,
-                                                            unsigned long long* moved) {
-    const long long stride = (long long)gridDim.x * blockDim.x;
-    long long i = ((long long)blockIdx.x * blockDim.x + threadIdx.x) % n16;
-    const unsigned long long t0 = traffic_ns();
+__global__ void __launch_bounds__(32) k_background_traffic(const uint8_t* src, uint8_t* dst, long long nchunks,
+                                                           unsigned long long on_ns, unsigned long long period_ns,
+                                                           unsigned long long duration_ns,
+                                                           unsigned long long* moved) {
+    extern __shared__ __align__(128) uint8_t ring[];
+    __shared__ uint64_t bar[kBgSlots];
+    if (threadIdx.x != 0) return;
+    for (int k = 0; k < kBgSlots; ++k) mbar_init(&bar[k], 1);
+    mbar_fence_init();
+    const unsigned long long t0 = global_ns();
     unsigned long long copied = 0;
-    while (true) {
-        const unsigned long long t = traffic_ns() - t0;
+    long long c = blockIdx.x % nchunks;
+    uint32_t uses[kBgSlots] = {0u, 0u};   // completed phases of each slot's barrier
+    bool failed = false;
+    while (!failed) {
+        const unsigned long long t = global_ns() - t0;
         if (t >= duration_ns) break;
         const unsigned long long phase = t % period_ns;
-        if (phase < on_ns) {
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                __stcs(dst + i, __ldcs(src + i));
-                i += stride;
-                if (i >= n16) i -= n16 * (i / n16);
-            }
-            copied += 8 * 16;
-        } else {
+        if (phase >= on_ns) {
             const unsigned long long rest = period_ns - phase;
             __nanosleep((unsigned)(rest < 20000ull ? rest : 20000ull));
+            continue;
+        }
+        // a burst of two chunks per slot (128 KB per CTA), then the time is
+        // read again
+        for (int b = 0; b < 2 && !failed; ++b) {
+            long long cc[kBgSlots];
+            for (int k = 0; k < kBgSlots; ++k) {
+                cc[k] = c;
+                mbar_arrive_expect_tx(&bar[k], kBgChunk);
+                bulk_load(ring + k * kBgChunk, src + (size_t)c * kBgChunk, kBgChunk, &bar[k]);
+                c += gridDim.x;
+                if (c >= nchunks) c %= nchunks;
+            }
+            for (int k = 0; k < kBgSlots; ++k) {
+                // the load lands whatever else runs; the limit only guards the
+                // wait. On expiry the remaining loads are still waited for
+                // (bounded again) before the thread leaves.
+                if (!mbar_wait(&bar[k], uses[k] & 1u, kBgWaitNs, nullptr)) {
+                    failed = true;
+                    for (int q = k; q < kBgSlots; ++q) mbar_wait(&bar[q], uses[q] & 1u, kBgWaitNs, nullptr);
+                    break;
+                }
+                ++uses[k];
+                bulk_store(dst + (size_t)cc[k] * kBgChunk, ring + k * kBgChunk, kBgChunk);
+                bulk_commit();
+                copied += 2ull * kBgChunk;
+            }
+            bulk_wait_read<0>();   // the slots may be loaded again
         }
     }
-    if (moved != nullptr) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) copied += __shfl_xor_sync(0xffffffffu, copied, o);
-        if ((threadIdx.x & 31) == 0) atomicAdd(moved, 2 * copied);   // read + written
-    }
+    bulk_wait_all();
+    if (moved != nullptr) atomicAdd(moved, copied);
 }
 
 }  // namespace echo_dev

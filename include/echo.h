@@ -580,10 +580,10 @@ ECHO_API int echo_bf16_allreduce_sim(const void* const* inputs, void* const* out
 
 /*
  * echo_background_traffic: competing HBM traffic for duration_us
- * microseconds of wall-clock time: one CTA per SM copies src to dst (bytes,
- * a multiple of 16, 16-byte aligned, not overlapping; the copy wraps around)
- * during the first duty_permille / 1000 of every period_us and sleeps for
- * the rest. The kernel ends by itself when the duration has passed, whatever
+ * microseconds of wall-clock time: one single-warp CTA per SM copies src to
+ * dst in 16 KB bulk copies through 32 KB of shared memory (bytes a multiple
+ * of 16384, 16-byte aligned, not overlapping; the copy wraps around) during
+ * the first duty_permille / 1000 of every period_us and sleeps for the rest. The kernel ends by itself when the duration has passed, whatever
  * else runs; it waits on nothing. When moved_dev is not NULL (8-byte aligned
  * device word) the bytes read and written are added to it. duty_permille 0
  * launches nothing.
