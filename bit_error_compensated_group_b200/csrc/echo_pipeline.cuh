@@ -151,36 +151,35 @@ struct Tile {
     int count;
 };
 
-template <int GROUP, int M = 1, bool RK = false>
+template <int GROUP, int M, bool RK, int KIND>
 struct RunWalker {
     static constexpr int T = M * kTileElems / GROUP;   // groups per tile (M sub-tiles)
-    // kind 0: non-owned runs of the ranks [rank_lo, rank_hi) (quantize); kind
-    // 1: the owned runs of those ranks (reduce). RK: one rank of a multi-GPU
-    // call (rank_hi = rank_lo + 1), whose calls may be chunked.
+    // KIND 0: non-owned runs of the ranks [rank_lo, rank_hi) (quantize);
+    // KIND 1: the owned runs of those ranks (reduce). RK: one rank of a
+    // multi-GPU call (rank_hi = rank_lo + 1), whose calls may be chunked.
     // G, P and the window are read from the kernel arguments when needed
     // rather than held in registers.
-    int kind;
     int run;            // current run index
     long long base;     // first tile index of the current run
     long long run_j0, run_len;
 
-    // run `run` before clipping. Kind 0, rank r = run / 2: [0, lo) for even
-    // runs, [hi, G) for odd; kind 1: [lo, hi) of rank `run`, where [lo, hi)
+    // run `run` before clipping. KIND 0, rank r = run / 2: [0, lo) for even
+    // runs, [hi, G) for odd; KIND 1: [lo, hi) of rank `run`, where [lo, hi)
     // is that rank's owned segment. In a chunked rank call (chunk_k > 0)
-    // kind 0 has a run per owner s = run - P rank_lo: owner s's part of the
-    // chunk, empty for the rank's own segment; kind 1 the owned segment's
+    // KIND 0 has a run per owner s = run - P rank_lo: owner s's part of the
+    // chunk, empty for the rank's own segment; KIND 1 the owned segment's
     // part. Clipped to the call's full-group window [c0, c1) (a partial last
     // group takes the kernels' scalar path).
     __device__ __forceinline__ void load_run(const Args& a) {
         long long b, e;
         if (RK && a.chunk_k > 0) {
-            const int s = kind == 0 ? run - a.P * a.rank_lo : run;
+            const int s = KIND == 0 ? run - a.P * a.rank_lo : run;
             segment_part(a, s, &b, &e);
-            if (kind == 0 && s == a.rank_lo) e = b;
+            if (KIND == 0 && s == a.rank_lo) e = b;
         } else {
-            const int r = kind == 0 ? run >> 1 : run;
+            const int r = KIND == 0 ? run >> 1 : run;
             const long long lo = (long long)r * a.G / a.P, hi = (long long)(r + 1) * a.G / a.P;
-            if (kind == 1) {
+            if (KIND == 1) {
                 b = lo;
                 e = hi;
             } else if ((run & 1) == 0) {
@@ -197,14 +196,14 @@ struct RunWalker {
         run_len = max(0LL, e - b);
     }
     __device__ __forceinline__ int runs_per_rank(const Args& a) const {
-        return kind == 1 ? 1 : ((RK && a.chunk_k > 0) ? a.P : 2);
+        return KIND == 1 ? 1 : ((RK && a.chunk_k > 0) ? a.P : 2);
     }
     __device__ __forceinline__ int runs(const Args& a) const { return runs_per_rank(a) * a.rank_hi; }
     __device__ __forceinline__ int rank_of_run(const Args& a) const {
-        return RK ? a.rank_lo : (kind == 0 ? (run >> 1) : run);
+        return RK ? a.rank_lo : (KIND == 0 ? (run >> 1) : run);
     }
 
-    __device__ __forceinline__ RunWalker(int kind_, const Args& a) : kind(kind_), base(0) {
+    __device__ __forceinline__ explicit RunWalker(const Args& a) : base(0) {
         run = runs_per_rank(a) * a.rank_lo;
         if (run < runs(a)) load_run(a);
     }
@@ -275,8 +274,8 @@ __device__ __forceinline__ void report_timeout(const Args& a, const PipeShared& 
 // on the 1 GB P = 8 message; the simulation's owners' pass, whose output
 // stores keep the memory system busier, ran 3.54 -> 3.78 ms with it and goes
 // without).
-template <int GROUP, int M, int NS, bool RK, int PF_CB = 0>
-__device__ __forceinline__ void produce(const Args& a, const PipeShared& p, RunWalker<GROUP, M, RK>& walker,
+template <int GROUP, int M, int NS, bool RK, int KIND, int PF_CB = 0>
+__device__ __forceinline__ void produce(const Args& a, const PipeShared& p, RunWalker<GROUP, M, RK, KIND>& walker,
                                         bool with_state) {
     long long issued = 0;
     Tile t;
@@ -739,9 +738,9 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
     griddep_launch_dependents();
     pipe_init<NS>(p);
     const int warp = threadIdx.x >> 5;
-    RunWalker<GROUP, M, RK> walker(0, a);
+    RunWalker<GROUP, M, RK, 0> walker(a);
     if (warp == kConsumerWarps) {
-        if ((threadIdx.x & 31) == 0) produce<GROUP, M, NS, RK>(a, p, walker, FB);
+        if ((threadIdx.x & 31) == 0) produce<GROUP, M, NS, RK, 0>(a, p, walker, FB);
         return;
     }
     // with feedback: 8 elements per lane, one pass per tile; without: 32 per
@@ -819,6 +818,11 @@ constexpr int kReduceRankBatch = 8;   // ranks whose payload loads are issued to
 // the simulation's owners' pass: load the next tile's first payload batch
 // while the current tile is computed
 constexpr bool kReducePrefetch = false;
+// more than kReduceRankBatch ranks: issue the next batch's payload loads
+// before the current batch is decoded
+constexpr bool kReducePipelinedBatches = false;
+// issue a tile's first payload batch before waiting for its staged x and EMAs
+constexpr bool kReduceLoadsBeforeWait = true;
 
 // The payload loads of ranks [r0, r0 + RB) for lane t's 8 elements of group
 // j: one code word (two at 8 bits) and the group's parameter word per rank;
@@ -877,7 +881,10 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
 #pragma unroll
         for (int p = 0; p < 4; ++p) xo[p] = inject2(xo[p], el[p], es[p], a);
     }
-    // binary32 sum in rank order 0..P-1: own x' unquantized, others decoded
+    // binary32 sum in rank order 0..P-1: own x' unquantized, others decoded.
+    // With more than RB ranks (kReducePipelinedBatches), batch b + 1's
+    // payload loads are issued before batch b is decoded.
+    uint32_t cwn[RB][CW], pwn[RB];
     for (int r0 = 0; r0 < a.P; r0 += RB) {
         uint32_t cw[RB][CW];
         uint32_t pw[RB];
@@ -888,9 +895,18 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
 #pragma unroll
                 for (int c = 0; c < CW; ++c) cw[k][c] = cw0[k][c];
             }
+        } else if (kReducePipelinedBatches) {
+#pragma unroll
+            for (int k = 0; k < RB; ++k) {
+                pw[k] = pwn[k];
+#pragma unroll
+                for (int c = 0; c < CW; ++c) cw[k][c] = cwn[k][c];
+            }
         } else {
             load_payload8<GROUP, BITS, RK, RB>(a, o, j, ln.t, act, r0, cw, pw);
         }
+        if (kReducePipelinedBatches && r0 + RB < a.P)
+            load_payload8<GROUP, BITS, RK, RB>(a, o, j, ln.t, act, r0 + RB, cwn, pwn);
 #pragma unroll
         for (int k = 0; k < RB; ++k) {
             const int r = r0 + k;
@@ -1259,11 +1275,11 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
     const PipeShared p = pipe_shared<NS>(smem);
     pipe_init<NS>(p, HALVES ? kConsumerWarps / 2 : kConsumerWarps);
     const int warp = threadIdx.x >> 5;
-    RunWalker<GROUP, M, RK> walker(1, a);
+    RunWalker<GROUP, M, RK, 1> walker(a);
     if (warp == kConsumerWarps) {
         // the owned groups' x and EMAs: the quantize pass writes neither, so
         // the producer may stage them while that pass is still running
-        if ((threadIdx.x & 31) == 0) produce<GROUP, M, NS, RK, RK ? GROUP * BITS / 8 : 0>(a, p, walker, FB);
+        if ((threadIdx.x & 31) == 0) produce<GROUP, M, NS, RK, 1, RK ? GROUP * BITS / 8 : 0>(a, p, walker, FB);
         return;
     }
     // the payload, the flag word and the outputs: only once the quantize pass
@@ -1317,11 +1333,14 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
         for (long long k = blockIdx.x; walker.locate(k, &t, a); k += gridDim.x, ++i) {
             const int s = (int)(i % NS);
             uint32_t cw[kReduceRankBatch][CW], pw[kReduceRankBatch];
-            load_payload8<GROUP, BITS, RK, kReduceRankBatch>(a, t.rank, t.j0 + gi, lt, gi < t.count, 0, cw, pw);
+            if (kReduceLoadsBeforeWait)
+                load_payload8<GROUP, BITS, RK, kReduceRankBatch>(a, t.rank, t.j0 + gi, lt, gi < t.count, 0, cw, pw);
             if (!mbar_wait(&p.full[s], (uint32_t)(i / NS) & 1u, a.wait_ns, p.abort)) {
                 if (lead) report_timeout(a, p);
                 return;
             }
+            if (!kReduceLoadsBeforeWait)
+                load_payload8<GROUP, BITS, RK, kReduceRankBatch>(a, t.rank, t.j0 + gi, lt, gi < t.count, 0, cw, pw);
             reduce_tile_group<GROUP, BITS, QM, RK>(a, p.stages + (size_t)s * kStageBytes, t, gi, gi < t.count, cw,
                                                    pw);
             __syncwarp();
