@@ -933,7 +933,7 @@ def run_background(args):
     period_us = 100
     levels = [int(v) for v in str(args.background).split(",") if v.strip()]
     out = {"loads_pct": levels, "period_us": period_us}
-    for key in list(calls) + ["background_alone", "background_during"]:
+    for key in list(calls) + ["background_alone", "background_during_estimate"]:
         out[key] = []
     for lv in levels:
         # the copy alone: its bandwidth at this duty cycle
@@ -964,7 +964,7 @@ def run_background(args):
         busy_s = w0.elapsed_time(w1) * 1e-3
         alone_gbs = out["background_alone"][-1]
         during = (int(moved.item()) / 1e9 - alone_gbs * max(0.0, dur_us * 1e-6 - busy_s)) / busy_s if lv else 0.0
-        out["background_during"].append(max(0.0, during))
+        out["background_during_estimate"].append(max(0.0, during))
     for key in calls:
         base = out[key][levels.index(0)] if 0 in levels else out[key][0]
         out[key + "_slowdown"] = [t / base for t in out[key]]

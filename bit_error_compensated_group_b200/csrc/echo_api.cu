@@ -182,6 +182,10 @@ int launch_stage(Stage stage, const echo_dev::Args& a, const echo_state* st, cud
                 static int grid[kMaxDevices];
                 rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, false, QM, true>, grid, tiles, a, st, s,
                                  echo_dev::pipe_smem(echo_dev::kStagesReduceNF), pdl);
+            } else if (a.state && a.P > echo_dev::kReduceRankBatch) {
+                static int grid[kMaxDevices];
+                rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, true, QM, false, true>, grid, tiles, a, st, s,
+                                 echo_dev::pipe_smem(echo_dev::kStagesReduceFB), pdl);
             } else if (a.state) {
                 static int grid[kMaxDevices];
                 rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, true, QM>, grid, tiles, a, st, s,

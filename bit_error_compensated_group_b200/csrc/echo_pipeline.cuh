@@ -815,14 +815,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_quantize_tma(const Args a) 
 // One owned group of a tile with feedback (x, e_long, e_short staged): 8
 // consecutive elements per lane, like the quantize pass.
 constexpr int kReduceRankBatch = 8;   // ranks whose payload loads are issued together
-// the simulation's owners' pass: load the next tile's first payload batch
-// while the current tile is computed
-constexpr bool kReducePrefetch = false;
-// more than kReduceRankBatch ranks: issue the next batch's payload loads
-// before the current batch is decoded
-constexpr bool kReducePipelinedBatches = false;
-// issue a tile's first payload batch before waiting for its staged x and EMAs
-constexpr bool kReduceLoadsBeforeWait = true;
+
 
 // The payload loads of ranks [r0, r0 + RB) for lane t's 8 elements of group
 // j: one code word (two at 8 bits) and the group's parameter word per rank;
@@ -853,9 +846,11 @@ __device__ __forceinline__ void load_payload8(const Args& a, int o, long long j,
 }
 
 // `cw0` / `pw0`: the first batch's payload words, already loaded by the
-// caller (for the next tile while the previous one was computed); later
-// batches (P > RB) are loaded here.
-template <int GROUP, int BITS, int QM, bool RK>
+// caller; later batches (P > RB) are loaded here -- with WIDE, each one
+// before the previous batch is decoded, so that its latency hides behind
+// that work (the registers it takes spill at P <= RB, which therefore runs
+// the instantiation without it).
+template <int GROUP, int BITS, int QM, bool RK, bool WIDE = false>
 __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* st, const Tile& t, int gi,
                                                   bool act, const uint32_t (&cw0)[kReduceRankBatch][BITS / 4],
                                                   const uint32_t (&pw0)[kReduceRankBatch]) {
@@ -881,9 +876,7 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
 #pragma unroll
         for (int p = 0; p < 4; ++p) xo[p] = inject2(xo[p], el[p], es[p], a);
     }
-    // binary32 sum in rank order 0..P-1: own x' unquantized, others decoded.
-    // With more than RB ranks (kReducePipelinedBatches), batch b + 1's
-    // payload loads are issued before batch b is decoded.
+    // binary32 sum in rank order 0..P-1: own x' unquantized, others decoded
     uint32_t cwn[RB][CW], pwn[RB];
     for (int r0 = 0; r0 < a.P; r0 += RB) {
         uint32_t cw[RB][CW];
@@ -895,7 +888,7 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
 #pragma unroll
                 for (int c = 0; c < CW; ++c) cw[k][c] = cw0[k][c];
             }
-        } else if (kReducePipelinedBatches) {
+        } else if (WIDE) {
 #pragma unroll
             for (int k = 0; k < RB; ++k) {
                 pw[k] = pwn[k];
@@ -905,7 +898,7 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
         } else {
             load_payload8<GROUP, BITS, RK, RB>(a, o, j, ln.t, act, r0, cw, pw);
         }
-        if (kReducePipelinedBatches && r0 + RB < a.P)
+        if (WIDE && r0 + RB < a.P)
             load_payload8<GROUP, BITS, RK, RB>(a, o, j, ln.t, act, r0 + RB, cwn, pwn);
 #pragma unroll
         for (int k = 0; k < RB; ++k) {
@@ -1261,7 +1254,9 @@ __device__ __forceinline__ void reduce_tile_group_nf(const Args& a, const uint8_
 
 // Two CTAs of kPipeThreads per SM: 96 registers per thread (each SM
 // sub-partition's 16384 registers then hold its share of the 18 warps).
-template <int GROUP, int BITS, bool FB, int QM, bool RK = false>
+// WIDE (the simulation with feedback and P > kReduceRankBatch): pipelined
+// payload batches, see reduce_tile_group.
+template <int GROUP, int BITS, bool FB, int QM, bool RK = false, bool WIDE = false>
 __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
     constexpr int M = FB ? 1 : kReduceSubtilesNF;
@@ -1287,62 +1282,24 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
     griddep_wait();
     const bool lead = (threadIdx.x & 31) == 0;
     Tile t;
-    if (FB && !RK && kReducePrefetch) {
-        // The simulation: the first batch of a tile's payload loads is issued
-        // while the previous tile is computed (registers carry it), so their
-        // latency hides behind that work instead of stalling the tile.
-        constexpr int CW = BITS / 4;
-        const int gi = warp * Lane<GROUP>::GPW + Lane<GROUP>().sub;
-        const int lt = Lane<GROUP>().t;
-        long long k = blockIdx.x, i = 0;
-        bool have = walker.locate(k, &t, a);
-        uint32_t cw[kReduceRankBatch][CW], pw[kReduceRankBatch];
-        if (have) load_payload8<GROUP, BITS, RK, kReduceRankBatch>(a, t.rank, t.j0 + gi, lt, gi < t.count, 0, cw, pw);
-        while (have) {
-            const int s = (int)(i % NS);
-            if (!mbar_wait(&p.full[s], (uint32_t)(i / NS) & 1u, a.wait_ns, p.abort)) {
-                if (lead) report_timeout(a, p);
-                return;
-            }
-            Tile tn;
-            const bool have_next = walker.locate(k + gridDim.x, &tn, a);
-            uint32_t cwn[kReduceRankBatch][CW], pwn[kReduceRankBatch];
-            load_payload8<GROUP, BITS, RK, kReduceRankBatch>(a, tn.rank, tn.j0 + gi, lt, have_next && gi < tn.count,
-                                                            0, cwn, pwn);
-            reduce_tile_group<GROUP, BITS, QM, RK>(a, p.stages + (size_t)s * kStageBytes, t, gi, gi < t.count, cw,
-                                                   pw);
-            __syncwarp();
-            if (lead) mbar_arrive(&p.empty[s]);
-#pragma unroll
-            for (int q = 0; q < kReduceRankBatch; ++q) {
-                pw[q] = pwn[q];
-#pragma unroll
-                for (int c = 0; c < CW; ++c) cw[q][c] = cwn[q][c];
-            }
-            t = tn;
-            have = have_next;
-            k += gridDim.x;
-            ++i;
-        }
-    } else if (FB && !RK) {
-        // The simulation, payload loads issued at the start of each tile
+    if (FB && !RK) {
+        // The simulation: 8 elements per lane, the first payload batch loaded
+        // once the tile is staged (issuing it before the wait measured 1-2 %
+        // slower)
         constexpr int CW = BITS / 4;
         const int gi = warp * Lane<GROUP>::GPW + Lane<GROUP>().sub;
         const int lt = Lane<GROUP>().t;
         long long i = 0;
         for (long long k = blockIdx.x; walker.locate(k, &t, a); k += gridDim.x, ++i) {
             const int s = (int)(i % NS);
-            uint32_t cw[kReduceRankBatch][CW], pw[kReduceRankBatch];
-            if (kReduceLoadsBeforeWait)
-                load_payload8<GROUP, BITS, RK, kReduceRankBatch>(a, t.rank, t.j0 + gi, lt, gi < t.count, 0, cw, pw);
             if (!mbar_wait(&p.full[s], (uint32_t)(i / NS) & 1u, a.wait_ns, p.abort)) {
                 if (lead) report_timeout(a, p);
                 return;
             }
-            if (!kReduceLoadsBeforeWait)
-                load_payload8<GROUP, BITS, RK, kReduceRankBatch>(a, t.rank, t.j0 + gi, lt, gi < t.count, 0, cw, pw);
-            reduce_tile_group<GROUP, BITS, QM, RK>(a, p.stages + (size_t)s * kStageBytes, t, gi, gi < t.count, cw,
-                                                   pw);
+            uint32_t cw[kReduceRankBatch][CW], pw[kReduceRankBatch];
+            load_payload8<GROUP, BITS, RK, kReduceRankBatch>(a, t.rank, t.j0 + gi, lt, gi < t.count, 0, cw, pw);
+            reduce_tile_group<GROUP, BITS, QM, RK, WIDE>(a, p.stages + (size_t)s * kStageBytes, t, gi, gi < t.count,
+                                                         cw, pw);
             __syncwarp();
             if (lead) mbar_arrive(&p.empty[s]);
         }
