@@ -197,12 +197,14 @@ def test_traffic_calls_reject_bad_arguments(L):
     assert L.echo_bf16_allreduce_sim(bad, arr, 100, 2, None) == E.ECHO_EINVAL      # misaligned
     assert L.echo_bf16_allreduce_sim(None, arr, 100, 2, None) == E.ECHO_EINVAL
     bt = L.echo_background_traffic
-    assert bt(4096, 4096 + 256, 1024, 500, 100, 1000, None, None) == E.ECHO_EINVAL    # overlapping
-    assert bt(4096, 1 << 20, 1000, 500, 100, 1000, None, None) == E.ECHO_EINVAL       # not a multiple of 16
-    assert bt(4096, 1 << 20, 1024, 1001, 100, 1000, None, None) == E.ECHO_EINVAL      # duty > 1000
-    assert bt(4096, 1 << 20, 1024, 500, 5, 1000, None, None) == E.ECHO_EINVAL         # period too short
-    assert bt(4096, 1 << 20, 1024, 500, 100, 0, None, None) == E.ECHO_EINVAL          # no duration
-    assert bt(4096, 1 << 20, 1024, 0, 100, 1000, None, None) == E.ECHO_OK             # duty 0: nothing to launch
+    chunk = 16384                                                                        # the copy's unit
+    assert bt(4096, 4096 + 256, chunk, 500, 100, 1000, None, None) == E.ECHO_EINVAL     # overlapping
+    assert bt(4096, 1 << 20, chunk + 16, 500, 100, 1000, None, None) == E.ECHO_EINVAL   # not a multiple of 16 KB
+    assert bt(4096, 1 << 20, 1024, 500, 100, 1000, None, None) == E.ECHO_EINVAL         # less than one chunk
+    assert bt(4096, 1 << 20, chunk, 1001, 100, 1000, None, None) == E.ECHO_EINVAL       # duty > 1000
+    assert bt(4096, 1 << 20, chunk, 500, 5, 1000, None, None) == E.ECHO_EINVAL          # period too short
+    assert bt(4096, 1 << 20, chunk, 500, 100, 0, None, None) == E.ECHO_EINVAL           # no duration
+    assert bt(4096, 1 << 20, chunk, 0, 100, 1000, None, None) == E.ECHO_OK              # duty 0: nothing to launch
 
 
 def test_chunk_query_rejects_bad_arguments(L):
