@@ -111,7 +111,11 @@ __device__ __forceinline__ size_t a2a_slot(const Args& a, int r, long long j) {
 
 // The pipelined kernels' simulation instantiations (RK = false) keep the
 // plain [P][G] slot and [P][2][S] state addressing; one rank of a
-// multi-GPU call (RK = true) uses the general form above.
+// multi-GPU call (RK = true) uses the general form above. In that mode every
+// buffer an Args points at -- the received rows included, which the caller's
+// collectives land there -- is this GPU's own memory: the bulk copies and L2
+// prefetches of the pipelines never read another GPU's memory, and Args must
+// never carry a peer pointer (no load here uses cluster multicast either).
 template <bool RK>
 __device__ __forceinline__ size_t a2a_slot_t(const Args& a, int r, long long j) {
     return RK ? a2a_slot(a, r, j) : (size_t)r * (size_t)a.G + (size_t)j;

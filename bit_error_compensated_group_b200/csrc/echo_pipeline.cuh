@@ -273,7 +273,8 @@ __device__ __forceinline__ void report_timeout(const Args& a, const PipeShared& 
 // slots find them there (measured on one B200: that pass 0.333 -> 0.316 ms
 // on the 1 GB P = 8 message; the simulation's owners' pass, whose output
 // stores keep the memory system busier, ran 3.54 -> 3.78 ms with it and goes
-// without).
+// without). Every source here is this GPU's own memory (see a2a_slot_t):
+// the loads are plain bulk copies, none with cluster multicast.
 template <int GROUP, int M, int NS, bool RK, int KIND, int PF_CB = 0>
 __device__ __forceinline__ void produce(const Args& a, const PipeShared& p, RunWalker<GROUP, M, RK, KIND>& walker,
                                         bool with_state) {
@@ -850,13 +851,14 @@ __device__ __forceinline__ void load_payload8(const Args& a, int o, long long j,
 // before the previous batch is decoded, so that its latency hides behind
 // that work (the registers it takes spill at P <= RB, which therefore runs
 // the instantiation without it).
-template <int GROUP, int BITS, int QM, bool RK, bool WIDE = false>
+// STATE = false (one rank of a multi-GPU call without feedback): the stage
+// holds x only, x' = x, and no EMA is read or written.
+template <int GROUP, int BITS, int QM, bool RK, bool WIDE = false, bool STATE = true, int RB = kReduceRankBatch>
 __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* st, const Tile& t, int gi,
-                                                  bool act, const uint32_t (&cw0)[kReduceRankBatch][BITS / 4],
-                                                  const uint32_t (&pw0)[kReduceRankBatch]) {
+                                                  bool act, const uint32_t (&cw0)[RB][BITS / 4],
+                                                  const uint32_t (&pw0)[RB]) {
     using LN = Lane<GROUP>;
     constexpr int L = LN::L, Q = (1 << BITS) - 1, CB = GROUP * BITS / 8;
-    constexpr int RB = kReduceRankBatch;
     constexpr int CW = BITS / 4;   // 32-bit code words per lane (8 codes)
     const LN ln;
     const int o = t.rank;
@@ -870,11 +872,13 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
     for (int p = 0; p < 4; ++p) xo[p] = acc[p] = make_float2(0.0f, 0.0f);
     if (act) {
         load_x8c_smem(xs + e0, xo);
-        float2 el[4], es[4];
-        load_f8_smem(els, e0, e0 + 4, el);
-        load_f8_smem(ess, e0, e0 + 4, es);
+        if (STATE) {
+            float2 el[4], es[4];
+            load_f8_smem(els, e0, e0 + 4, el);
+            load_f8_smem(ess, e0, e0 + 4, es);
 #pragma unroll
-        for (int p = 0; p < 4; ++p) xo[p] = inject2(xo[p], el[p], es[p], a);
+            for (int p = 0; p < 4; ++p) xo[p] = inject2(xo[p], el[p], es[p], a);
+        }
     }
     // binary32 sum in rank order 0..P-1: own x' unquantized, others decoded
     uint32_t cwn[RB][CW], pwn[RB];
@@ -959,6 +963,7 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
         for (int p = 0; p < 4; ++p) yb[p] = bf16x2_rn(acc[p]);
         *reinterpret_cast<uint4*>(a.out[0] + j * GROUP + e0) = make_uint4(yb[0], yb[1], yb[2], yb[3]);
     }
+    if (!STATE) return;
     float2 el[4], es[4], nl[4], ns[4];
     load_f8_smem(els, e0, e0 + 4, el);
     load_f8_smem(ess, e0, e0 + 4, es);
@@ -1339,6 +1344,59 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
     }
 }
 
+// The owners' pass of one rank of a multi-GPU call without feedback. It
+// moves only 800 bytes per owned group (x, P - 1 incoming payloads, the
+// gathered payload) against P - 1 decodes of every element, so it is bound by
+// instruction latency, not by HBM: this form runs three CTAs per SM (72
+// registers, 3-stage ring of 4-sub-tile stages) with 8 elements per lane, for
+// more warps in flight than k_reduce_tma's two CTAs of 16-element lanes.
+constexpr int kStagesRankNF = 3;
+constexpr int kRankNfBatch = 4;   // ranks whose payload loads are issued together (register budget)
+
+template <int GROUP, int BITS, int QM>
+__global__ void __launch_bounds__(kPipeThreads, 3) k_reduce_rank_nf(const Args a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    constexpr int M = kReduceSubtilesNF, NS = kStagesRankNF;
+    const PipeShared p = pipe_shared<NS>(smem);
+    pipe_init<NS>(p);
+    const int warp = threadIdx.x >> 5;
+    RunWalker<GROUP, M, true, 1> walker(a);
+    if (warp == kConsumerWarps) {
+        if ((threadIdx.x & 31) == 0) produce<GROUP, M, NS, true, 1, GROUP * BITS / 8>(a, p, walker, false);
+        return;
+    }
+    constexpr int CW = BITS / 4, GPW = Lane<GROUP>::GPW;
+    constexpr int PASSES = M * kTileElems / (kConsumerWarps * 32 * 8);
+    const bool lead = (threadIdx.x & 31) == 0;
+    const int gi0 = warp * GPW + Lane<GROUP>().sub;
+    const int lt = Lane<GROUP>().t;
+    long long i = 0;
+    Tile t;
+    for (long long k = blockIdx.x; walker.locate(k, &t, a); k += gridDim.x, ++i) {
+        const int s = (int)(i % NS);
+        if (!mbar_wait(&p.full[s], (uint32_t)(i / NS) & 1u, a.wait_ns, p.abort)) {
+            if (lead) report_timeout(a, p);
+            return;
+        }
+        const uint8_t* stage = p.stages + (size_t)s * kStageBytes;
+#pragma unroll 1
+        for (int m = 0; m < PASSES; ++m) {
+            const int gi = gi0 + m * kConsumerWarps * GPW;
+            uint32_t cw[kRankNfBatch][CW], pw[kRankNfBatch];
+            load_payload8<GROUP, BITS, true, kRankNfBatch>(a, t.rank, t.j0 + gi, lt, gi < t.count, 0, cw, pw);
+            reduce_tile_group<GROUP, BITS, QM, true, false, false, kRankNfBatch>(a, stage, t, gi, gi < t.count, cw,
+                                                                                   pw);
+        }
+        __syncwarp();
+        if (lead) mbar_arrive(&p.empty[s]);
+    }
+    if (a.tail && blockIdx.x == gridDim.x - 1 && warp == 0) {
+        const long long j = a.G - 1;
+        const int o = (int)((j * a.P + a.P - 1) / a.G);
+        if (o >= a.rank_lo && o < a.rank_hi) reduce_range<GROUP, BITS, QM>(a, o, j, j + 1, 0, 1);
+    }
+}
+
 // ------------------------------------------------------------ gather
 //
 // Every rank receives the same decoded group, so the kernel decodes a tile of
@@ -1434,6 +1492,7 @@ __global__ void __launch_bounds__(kGatherThreads) k_gather_tma(const Args a) {
 // per CTA in shared memory (one thread per owner, then a warp scan).
 constexpr int kDecodeThreads = 256;
 constexpr int kDecodeUnroll = 8;
+constexpr bool kDecodePrefetch = false;   // next tile's loads before this tile's decode
 constexpr int kDecodeElems = 16;
 
 __device__ __forceinline__ void store_v8_cs(void* p, uint4 lo, uint4 hi) {
@@ -1492,35 +1551,43 @@ __global__ void __launch_bounds__(kDecodeThreads) k_decode_rank(const Args a) {
     uint16_t* const out = a.out[a.out_lo];
     const bool v8 = (reinterpret_cast<uintptr_t>(out) & 31) == 0;
     int o = 0;
-    for (long long k = blockIdx.x; k < ntiles; k += gridDim.x) {
+    // tile k: chunk lc of it covers group lc / L, part lc % L, so its codes
+    // start lc * CHUNK_BYTES after the tile's first group's and its output
+    // lc * E elements after the tile's first element
+    struct TileRef {
+        int nchunks;
+        const uint8_t* codes;
+        const uint32_t* params;
+        uint16_t* y;
+    };
+    auto locate = [&](long long k, TileRef& r) {
         while (k >= tile_pre[o + 1]) ++o;
         const long long off = (k - tile_pre[o]) * TG;
         const long long j0 = run_b[o] + off;
-        // chunk lc of the tile: group lc / L, its part lc % L, so its codes
-        // start lc * CHUNK_BYTES after the tile's first group's, its output
-        // lc * E elements after the tile's first element
-        const int nchunks = (int)min((long long)TG, run_e[o] - j0) * L;
-        const uint8_t* codes = a.g_codes + (size_t)(run_slot[o] + off) * CB;
-        const uint32_t* params = a.g_params + (run_slot[o] + off);
-        uint16_t* const y = out + j0 * GROUP;
-        uint4 w[U];
-        uint32_t pw[U];
+        r.nchunks = (int)min((long long)TG, run_e[o] - j0) * L;
+        r.codes = a.g_codes + (size_t)(run_slot[o] + off) * CB;
+        r.params = a.g_params + (run_slot[o] + off);
+        r.y = out + j0 * GROUP;
+    };
+    auto load = [&](const TileRef& r, uint4 (&w)[U], uint32_t (&pw)[U]) {
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int lc = u * kDecodeThreads + tid;
-            if (lc < nchunks) {
-                w[u] = load_codes16<BITS>(codes + lc * CHUNK_BYTES);
-                pw[u] = params[lc / L];
+            if (lc < r.nchunks) {
+                w[u] = load_codes16<BITS>(r.codes + lc * CHUNK_BYTES);
+                pw[u] = r.params[lc / L];
             }
         }
+    };
+    auto decode_store = [&](const TileRef& r, const uint4 (&w)[U], const uint32_t (&pw)[U]) {
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int lc = u * kDecodeThreads + tid;
-            if (lc < nchunks) {
+            if (lc < r.nchunks) {
                 const uint4 y0 = decode8_bf16<BITS, QM>(make_uint2(w[u].x, BITS == 4 ? 0u : w[u].y), pw[u]);
                 const uint4 y1 = decode8_bf16<BITS, QM>(BITS == 4 ? make_uint2(w[u].y, 0u) : make_uint2(w[u].z, w[u].w),
                                                         pw[u]);
-                uint16_t* dst = y + lc * E;
+                uint16_t* dst = r.y + lc * E;
                 if (v8) {
                     store_v8_cs(dst, y0, y1);
                 } else {
@@ -1528,6 +1595,44 @@ __global__ void __launch_bounds__(kDecodeThreads) k_decode_rank(const Args a) {
                     __stcs(reinterpret_cast<uint4*>(dst + 8), y1);
                 }
             }
+        }
+    };
+    if (kDecodePrefetch) {
+        // the next tile's loads are issued before this tile is decoded
+        long long k = blockIdx.x;
+        TileRef cur = {0, nullptr, nullptr, nullptr};
+        uint4 w[U];
+        uint32_t pw[U];
+        if (k < ntiles) {
+            locate(k, cur);
+            load(cur, w, pw);
+        }
+        while (k < ntiles) {
+            const long long kn = k + gridDim.x;
+            TileRef nxt = {0, nullptr, nullptr, nullptr};
+            uint4 wn[U];
+            uint32_t pwn[U];
+            if (kn < ntiles) {
+                locate(kn, nxt);
+                load(nxt, wn, pwn);
+            }
+            decode_store(cur, w, pw);
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                w[u] = wn[u];
+                pw[u] = pwn[u];
+            }
+            cur = nxt;
+            k = kn;
+        }
+    } else {
+        for (long long k = blockIdx.x; k < ntiles; k += gridDim.x) {
+            TileRef cur;
+            locate(k, cur);
+            uint4 w[U];
+            uint32_t pw[U];
+            load(cur, w, pw);
+            decode_store(cur, w, pw);
         }
     }
     // the partial last group (not a multiple of 16 bytes): guarded stores
