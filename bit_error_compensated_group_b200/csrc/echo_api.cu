@@ -102,9 +102,6 @@ int pipe_grid(K kernel, const echo_state* st, int smem) {
 
 enum class Stage { Quantize, Reduce, Gather };
 
-// one rank's owners' pass without feedback: the three-CTA form
-// (k_reduce_rank_nf) or k_reduce_tma's two-CTA form
-constexpr bool kRankNfThreeCtas = false;
 
 // An upper bound on the tiles a pipelined launch walks: the runs (2 per rank
 // for quantize, 1 per owner for reduce) cut into tiles of `tile_groups`.
@@ -182,10 +179,6 @@ int launch_stage(Stage stage, const echo_dev::Args& a, const echo_state* st, cud
                 static int grid[kMaxDevices];
                 rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, true, QM, true>, grid, tiles, a, st, s,
                                  echo_dev::pipe_smem(echo_dev::kStagesReduceFB), pdl);
-            } else if (st->rank >= 0 && kRankNfThreeCtas) {
-                static int grid[kMaxDevices];
-                rc = launch_pipe(echo_dev::k_reduce_rank_nf<GROUP, BITS, QM>, grid, tiles, a, st, s,
-                                 echo_dev::pipe_smem(echo_dev::kStagesRankNF), pdl);
             } else if (st->rank >= 0) {
                 static int grid[kMaxDevices];
                 rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, false, QM, true>, grid, tiles, a, st, s,

@@ -851,14 +851,13 @@ __device__ __forceinline__ void load_payload8(const Args& a, int o, long long j,
 // before the previous batch is decoded, so that its latency hides behind
 // that work (the registers it takes spill at P <= RB, which therefore runs
 // the instantiation without it).
-// STATE = false (one rank of a multi-GPU call without feedback): the stage
-// holds x only, x' = x, and no EMA is read or written.
-template <int GROUP, int BITS, int QM, bool RK, bool WIDE = false, bool STATE = true, int RB = kReduceRankBatch>
+template <int GROUP, int BITS, int QM, bool RK, bool WIDE = false>
 __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* st, const Tile& t, int gi,
-                                                  bool act, const uint32_t (&cw0)[RB][BITS / 4],
-                                                  const uint32_t (&pw0)[RB]) {
+                                                  bool act, const uint32_t (&cw0)[kReduceRankBatch][BITS / 4],
+                                                  const uint32_t (&pw0)[kReduceRankBatch]) {
     using LN = Lane<GROUP>;
     constexpr int L = LN::L, Q = (1 << BITS) - 1, CB = GROUP * BITS / 8;
+    constexpr int RB = kReduceRankBatch;
     constexpr int CW = BITS / 4;   // 32-bit code words per lane (8 codes)
     const LN ln;
     const int o = t.rank;
@@ -872,13 +871,11 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
     for (int p = 0; p < 4; ++p) xo[p] = acc[p] = make_float2(0.0f, 0.0f);
     if (act) {
         load_x8c_smem(xs + e0, xo);
-        if (STATE) {
-            float2 el[4], es[4];
-            load_f8_smem(els, e0, e0 + 4, el);
-            load_f8_smem(ess, e0, e0 + 4, es);
+        float2 el[4], es[4];
+        load_f8_smem(els, e0, e0 + 4, el);
+        load_f8_smem(ess, e0, e0 + 4, es);
 #pragma unroll
-            for (int p = 0; p < 4; ++p) xo[p] = inject2(xo[p], el[p], es[p], a);
-        }
+        for (int p = 0; p < 4; ++p) xo[p] = inject2(xo[p], el[p], es[p], a);
     }
     // binary32 sum in rank order 0..P-1: own x' unquantized, others decoded
     uint32_t cwn[RB][CW], pwn[RB];
@@ -963,7 +960,6 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
         for (int p = 0; p < 4; ++p) yb[p] = bf16x2_rn(acc[p]);
         *reinterpret_cast<uint4*>(a.out[0] + j * GROUP + e0) = make_uint4(yb[0], yb[1], yb[2], yb[3]);
     }
-    if (!STATE) return;
     float2 el[4], es[4], nl[4], ns[4];
     load_f8_smem(els, e0, e0 + 4, el);
     load_f8_smem(ess, e0, e0 + 4, es);
@@ -1336,59 +1332,6 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
             __syncwarp();
             if (lead) mbar_arrive(&p.empty[s]);
         }
-    }
-    if (a.tail && blockIdx.x == gridDim.x - 1 && warp == 0) {
-        const long long j = a.G - 1;
-        const int o = (int)((j * a.P + a.P - 1) / a.G);
-        if (o >= a.rank_lo && o < a.rank_hi) reduce_range<GROUP, BITS, QM>(a, o, j, j + 1, 0, 1);
-    }
-}
-
-// The owners' pass of one rank of a multi-GPU call without feedback. It
-// moves only 800 bytes per owned group (x, P - 1 incoming payloads, the
-// gathered payload) against P - 1 decodes of every element, so it is bound by
-// instruction latency, not by HBM: this form runs three CTAs per SM (72
-// registers, 3-stage ring of 4-sub-tile stages) with 8 elements per lane, for
-// more warps in flight than k_reduce_tma's two CTAs of 16-element lanes.
-constexpr int kStagesRankNF = 3;
-constexpr int kRankNfBatch = 4;   // ranks whose payload loads are issued together (register budget)
-
-template <int GROUP, int BITS, int QM>
-__global__ void __launch_bounds__(kPipeThreads, 3) k_reduce_rank_nf(const Args a) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    constexpr int M = kReduceSubtilesNF, NS = kStagesRankNF;
-    const PipeShared p = pipe_shared<NS>(smem);
-    pipe_init<NS>(p);
-    const int warp = threadIdx.x >> 5;
-    RunWalker<GROUP, M, true, 1> walker(a);
-    if (warp == kConsumerWarps) {
-        if ((threadIdx.x & 31) == 0) produce<GROUP, M, NS, true, 1, GROUP * BITS / 8>(a, p, walker, false);
-        return;
-    }
-    constexpr int CW = BITS / 4, GPW = Lane<GROUP>::GPW;
-    constexpr int PASSES = M * kTileElems / (kConsumerWarps * 32 * 8);
-    const bool lead = (threadIdx.x & 31) == 0;
-    const int gi0 = warp * GPW + Lane<GROUP>().sub;
-    const int lt = Lane<GROUP>().t;
-    long long i = 0;
-    Tile t;
-    for (long long k = blockIdx.x; walker.locate(k, &t, a); k += gridDim.x, ++i) {
-        const int s = (int)(i % NS);
-        if (!mbar_wait(&p.full[s], (uint32_t)(i / NS) & 1u, a.wait_ns, p.abort)) {
-            if (lead) report_timeout(a, p);
-            return;
-        }
-        const uint8_t* stage = p.stages + (size_t)s * kStageBytes;
-#pragma unroll 1
-        for (int m = 0; m < PASSES; ++m) {
-            const int gi = gi0 + m * kConsumerWarps * GPW;
-            uint32_t cw[kRankNfBatch][CW], pw[kRankNfBatch];
-            load_payload8<GROUP, BITS, true, kRankNfBatch>(a, t.rank, t.j0 + gi, lt, gi < t.count, 0, cw, pw);
-            reduce_tile_group<GROUP, BITS, QM, true, false, false, kRankNfBatch>(a, stage, t, gi, gi < t.count, cw,
-                                                                                   pw);
-        }
-        __syncwarp();
-        if (lead) mbar_arrive(&p.empty[s]);
     }
     if (a.tail && blockIdx.x == gridDim.x - 1 && warp == 0) {
         const long long j = a.G - 1;

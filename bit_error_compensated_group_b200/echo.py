@@ -554,6 +554,8 @@ def exchange_chunk(plan: ExchangePlan, step: str, chunk: int, chunks: int, rank:
     for peer in range(P):
         if peer == rank:
             continue
+        # point-to-point ops name the peer by its global rank
+        dst = peer if group is None else dist.get_global_rank(group, peer)
         if step == "all_to_all":
             pieces = ((a2a_send[peer], a2a_recv[peer]),)
         elif step == "all_gather":
@@ -563,9 +565,9 @@ def exchange_chunk(plan: ExchangePlan, step: str, chunk: int, chunks: int, rank:
         for send, recv in pieces:
             for k in range(2):   # codes, then parameter words
                 if send[k].numel():
-                    ops.append(dist.P2POp(dist.isend, send[k], peer, group))
+                    ops.append(dist.P2POp(dist.isend, send[k], dst, group))
                 if recv[k].numel():
-                    ops.append(dist.P2POp(dist.irecv, recv[k], peer, group))
+                    ops.append(dist.P2POp(dist.irecv, recv[k], dst, group))
     if step == "all_gather":
         for k in range(2):
             if ag_send[k].numel():
@@ -590,6 +592,7 @@ class EchoRank:
         if quantizer != ECHO_QUANT_DIRECTED:
             echo_set_quantizer(self.handle, quantizer)
         self._plans = {}
+        self._comm_stream = None   # the chunked call's communication stream, made on first use
 
     def plan(self, bits: int) -> ExchangePlan:
         if bits not in self._plans:
@@ -623,9 +626,10 @@ class EchoRank:
         of the group calls this). chunks = 1: on torch's current stream, the
         collectives between the kernels. chunks > 1: the call in column
         chunks (see echo_rank_quantize_chunk), chunk c's exchanges on
-        `comm_stream` (a new stream if None) overlapping chunk c + 1's
-        kernels on the current stream, ordered by CUDA events; the current
-        stream continues once the last chunk is decoded."""
+        `comm_stream` (if None, a stream this handle creates once and keeps)
+        overlapping chunk c + 1's kernels on the current stream, ordered by
+        CUDA events; the current stream continues once the last chunk is
+        decoded."""
         fb = (eta, alpha_long, alpha_short, w)
         if chunks <= 1 or self.P == 1:
             self.quantize(x, bits, *fb)
@@ -637,6 +641,10 @@ class EchoRank:
                 self.decode(out, bits)
             return
         plan = self.plan(bits)
+        if comm_stream is None:
+            if self._comm_stream is None:
+                self._comm_stream = torch.cuda.Stream(device=self.workspace.device)
+            comm_stream = self._comm_stream
 
         def comm(step, c):
             for req in exchange_chunk(plan, step, c, chunks, self.rank, group):

@@ -116,3 +116,55 @@ def test_exchange_delivers_each_segment(world, n, group, bits, chunks):
     assert [g[0] for g in got] == list(range(world))
     for rank, bad, seg in got:
         assert bad == [], (rank, bad)
+
+
+def _subgroup_worker(rank, world, port, q):
+    """Ranks 2 and 3 of 4 form the Echo group; their chunked exchange names
+    peers by group rank and must reach the right global ranks."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bit_error_compensated_group_b200 as E
+    from datetime import timedelta
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        sub = dist.new_group([2, 3])
+        bad = []
+        if rank in (2, 3):
+            P, me, n, group, bits, chunks = 2, rank - 2, 777, 32, 4, 3
+            L = E.echo_query_rank_layout(n, P, me, group, 4, bits)
+            ws = torch.zeros(int(L.workspace_bytes), dtype=torch.uint8)
+            plan = E.ExchangePlan(ws, n, P, me, group, 4, bits)
+            G, cb = int(L.groups), int(L.code_bytes)
+            for j in range(G):
+                plan.send_codes[j * cb:(j + 1) * cb] = _tag_codes(me, j, cb).to(torch.uint8)
+                plan.send_params[j] = _tag_param(me, j)
+            seg, b0 = int(L.seg_groups), int(L.seg_begin)
+            for t in range(chunks):
+                for req in E.exchange_chunk(plan, "all_to_all", t, chunks, me, sub):
+                    req.wait()
+            other = 1 - me
+            for k in range(seg):
+                got = plan.recv_codes[(other * seg + k) * cb:(other * seg + k + 1) * cb].to(torch.int64)
+                if not torch.equal(got, _tag_codes(other, b0 + k, cb)):
+                    bad.append(("a2a codes", other, b0 + k))
+        dist.barrier()
+        q.put((rank, bad[:5]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_chunked_exchange_in_a_subgroup():
+    world = 4
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_subgroup_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+        assert p.exitcode == 0
+    got = sorted(q.get(timeout=5) for _ in range(world))
+    for rank, bad in got:
+        assert bad == [], (rank, bad)
