@@ -22,7 +22,11 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = [
     "-O3", "-lineinfo", "-std=c++17",
     "-fmad=false",                 # every float op below is an explicit _rn intrinsic anyway
-    "-split-compile", "0",         # optimize the kernel instantiations on all host cores
+    # no -split-compile: splitting the module for parallel optimization made
+    # the speed of most kernels depend on what else the module held (a change
+    # to the decoder alone moved the quantize pass by 1-12 %); compiled as one
+    # unit (about three minutes), builds that differ only in one kernel run
+    # the others at the same speed
     "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
     "-shared", "-cudart", "static",
 ]

@@ -1435,7 +1435,7 @@ __global__ void __launch_bounds__(kGatherThreads) k_gather_tma(const Args a) {
 // per CTA in shared memory (one thread per owner, then a warp scan).
 constexpr int kDecodeThreads = 256;
 constexpr int kDecodeUnroll = 8;
-constexpr bool kDecodePrefetch = false;   // next tile's loads before this tile's decode
+constexpr bool kDecodePrefetch = true;   // next tile's loads before this tile's decode
 constexpr int kDecodeElems = 16;
 
 __device__ __forceinline__ void store_v8_cs(void* p, uint4 lo, uint4 hi) {
