@@ -43,6 +43,12 @@ CASES = [
     (6, 70001, 64, 4, True, O.Q_INT_ZERO),
     (16, 50000, 128, 4, True, O.Q_DIRECTED),
     (64, 3 * 64 * 128 + 17, 128, 4, True, O.Q_DIRECTED),   # largest P
+    # without feedback, P <= 8: the owners' pass stages the received rows in shared memory
+    (2, 4096, 128, 4, False, O.Q_DIRECTED),
+    (3, 1000, 64, 8, False, O.Q_DIRECTED),
+    (8, 50000, 32, 4, False, O.Q_NEAREST),             # 64-group tiles
+    (5, 148 * 8 * 256 + 37, 256, 8, False, O.Q_INT_ZERO),
+    (16, 50000, 128, 4, False, O.Q_DIRECTED),          # P > 8: the rows are read from global memory
 ]
 
 
