@@ -28,6 +28,7 @@ import argparse
 import hashlib
 import json
 import os
+import queue
 import statistics
 import subprocess
 import sys
@@ -331,7 +332,19 @@ class OraclePool:
         for k in range(self.workers):
             lo, hi = k * self.cols // self.workers, (k + 1) * self.cols // self.workers
             self.tasks[k].put((lo, hi, self.j0, w.n, w.group, w.bits if bits is None else bits, fb))
-        got = [self.results.get(timeout=600) for _ in range(self.workers)]
+        got = []
+        deadline = time.monotonic() + 600
+        while len(got) < self.workers:
+            # a worker that died (e.g. at start-up) ends the run at once
+            # rather than after the whole time limit
+            try:
+                got.append(self.results.get(timeout=1.0))
+            except queue.Empty:
+                dead = [pr.exitcode for pr in self.procs if pr.exitcode is not None]
+                if dead:
+                    raise RuntimeError(f"oracle worker process exited with {dead}")
+                if time.monotonic() > deadline:
+                    raise TimeoutError("oracle workers gave no result within 600 s")
         dt = max(g[2] for g in got) - min(g[1] for g in got)
         er = w.P * self.cols * w.group
         return er * 2 / dt / 1e9, dt, er

@@ -580,6 +580,13 @@ __device__ __forceinline__ void store_f8_cs(float* p, const float2 v[4]) {
                  : "memory");
 }
 
+// 8 bf16 pairs to global memory in one 32-byte streaming store (p 32-byte aligned)
+__device__ __forceinline__ void store_v8_cs(void* p, uint4 lo, uint4 hi) {
+    asm volatile("st.global.cs.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(lo.x), "r"(lo.y),
+                 "r"(lo.z), "r"(lo.w), "r"(hi.x), "r"(hi.y), "r"(hi.z), "r"(hi.w)
+                 : "memory");
+}
+
 // ------------------------------------------------------------ quantize
 
 // One non-owned group of a tile with feedback (x, e_long, e_short staged):
@@ -847,11 +854,8 @@ __device__ __forceinline__ void load_payload8(const Args& a, int o, long long j,
 }
 
 // `cw0` / `pw0`: the first batch's payload words, already loaded by the
-// caller; later batches (P > RB) are loaded here -- with WIDE, each one
-// before the previous batch is decoded, so that its latency hides behind
-// that work (the registers it takes spill at P <= RB, which therefore runs
-// the instantiation without it).
-template <int GROUP, int BITS, int QM, bool RK, bool WIDE = false>
+// caller; later batches (P > RB) are loaded here.
+template <int GROUP, int BITS, int QM, bool RK>
 __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* st, const Tile& t, int gi,
                                                   bool act, const uint32_t (&cw0)[kReduceRankBatch][BITS / 4],
                                                   const uint32_t (&pw0)[kReduceRankBatch]) {
@@ -878,7 +882,6 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
         for (int p = 0; p < 4; ++p) xo[p] = inject2(xo[p], el[p], es[p], a);
     }
     // binary32 sum in rank order 0..P-1: own x' unquantized, others decoded
-    uint32_t cwn[RB][CW], pwn[RB];
     for (int r0 = 0; r0 < a.P; r0 += RB) {
         uint32_t cw[RB][CW];
         uint32_t pw[RB];
@@ -889,18 +892,9 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
 #pragma unroll
                 for (int c = 0; c < CW; ++c) cw[k][c] = cw0[k][c];
             }
-        } else if (WIDE) {
-#pragma unroll
-            for (int k = 0; k < RB; ++k) {
-                pw[k] = pwn[k];
-#pragma unroll
-                for (int c = 0; c < CW; ++c) cw[k][c] = cwn[k][c];
-            }
         } else {
             load_payload8<GROUP, BITS, RK, RB>(a, o, j, ln.t, act, r0, cw, pw);
         }
-        if (WIDE && r0 + RB < a.P)
-            load_payload8<GROUP, BITS, RK, RB>(a, o, j, ln.t, act, r0 + RB, cwn, pwn);
 #pragma unroll
         for (int k = 0; k < RB; ++k) {
             const int r = r0 + k;
@@ -1253,21 +1247,137 @@ __device__ __forceinline__ void reduce_tile_group_nf(const Args& a, const uint8_
     }
 }
 
+// One rank of a multi-GPU call without feedback: 16 consecutive elements per
+// lane, so that a received row's codes for them are one 8-byte load (16 bytes
+// at 8 bits) and the gather payload's one store (against two 4-byte ones with
+// chunks t and t + L: 0.191 -> 0.172 ms on the 1 GB P = 8 message, A/B on one
+// box; the simulation's pass, with its P output stores, ran 1.97 -> 2.21 ms
+// in this layout and keeps the other). Lanes of a group past the tile's end
+// load the tile's last group (every address stays inside the received rows,
+// this rank's own unused row included) and store nothing, so the loads need
+// no predicate. The sum starts from zeros only to keep the register
+// allocator from spilling (every element's first term replaces it).
+template <int GROUP, int BITS, int QM>
+__device__ __forceinline__ void reduce_tile_group_nf_rank(const Args& a, const uint8_t* st, const Tile& t, int gi,
+                                                          bool act) {
+    using LN = Lane16<GROUP>;
+    constexpr int L = LN::L, Q = (1 << BITS) - 1, CB = GROUP * BITS / 8;
+    constexpr int RB = BITS == 4 ? 8 : 4;   // ranks whose payload loads are issued together
+    constexpr int CW = BITS / 2;            // 32-bit code words per 16 elements
+    const LN ln;
+    const int o = t.rank;
+    const long long j = t.j0 + gi;
+    const long long jl = t.j0 + min(gi, t.count - 1);
+    const uint4* xs = reinterpret_cast<const uint4*>(st + (size_t)gi * GROUP * 2) + 2 * ln.t;
+    const uint4 xw[2] = {xs[0], xs[1]};
+    float2 acc[8];
+#pragma unroll
+    for (int p = 0; p < 8; ++p) acc[p] = make_float2(0.0f, 0.0f);
+    // binary32 sum in rank order 0..P-1: own x unquantized, others decoded
+    for (int r0 = 0; r0 < a.P; r0 += RB) {
+        uint32_t cw[RB][CW];
+        uint32_t pw[RB];
+#pragma unroll
+        for (int k = 0; k < RB; ++k) {
+            const size_t slot = a2a_slot(a, min(r0 + k, a.P - 1), jl);
+            const uint8_t* codes = a.a2a_codes + slot * CB + 4 * CW * ln.t;
+            if (BITS == 4) {
+                const uint2 v = *reinterpret_cast<const uint2*>(codes);
+                cw[k][0] = v.x;
+                cw[k][1] = v.y;
+            } else {
+                const uint4 v = *reinterpret_cast<const uint4*>(codes);
+                cw[k][0] = v.x;
+                cw[k][1] = v.y;
+                cw[k][2] = v.z;
+                cw[k][3] = v.w;
+            }
+            pw[k] = a.a2a_params[slot];
+        }
+#pragma unroll
+        for (int k = 0; k < RB; ++k) {
+            const int r = r0 + k;
+            if (r >= a.P) break;
+            float2 term[8];
+            if (r == o) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    term[4 * h] = bf16_pair(xw[h].x);
+                    term[4 * h + 1] = bf16_pair(xw[h].y);
+                    term[4 * h + 2] = bf16_pair(xw[h].z);
+                    term[4 * h + 3] = bf16_pair(xw[h].w);
+                }
+            } else {
+                const float sk = param_s(pw[k]);
+                const float2 s2 = splat(sk);
+                const float2 z2 = splat(param_zf<QM>(pw[k], sk));
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    float2 q[4];
+                    unpack_codes8<BITS>(&cw[k][h * CW / 2], q);
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) term[4 * h + p] = fma2_rn(q[p], s2, z2);
+                }
+            }
+#pragma unroll
+            for (int p = 0; p < 8; ++p) acc[p] = (r == 0) ? term[p] : add2_rn(acc[p], term[p]);
+        }
+    }
+    float lmin = __int_as_float(0x7f800000), lmax = -__int_as_float(0x7f800000);
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+        lmin = nan_min3(lmin, acc[p].x, acc[p].y);
+        lmax = nan_max3(lmax, acc[p].x, acc[p].y);
+    }
+    if (a.P >= 2) {
+        const GridP g = make_grid_p<L, Q, QM>(lmin, lmax);
+        raise_flags(a, act && g.bad);
+        if (!act) return;
+        uint8_t* codes = a.g_codes + (size_t)(j - a.g_col_base) * CB + 4 * CW * ln.t;
+        uint2 pk[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float2 e[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) e[p] = encode2<QM, Q>(acc[4 * h + p], g, a);
+            pk[h] = pack_codes8<BITS>(e);
+        }
+        if (BITS == 4) *reinterpret_cast<uint2*>(codes) = make_uint2(pk[0].x, pk[1].x);
+        else *reinterpret_cast<uint4*>(codes) = make_uint4(pk[0].x, pk[0].y, pk[1].x, pk[1].y);
+        if (ln.t == 0) a.g_params[j - a.g_col_base] = g.param;
+    } else {
+        // a single rank sends nothing: its output is its own x
+        raise_flags(a, act && !(lmin >= -65504.0f && lmax <= 65504.0f));
+        if (!act) return;
+        uint32_t yw[8];
+#pragma unroll
+        for (int p = 0; p < 8; ++p) yw[p] = bf16x2_rn(acc[p]);
+        uint4* y = reinterpret_cast<uint4*>(a.out[o] + j * GROUP) + 2 * ln.t;
+        y[0] = make_uint4(yw[0], yw[1], yw[2], yw[3]);
+        y[1] = make_uint4(yw[4], yw[5], yw[6], yw[7]);
+    }
+}
+
 // Two CTAs of kPipeThreads per SM: 96 registers per thread (each SM
 // sub-partition's 16384 registers then hold its share of the 18 warps).
-// WIDE (the simulation with feedback and P > kReduceRankBatch): pipelined
-// payload batches, see reduce_tile_group.
+// WIDE: the simulation with feedback and P > kReduceRankBatch.
 template <int GROUP, int BITS, bool FB, int QM, bool RK = false, bool WIDE = false>
 __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
     extern __shared__ __align__(128) uint8_t smem[];
     constexpr int M = FB ? 1 : kReduceSubtilesNF;
     constexpr int NS = FB ? kStagesReduceFB : kStagesReduceNF;
-    // One rank of a multi-GPU call with feedback: 16 elements per lane, the
-    // two halves of the consumer warps taking alternate tiles (each stage is
-    // released by one half). The simulation with feedback: 8 elements per
-    // lane, all consumer warps on every tile. Without feedback: 16 elements
-    // per lane, two passes of all warps over a 4-sub-tile stage.
-    constexpr bool HALVES = FB && RK;
+    // One rank of a multi-GPU call with feedback, and the simulation with
+    // feedback at P > kReduceRankBatch: 16 elements per lane, the two halves
+    // of the consumer warps taking alternate tiles (each stage is released by
+    // one half), so that the per-group work of each incoming payload (its
+    // parameter word, its slot address) serves twice the elements. The
+    // simulation with feedback at P <= kReduceRankBatch: 8 elements per lane,
+    // all consumer warps on every tile (the halves measured 2.6 % slower
+    // there; at P = 16 they took the pass from 2.85 to 2.77 ms, 85.6 ->
+    // 88.1 % of its roofline on 512 MB per rank, A/B on one box). Without
+    // feedback: 16 elements per lane, two passes of all warps over a
+    // 4-sub-tile stage.
+    constexpr bool HALVES = FB && (RK || WIDE);
     const PipeShared p = pipe_shared<NS>(smem);
     pipe_init<NS>(p, HALVES ? kConsumerWarps / 2 : kConsumerWarps);
     const int warp = threadIdx.x >> 5;
@@ -1283,10 +1393,10 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
     griddep_wait();
     const bool lead = (threadIdx.x & 31) == 0;
     Tile t;
-    if (FB && !RK) {
-        // The simulation: 8 elements per lane, the first payload batch loaded
-        // once the tile is staged (issuing it before the wait measured 1-2 %
-        // slower)
+    if (FB && !HALVES) {
+        // The simulation at P <= kReduceRankBatch: 8 elements per lane, the
+        // first payload batch loaded once the tile is staged (issuing it
+        // before the wait measured 1-2 % slower)
         constexpr int CW = BITS / 4;
         const int gi = warp * Lane<GROUP>::GPW + Lane<GROUP>().sub;
         const int lt = Lane<GROUP>().t;
@@ -1299,8 +1409,8 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
             }
             uint32_t cw[kReduceRankBatch][CW], pw[kReduceRankBatch];
             load_payload8<GROUP, BITS, RK, kReduceRankBatch>(a, t.rank, t.j0 + gi, lt, gi < t.count, 0, cw, pw);
-            reduce_tile_group<GROUP, BITS, QM, RK, WIDE>(a, p.stages + (size_t)s * kStageBytes, t, gi, gi < t.count,
-                                                         cw, pw);
+            reduce_tile_group<GROUP, BITS, QM, RK>(a, p.stages + (size_t)s * kStageBytes, t, gi, gi < t.count, cw,
+                                                   pw);
             __syncwarp();
             if (lead) mbar_arrive(&p.empty[s]);
         }
@@ -1326,7 +1436,10 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_reduce_tma(const Args a) {
 #pragma unroll 1
                 for (int m = 0; m < PASSES; ++m) {
                     const int g = gi + m * kConsumerWarps * GPW;
-                    reduce_tile_group_nf<GROUP, BITS, QM, RK>(a, stage, t, g, g < t.count);
+                    if (RK)
+                        reduce_tile_group_nf_rank<GROUP, BITS, QM>(a, stage, t, g, g < t.count);
+                    else
+                        reduce_tile_group_nf<GROUP, BITS, QM, false>(a, stage, t, g, g < t.count);
                 }
             }
             __syncwarp();
@@ -1438,11 +1551,6 @@ constexpr int kDecodeUnroll = 8;
 constexpr bool kDecodePrefetch = true;   // next tile's loads before this tile's decode
 constexpr int kDecodeElems = 16;
 
-__device__ __forceinline__ void store_v8_cs(void* p, uint4 lo, uint4 hi) {
-    asm volatile("st.global.cs.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(lo.x), "r"(lo.y),
-                 "r"(lo.z), "r"(lo.w), "r"(hi.x), "r"(hi.y), "r"(hi.z), "r"(hi.w)
-                 : "memory");
-}
 
 // 16 consecutive codes of a group: 8 bytes at 4 bits (x, y), 16 at 8 bits
 template <int BITS>
