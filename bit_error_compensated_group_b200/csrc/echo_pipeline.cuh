@@ -942,9 +942,11 @@ __device__ __forceinline__ void reduce_tile_group(const Args& a, const uint8_t* 
         if (ln.t == 0) a.g_params[j - a.g_col_base] = g.param;
         if (a.write_outputs) {
             // phase 4 in the owner's pass: every rank's output gets the decoded
-            // requantized sum -- the same bits a decode of the gathered payload gives
+            // requantized sum -- the same bits a decode of the gathered payload
+            // gives. Plain stores: with the evict-first hint the pass ran
+            // 3.49 ms against 3.45 (A/B on one box)
             const uint4 y4 = make_uint4(yb[0], yb[1], yb[2], yb[3]);
-            for (int r = 0; r < a.P; ++r) __stcs(reinterpret_cast<uint4*>(a.out[r] + j * GROUP + e0), y4);
+            for (int r = 0; r < a.P; ++r) *reinterpret_cast<uint4*>(a.out[r] + j * GROUP + e0) = y4;
         }
     } else {
         // a single rank sends nothing: its output is its own x'
@@ -1085,11 +1087,12 @@ __device__ __forceinline__ void reduce_tile_group16(const Args& a, const uint8_t
         if (ln.t == 0) a.g_params[j - a.g_col_base] = g.param;
         if (a.write_outputs) {
             // phase 4 in the owner's pass: every rank's output gets the decoded
-            // requantized sum -- the same bits a decode of the gathered payload gives
+            // requantized sum -- the same bits a decode of the gathered payload
+            // gives (plain stores, as in the 8-element pass)
             for (int r = 0; r < a.P; ++r) {
                 uint16_t* y = a.out[r] + j * GROUP;
-                __stcs(reinterpret_cast<uint4*>(y + 8 * ln.chunk(0)), make_uint4(yb[0], yb[1], yb[2], yb[3]));
-                __stcs(reinterpret_cast<uint4*>(y + 8 * ln.chunk(1)), make_uint4(yb[4], yb[5], yb[6], yb[7]));
+                *reinterpret_cast<uint4*>(y + 8 * ln.chunk(0)) = make_uint4(yb[0], yb[1], yb[2], yb[3]);
+                *reinterpret_cast<uint4*>(y + 8 * ln.chunk(1)) = make_uint4(yb[4], yb[5], yb[6], yb[7]);
             }
         }
     } else {
@@ -1228,11 +1231,12 @@ __device__ __forceinline__ void reduce_tile_group_nf(const Args& a, const uint8_
         if (ln.t == 0) a.g_params[j - a.g_col_base] = g.param;
         if (a.write_outputs) {
             // phase 4 in the owner's pass: every rank's output gets the decoded
-            // requantized sum -- the same bits a decode of the gathered payload gives
+            // requantized sum -- the same bits a decode of the gathered payload
+            // gives (plain stores, as in the 8-element pass)
             for (int r = 0; r < a.P; ++r) {
                 uint16_t* y = a.out[r] + j * GROUP;
-                __stcs(reinterpret_cast<uint4*>(y + 8 * ln.chunk(0)), make_uint4(yw[0], yw[1], yw[2], yw[3]));
-                __stcs(reinterpret_cast<uint4*>(y + 8 * ln.chunk(1)), make_uint4(yw[4], yw[5], yw[6], yw[7]));
+                *reinterpret_cast<uint4*>(y + 8 * ln.chunk(0)) = make_uint4(yw[0], yw[1], yw[2], yw[3]);
+                *reinterpret_cast<uint4*>(y + 8 * ln.chunk(1)) = make_uint4(yw[4], yw[5], yw[6], yw[7]);
             }
         }
     } else {
@@ -1255,7 +1259,9 @@ __device__ __forceinline__ void reduce_tile_group_nf(const Args& a, const uint8_
 // in this layout and keeps the other). Lanes of a group past the tile's end
 // load the tile's last group (every address stays inside the received rows,
 // this rank's own unused row included) and store nothing, so the loads need
-// no predicate. The sum starts from zeros only to keep the register
+// no predicate. The own x is read from the staged tile when its turn in the
+// rank order comes rather than held in registers through the sum (0.171 ->
+// 0.162 ms), and the sum starts from zeros only to keep the register
 // allocator from spilling (every element's first term replaces it).
 template <int GROUP, int BITS, int QM>
 __device__ __forceinline__ void reduce_tile_group_nf_rank(const Args& a, const uint8_t* st, const Tile& t, int gi,
@@ -1269,7 +1275,6 @@ __device__ __forceinline__ void reduce_tile_group_nf_rank(const Args& a, const u
     const long long j = t.j0 + gi;
     const long long jl = t.j0 + min(gi, t.count - 1);
     const uint4* xs = reinterpret_cast<const uint4*>(st + (size_t)gi * GROUP * 2) + 2 * ln.t;
-    const uint4 xw[2] = {xs[0], xs[1]};
     float2 acc[8];
 #pragma unroll
     for (int p = 0; p < 8; ++p) acc[p] = make_float2(0.0f, 0.0f);
@@ -1302,10 +1307,11 @@ __device__ __forceinline__ void reduce_tile_group_nf_rank(const Args& a, const u
             if (r == o) {
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    term[4 * h] = bf16_pair(xw[h].x);
-                    term[4 * h + 1] = bf16_pair(xw[h].y);
-                    term[4 * h + 2] = bf16_pair(xw[h].z);
-                    term[4 * h + 3] = bf16_pair(xw[h].w);
+                    const uint4 xh = xs[h];   // read when its turn comes: no registers held through the sum
+                    term[4 * h] = bf16_pair(xh.x);
+                    term[4 * h + 1] = bf16_pair(xh.y);
+                    term[4 * h + 2] = bf16_pair(xh.z);
+                    term[4 * h + 3] = bf16_pair(xh.w);
                 }
             } else {
                 const float sk = param_s(pw[k]);
