@@ -1170,6 +1170,60 @@ def run_dist(args):
     dist.destroy_process_group()
 
 
+def run_shapes(args):
+    """The owners' pass and the quantize pass across P (and group sizes and
+    widths): 2^28 N(0,1) elements per rank (512 MB), feedback on, through the
+    phase entry points with an event between the two kernels; each kernel's
+    fraction of the measured copy peak for its own algorithmic bytes."""
+    import torch
+    import bit_error_compensated_group_b200 as E
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    peak, _ = _peak_hbm()
+    n = 1 << 28
+    fb = (1.0, 0.05, 0.5, 0.5)
+    out = []
+    for P, group, bits in [(2, 128, 4), (4, 128, 4), (8, 128, 4), (16, 128, 4), (8, 32, 4), (8, 256, 4),
+                           (8, 128, 8)]:
+        g = torch.Generator(device=dev)
+        g.manual_seed(5)
+        inputs = [torch.randn(n, generator=g, device=dev).to(torch.bfloat16) for _ in range(P)]
+        outputs = [torch.empty_like(t) for t in inputs]
+        ar = E.EchoAllReduce(n, P, group, bits, True)
+        try:
+            def step(evs=None):
+                if evs is not None:
+                    evs[0].record(stream)
+                E.echo_phase_quantize(inputs, ar.handle, bits, *fb, stream=stream)
+                if evs is not None:
+                    evs[1].record(stream)
+                E.echo_phase_reduce(inputs, outputs, ar.handle, bits, *fb, stream=stream)
+                if evs is not None:
+                    evs[2].record(stream)
+            for _ in range(args.warmup):
+                step()
+            torch.cuda.synchronize(dev)
+            evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+            for e in evs:
+                step(e)
+            torch.cuda.synchronize(dev)
+            rc, flags = ar.status()
+        finally:
+            ar.close()
+        q = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+        r = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+        ab = algorithmic_bytes(P, n, group, bits)
+        out.append({"P": P, "group": group, "bits": bits, "quantize_ms": q, "reduce_ms": r, "call_ms": q + r,
+                    "call_frac": ab["total"] / ((q + r) * 1e-3) / 1e9 / peak,
+                    "quantize_frac": ab["quantize"] / (q * 1e-3) / 1e9 / peak,
+                    "reduce_frac": ab["reduce_gather"] / (r * 1e-3) / 1e9 / peak, "status": rc, "flags": flags})
+        del inputs, outputs
+        torch.cuda.empty_cache()
+    print(json.dumps({"shapes": out, "elements_per_rank": n, "steps": args.steps, "warmup": args.warmup,
+                      "peak_gbs": peak}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -1189,6 +1243,9 @@ def main():
                     help="under torchrun: the multi-GPU call (P = world size) against NCCL's bf16 all-reduce")
     ap.add_argument("--ranks", action="store_true",
                     help="print one rank's kernel times of a multi-GPU call (rank 0 of P = 8, 1 GB) instead")
+    ap.add_argument("--shapes", action="store_true",
+                    help="print each kernel's time and roofline fraction across P, group size and width "
+                         "(512 MB per rank) instead")
     ap.add_argument("--workloads", action="store_true",
                     help="print every workload's GPU and oracle time per call instead of the main line")
     ap.add_argument("--background", default=None,
@@ -1210,6 +1267,8 @@ def main():
         run_ablation(args)
     elif args.workloads:
         run_workloads(args)
+    elif args.shapes:
+        run_shapes(args)
     elif args.ranks:
         run_ranks(args)
     elif args.background is not None:

@@ -87,3 +87,17 @@ def test_background_study_line():
         assert len(bg[key]) == 3 and all(v > 0 for v in bg[key][1:]), key
     assert bg["echo_slowdown"][0] == 1.0 and bg["background_alone"][0] == 0.0
     assert bg["background_alone"][2] > bg["background_alone"][1] > 0
+
+
+@pytest.mark.gpu
+def test_shapes_line():
+    out = subprocess.run([sys.executable, "bench.py", "--shapes", "--steps", "2", "--warmup", "1"], cwd=ROOT,
+                         capture_output=True, text=True, timeout=900, check=True).stdout
+    shapes = _last_json(out)["shapes"]
+    assert [(s["P"], s["group"], s["bits"]) for s in shapes][:4] == [(2, 128, 4), (4, 128, 4), (8, 128, 4),
+                                                                     (16, 128, 4)]
+    for s in shapes:
+        assert s["status"] == 0 and s["flags"] == 0
+        assert s["quantize_ms"] > 0 and s["reduce_ms"] > 0
+        assert s["call_ms"] == pytest.approx(s["quantize_ms"] + s["reduce_ms"])
+        assert 0 < s["reduce_frac"] < 1.5 and 0 < s["quantize_frac"] < 1.5
