@@ -1528,11 +1528,14 @@ __global__ void __launch_bounds__(kGatherThreads) k_gather_tma(const Args a) {
 
 // Phase 4 on one rank of a multi-GPU call: every group of the gathered
 // payload (P owner segments, each padded to g_seg_stride groups) decoded into
-// this rank's output (a.out[a.out_lo]). With a single output there is no tile to share between
-// stores, so each thread decodes E-element chunks straight from registers:
-// the loads of U chunks (one code load and the parameter word each) are
-// issued together, then each chunk leaves in one 32-byte streaming store
-// (16-byte stores when the output is not 32-byte aligned).
+// this rank's output (a.out[a.out_lo]). With a single output there is no
+// tile to share between stores, so each thread decodes E-element chunks
+// straight from registers: the loads of U chunks (one code load and the
+// parameter word each) are issued together, then each 16 elements of a chunk
+// leave in one 32-byte streaming store (16-byte stores when the output is not
+// 32-byte aligned). 32-element chunks (one 16-byte code load at 4 bits) ran
+// the 1 GB P = 8 decode in 0.233-0.235 ms against 0.239 with 16-element ones
+// (A/B on one box).
 //
 // Work layout: owner o's run is its segment (in a chunked call, the chunk's
 // part of it) clipped to the call's full-group window; a run is cut into
@@ -1545,25 +1548,42 @@ __global__ void __launch_bounds__(kGatherThreads) k_gather_tma(const Args a) {
 constexpr int kDecodeThreads = 256;
 constexpr int kDecodeUnroll = 8;
 constexpr bool kDecodePrefetch = true;   // next tile's loads before this tile's decode
-constexpr int kDecodeElems = 16;
+constexpr int kDecodeElems = 32;   // elements per chunk (16 or 32); kDecodeUnroll counts 16-element chunks
 
-
-// 16 consecutive codes of a group: 8 bytes at 4 bits (x, y), 16 at 8 bits
-template <int BITS>
-__device__ __forceinline__ uint4 load_codes16(const uint8_t* p) {
-    if (BITS == 4) {
-        const uint2 v = *reinterpret_cast<const uint2*>(p);
-        return make_uint4(v.x, v.y, 0u, 0u);
+// E consecutive codes of a group: E * BITS / 32 words (8, 16 or 32 bytes)
+template <int E, int BITS>
+struct ChunkCodes {
+    static constexpr int W = E * BITS / 32;
+    uint32_t w[W];
+    __device__ __forceinline__ void load(const uint8_t* p) {
+        if (W == 2) {
+            const uint2 v = *reinterpret_cast<const uint2*>(p);
+            w[0] = v.x;
+            w[1] = v.y;
+        } else {
+#pragma unroll
+            for (int q = 0; q < W / 4; ++q) {
+                const uint4 v = reinterpret_cast<const uint4*>(p)[q];
+                w[4 * q] = v.x;
+                w[4 * q + 1] = v.y;
+                w[4 * q + 2] = v.z;
+                w[4 * q + 3] = v.w;
+            }
+        }
     }
-    return *reinterpret_cast<const uint4*>(p);
-}
+    // the words of 8-element part k (one at 4 bits, two at 8)
+    __device__ __forceinline__ uint2 part(int k) const {
+        return BITS == 4 ? make_uint2(w[k], 0u) : make_uint2(w[2 * k], w[2 * k + 1]);
+    }
+};
 
 template <int GROUP, int BITS, int QM>
 __global__ void __launch_bounds__(kDecodeThreads) k_decode_rank(const Args a) {
-    constexpr int E = kDecodeElems, L = GROUP / E, CB = GROUP * BITS / 8, U = kDecodeUnroll;
+    constexpr int E = kDecodeElems, L = GROUP / E, CB = GROUP * BITS / 8, U = kDecodeUnroll * 16 / E;
     constexpr int CHUNK_BYTES = E * BITS / 8;
     constexpr int TG = U * kDecodeThreads / L;   // groups per tile
-    static_assert(E == 16 && GROUP % E == 0, "16-element chunks");
+    static_assert((E == 16 || E == 32) && GROUP % E == 0, "16- or 32-element chunks");
+    using Codes = ChunkCodes<E, BITS>;
     static_assert(ECHO_MAX_RANKS <= 64, "one warp scans the owners' tile counts");
     __shared__ long long run_b[ECHO_MAX_RANKS], run_e[ECHO_MAX_RANKS], run_slot[ECHO_MAX_RANKS];
     __shared__ long long tile_pre[ECHO_MAX_RANKS + 1];
@@ -1616,25 +1636,26 @@ __global__ void __launch_bounds__(kDecodeThreads) k_decode_rank(const Args a) {
         r.params = a.g_params + (run_slot[o] + off);
         r.y = out + j0 * GROUP;
     };
-    auto load = [&](const TileRef& r, uint4 (&w)[U], uint32_t (&pw)[U]) {
+    auto load = [&](const TileRef& r, Codes (&w)[U], uint32_t (&pw)[U]) {
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int lc = u * kDecodeThreads + tid;
             if (lc < r.nchunks) {
-                w[u] = load_codes16<BITS>(r.codes + lc * CHUNK_BYTES);
+                w[u].load(r.codes + lc * CHUNK_BYTES);
                 pw[u] = r.params[lc / L];
             }
         }
     };
-    auto decode_store = [&](const TileRef& r, const uint4 (&w)[U], const uint32_t (&pw)[U]) {
+    auto decode_store = [&](const TileRef& r, const Codes (&w)[U], const uint32_t (&pw)[U]) {
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int lc = u * kDecodeThreads + tid;
-            if (lc < r.nchunks) {
-                const uint4 y0 = decode8_bf16<BITS, QM>(make_uint2(w[u].x, BITS == 4 ? 0u : w[u].y), pw[u]);
-                const uint4 y1 = decode8_bf16<BITS, QM>(BITS == 4 ? make_uint2(w[u].y, 0u) : make_uint2(w[u].z, w[u].w),
-                                                        pw[u]);
-                uint16_t* dst = r.y + lc * E;
+#pragma unroll
+            for (int m = 0; m < E / 16; ++m) {
+                if (lc >= r.nchunks) break;
+                const uint4 y0 = decode8_bf16<BITS, QM>(w[u].part(2 * m), pw[u]);
+                const uint4 y1 = decode8_bf16<BITS, QM>(w[u].part(2 * m + 1), pw[u]);
+                uint16_t* dst = r.y + lc * E + 16 * m;
                 if (v8) {
                     store_v8_cs(dst, y0, y1);
                 } else {
@@ -1648,7 +1669,7 @@ __global__ void __launch_bounds__(kDecodeThreads) k_decode_rank(const Args a) {
         // the next tile's loads are issued before this tile is decoded
         long long k = blockIdx.x;
         TileRef cur = {0, nullptr, nullptr, nullptr};
-        uint4 w[U];
+        Codes w[U];
         uint32_t pw[U];
         if (k < ntiles) {
             locate(k, cur);
@@ -1657,7 +1678,7 @@ __global__ void __launch_bounds__(kDecodeThreads) k_decode_rank(const Args a) {
         while (k < ntiles) {
             const long long kn = k + gridDim.x;
             TileRef nxt = {0, nullptr, nullptr, nullptr};
-            uint4 wn[U];
+            Codes wn[U];
             uint32_t pwn[U];
             if (kn < ntiles) {
                 locate(kn, nxt);
@@ -1676,7 +1697,7 @@ __global__ void __launch_bounds__(kDecodeThreads) k_decode_rank(const Args a) {
         for (long long k = blockIdx.x; k < ntiles; k += gridDim.x) {
             TileRef cur;
             locate(k, cur);
-            uint4 w[U];
+            Codes w[U];
             uint32_t pw[U];
             load(cur, w, pw);
             decode_store(cur, w, pw);
