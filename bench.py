@@ -321,6 +321,7 @@ class OraclePool:
         self.procs = [ctx.Process(target=_oracle_worker, daemon=True,
                                   args=(k, self.shm.name, (w.P, m), self.barrier, self.tasks[k], self.results))
                       for k in range(workers)]
+        self.broken = False
         for pr in self.procs:
             pr.start()
 
@@ -342,18 +343,27 @@ class OraclePool:
             except queue.Empty:
                 dead = [pr.exitcode for pr in self.procs if pr.exitcode is not None]
                 if dead:
+                    self.broken = True
                     raise RuntimeError(f"oracle worker process exited with {dead}")
                 if time.monotonic() > deadline:
+                    self.broken = True
                     raise TimeoutError("oracle workers gave no result within 600 s")
         dt = max(g[2] for g in got) - min(g[1] for g in got)
         er = w.P * self.cols * w.group
         return er * 2 / dt / 1e9, dt, er
 
     def close(self):
-        for q in self.tasks:
-            q.put(None)
+        # after a failed pass the survivors may be waiting at the barrier:
+        # end them at once; otherwise let every worker leave its loop
+        if not self.broken:
+            for q in self.tasks:
+                q.put(None)
+            for pr in self.procs:
+                pr.join(timeout=30)
         for pr in self.procs:
-            pr.join(timeout=30)
+            if pr.is_alive():
+                pr.terminate()
+                pr.join(timeout=10)
         self.shm.close()
         self.shm.unlink()
 

@@ -101,3 +101,37 @@ def test_shapes_line():
         assert s["quantize_ms"] > 0 and s["reduce_ms"] > 0
         assert s["call_ms"] == pytest.approx(s["quantize_ms"] + s["reduce_ms"])
         assert 0 < s["reduce_frac"] < 1.5 and 0 < s["quantize_frac"] < 1.5
+
+
+def test_oracle_pool_fails_fast_when_a_worker_dies():
+    """A worker process that is gone (killed, or crashed at start-up) ends the
+    pass with an error within seconds instead of the pool's 600 s limit, and
+    closing the pool does not wait on the survivors."""
+    import time
+    sys.path.insert(0, ROOT)
+    import bench
+    pool = bench.OraclePool(2, 64)
+    try:
+        pool.procs[0].terminate()
+        pool.procs[0].join(timeout=30)
+        t0 = time.monotonic()
+        with pytest.raises(RuntimeError, match="exited"):
+            pool.run()
+        assert time.monotonic() - t0 < 60
+    finally:
+        t1 = time.monotonic()
+        pool.close()
+        assert time.monotonic() - t1 < 30
+    assert not any(pr.is_alive() for pr in pool.procs)
+
+
+def test_oracle_pool_pass():
+    sys.path.insert(0, ROOT)
+    import bench
+    pool = bench.OraclePool(2, 64)
+    try:
+        gbs, dt, er = pool.run()
+    finally:
+        pool.close()
+    assert gbs > 0 and dt > 0 and er == pool.w.P * 64 * pool.w.group
+    assert not any(pr.is_alive() for pr in pool.procs)
