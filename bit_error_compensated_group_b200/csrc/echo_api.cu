@@ -184,6 +184,8 @@ int launch_stage(Stage stage, const echo_dev::Args& a, const echo_state* st, cud
                 rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, false, QM, true>, grid, tiles, a, st, s,
                                  echo_dev::pipe_smem(echo_dev::kStagesReduceNF), pdl);
             } else if (a.state && a.P > echo_dev::kReduceRankBatch) {
+                // more incoming payloads than one load batch: 16 elements per
+                // lane, the consumer halves taking alternate tiles
                 static int grid[kMaxDevices];
                 rc = launch_pipe(echo_dev::k_reduce_tma<GROUP, BITS, true, QM, false, true>, grid, tiles, a, st, s,
                                  echo_dev::pipe_smem(echo_dev::kStagesReduceFB), pdl);
